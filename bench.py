@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of one LSH-sampled decode layer-step (MagicPIG hot path) on B200.
+
+A step = every row of the hot path over one batch of synthetic input:
+  mp_hash_keys   SimHash of every cached key (tcgen05-free SIMT or tensor-core
+                 hash, see the roofline "bound"),
+  mp_append_token  one new token per sequence (K/V row + codes, length + 1),
+  mp_decode_attend query hash, collision scan + compaction, sampled attention
+                 with the -log u correction, exact sink/window set, LSE merge.
+Metric: decode context tokens scanned per second per layer-step
+(sum over sequences of the post-append length, divided by the step time).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One process per GPU (torchrun for N > 1): every rank runs an independent
+replica with its own seed (no collective on the data path), so `value` is the
+sum over ranks of the tokens scanned divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "llama8b_16k"
+FLUSH_BYTES = 256 << 20  # > 126 MB L2
+METRIC = "decode context-tokens scanned/s per layer-step"
+HASH_IMPL = "simt-fp32"   # implementation of mp_hash_keys in this build
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    sm_max_mhz=float(d.get("sm_max_mhz", 1965.0)), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
+
+
+def workload_for_rank(name, rank):
+    import workloads
+    w = workloads.get(name)
+    return w.with_(seed=w.seed + 7919 * rank) if rank else w
+
+
+def step_tokens(lens_after):
+    return int(np.sum(lens_after))
+
+
+# ------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smmax=float(f[2]), reasons=[
+                    n for n, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                       "sw_power_cap"), f[5:9]) if v.lower() == "active"]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = sorted({r for row in rows for r in row["reasons"]})
+        return dict(sm_mhz=statistics.median(r["sm"] for r in rows), sm_max_mhz=max(r["smmax"] for r in rows),
+                    reasons=reasons, samples=len(rows))
+
+
+# --------------------------------------------------------- our arm ----
+
+class Bench:
+    def __init__(self, w, device):
+        import torch
+        import lsh_sampled_sparse_simhash_b200 as mp
+        from workloads import make_inputs
+        self.mp, self.torch, self.w = mp, torch, w
+        inp = make_inputs(w)
+        self.inp = inp
+        self.shape = mp.Shape(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.capacity, w.k_bits,
+                              w.n_tables, w.sink, w.window)
+
+        def dev(a):
+            return torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a)).to(device)
+
+        self.W, self.q, self.K, self.V = dev(inp["W"]), dev(inp["q"]), dev(inp["K"]), dev(inp["V"])
+        self.k_new, self.v_new = dev(inp["k_new"]), dev(inp["v_new"])
+        self.lens0 = dev(inp["seq_lens"].astype(np.int32))
+        self.lens = self.lens0.clone()
+        self.prefill = int(inp["seq_lens"].max())
+        self.max_len = self.prefill + 1
+        kind, cshape = mp.codes_shape(self.shape)
+        self.codes = torch.zeros(cshape, dtype=torch.uint8 if kind == "uint8" else torch.int32, device=device)
+        self.ws = torch.empty(mp.decode_workspace_bytes(self.shape, self.max_len), dtype=torch.uint8, device=device)
+        B, Hq, d = w.batch, w.n_q_heads, w.head_dim
+        self.out = torch.empty((B, Hq, d), dtype=torch.float32, device=device)
+        self.lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
+        self.ns = torch.empty((B, Hq), dtype=torch.int32, device=device)
+        self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.tokens = step_tokens(inp["seq_lens"] + 1)
+        self.launches_per_step = 7  # hash 1, append 2, decode 4 (qhash, scan, attend, merge)
+
+    def hash(self):
+        self.mp.hash_keys(self.shape, self.K, self.W, self.prefill, self.codes, seq_lens=self.lens0)
+
+    def append(self):
+        self.mp.append_token(self.shape, self.k_new, self.v_new, self.W, self.K, self.V, self.codes, self.lens)
+
+    def decode(self):
+        self.mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
+                              self.out, self.lse, self.ns, self.ws)
+
+    def step(self):
+        self.lens.copy_(self.lens0, non_blocking=True)
+        self.hash()
+        self.append()
+        self.decode()
+
+    def union_rows(self):
+        """Unique sampled (token, kv head) rows of one decode (for the bytes roofline)."""
+        torch = self.torch
+        w = self.w
+        self.step()
+        mem = torch.zeros((w.batch, w.n_q_heads, w.capacity), dtype=torch.uint8, device=self.q.device)
+        self.mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
+                              self.out, self.lse, self.ns, self.ws, member_out=mem)
+        torch.cuda.synchronize()
+        m = mem.view(w.batch, w.n_kv_heads, w.group, w.capacity).amax(dim=2)
+        return int(m.sum().item()), float(self.ns.float().mean().item())
+
+    def timed(self, steps, warmup):
+        torch = self.torch
+        for _ in range(warmup):
+            self.flush.zero_()
+            self.step()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        return ev
+
+    def run_timed(self, ev):
+        for e in ev:
+            self.flush.zero_()
+            self.lens.copy_(self.lens0, non_blocking=True)
+            e[0].record()
+            self.hash()
+            e[1].record()
+            self.append()
+            e[2].record()
+            self.decode()
+            e[3].record()
+
+    def run_e2e(self, steps, warmup):
+        """Public API with host buffers: per step, H2D of the step's inputs
+        (q, k_new, v_new, lengths) from pinned memory, the three calls, and
+        D2H of out / lse / n_sampled into pinned memory; device-timed."""
+        torch = self.torch
+        hq = torch.from_numpy(self.inp["q"].view(np.int16)).pin_memory()
+        hk = torch.from_numpy(self.inp["k_new"].view(np.int16)).pin_memory()
+        hv = torch.from_numpy(self.inp["v_new"].view(np.int16)).pin_memory()
+        hl = torch.from_numpy(self.inp["seq_lens"].astype(np.int32)).pin_memory()
+        ho = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        hlse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+        hns = torch.empty(self.ns.shape, dtype=torch.int32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hl))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hns))
+        times = []
+        for i in range(warmup + steps):
+            self.flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            self.q.copy_(hq, non_blocking=True)
+            self.k_new.copy_(hk, non_blocking=True)
+            self.v_new.copy_(hv, non_blocking=True)
+            self.lens.copy_(hl, non_blocking=True)
+            self.hash()
+            self.append()
+            self.decode()
+            ho.copy_(self.out, non_blocking=True)
+            hlse.copy_(self.lse, non_blocking=True)
+            hns.copy_(self.ns, non_blocking=True)
+            e.record()
+            e.synchronize()
+            if i >= warmup:
+                times.append(s.elapsed_time(e))
+        return statistics.mean(times), h2d, d2h
+
+
+def traffic_record(kernel, workload):
+    """dram bytes per launch from a committed ncu summary, if its kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        recs = json.load(open(path))
+    except ValueError:
+        return None
+    rec = recs.get(f"{kernel}@{workload}")
+    if not rec:
+        return None
+    import hashlib
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
+        return None
+    return rec["bytes_per_launch"]
+
+
+# ------------------------------------------------------ oracle (CPU) ----
+
+def oracle_unit_step(inp, w, b, kh):
+    """The fp64 oracle over one (b, kv head) unit of a step: SimHash of the
+    unit's post-append keys, query codes of its heads, then the decode."""
+    import oracle
+    n = int(inp["seq_lens"][b]) + 1
+    G = w.group
+    Kc = inp["K"][b, kh, :n].copy()
+    Kc[n - 1] = inp["k_new"][b, kh]
+    Vc = inp["V"][b, kh, :n].copy()
+    Vc[n - 1] = inp["v_new"][b, kh]
+    kc = oracle.simhash(Kc, inp["W"], w.k_bits, w.n_tables)
+    q = inp["q"][b:b + 1, kh * G:(kh + 1) * G]
+    qc = oracle.simhash(q, inp["W"], w.k_bits, w.n_tables)
+    oracle.decode(q, Kc[None, None], Vc[None, None], kc[None, None], qc, np.array([n], np.int32),
+                  Kbits=w.k_bits, L=w.n_tables, sink=w.sink, window=w.window)
+    return n
+
+
+def oracle_rate(inp, w, budget_s):
+    """Units of the step in (b, kv head) order until ~budget_s of CPU work;
+    the rate is scaled to the whole step by token count."""
+    import oracle
+    units = [(b, kh) for b in range(w.batch) for kh in range(w.n_kv_heads)]
+    total_unit_tokens = sum(int(inp["seq_lens"][b]) + 1 for b, _ in units)
+    done_tokens, t0, k = 0, time.perf_counter(), 0
+    for b, kh in units:
+        done_tokens += oracle_unit_step(inp, w, b, kh)
+        k += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    est_step = dt * total_unit_tokens / done_tokens
+    value = step_tokens(inp["seq_lens"] + 1) / est_step
+    sample = (f"{k} of {len(units)} (b, kv-head) units of one step ({done_tokens} unit-tokens: hash of their "
+              f"keys + collision scan + estimator), scaled to the full step by token count")
+    return value, dict(kind="oracle", cores=oracle.num_threads(), sample=sample, seconds=round(dt, 2))
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from workloads import make_inputs
+    oracle.build()
+    w = workload_for_rank(args.workload, 0)
+    inp = make_inputs(w)
+    G = w.group
+    units = [(b, kh) for b in range(w.batch) for kh in range(w.n_kv_heads)]
+    total_unit_tokens = sum(int(inp["seq_lens"][b]) + 1 for b, _ in units)
+    rates = []
+    for i in range(args.warmup + args.steps):
+        b, kh = units[i % len(units)]
+        t0 = time.perf_counter()
+        n = oracle_unit_step(inp, w, b, kh)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            rates.append(step_tokens(inp["seq_lens"] + 1) / (dt * total_unit_tokens / n))
+    value = statistics.mean(rates)
+    unit = "tokens/s"
+    line = dict(impl="reference", metric=METRIC, value=value, unit=unit, n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=1e3 * step_tokens(inp["seq_lens"] + 1) / value,
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                config=config_of(w),
+                cpu_baseline=dict(value=value, unit=unit, cores=oracle.num_threads(), kind="oracle",
+                                  sample="each step: one (b, kv-head) unit (hash of its keys + collision scan "
+                                         "+ estimator), scaled to the full step by token count"),
+                e2e=dict(value=value, unit=unit, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line, default=_jsonable), flush=True)
+
+
+def _jsonable(o):
+    if hasattr(o, "item"):
+        return o.item()
+    raise TypeError(type(o).__name__)
+
+
+def config_of(w):
+    return dict(workload=w.name, batch=w.batch, q_heads=w.n_q_heads, kv_heads=w.n_kv_heads,
+                head_dim=w.head_dim, context=w.context, ragged_min=w.ragged_min or None, k_bits=w.k_bits,
+                n_tables=w.n_tables, sink=w.sink, window=w.window, planted_per_kv_head=w.n_planted,
+                step="hash all cached keys + append 1 token/sequence + LSH-sampled decode",
+                l2="flushed between timed steps (256 MiB write)", parallelism="replicas (1 rank = 1 GPU)")
+
+
+# --------------------------------------------------------------- main ----
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", local if world > 1 else 0)
+    import __graft_entry__
+    __graft_entry__.build()
+    w = workload_for_rank(args.workload, rank)
+    bench = Bench(w, device)
+    union, mean_ns = bench.union_rows()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    ev = bench.timed(args.steps, args.warmup)
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local if world > 1 else 0)
+    clocks.start()
+    bench.run_timed(ev)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    hash_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    append_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    total = torch.tensor([sum(step_ms)], dtype=torch.float64, device=device)
+    tokens = torch.tensor([bench.tokens * args.steps], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(total, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tokens, op=dist.ReduceOp.SUM)
+    total_s = total.item() / 1e3
+    value = tokens.item() / total_s
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = bench.run_e2e(min(args.steps, 20), 3)
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = dict(value=bench.tokens * world / (t.item() / 1e3), unit="tokens/s", h2d_bytes_per_step=h2d,
+                   d2h_bytes_per_step=d2h, ms_per_step=t.item())
+
+    if rank == 0:
+        peaks = load_peaks()
+        B = w.batch
+        lens_after = bench.inp["seq_lens"] + 1
+        LK = w.n_tables * w.k_bits
+        code_bytes = int(lens_after.sum()) * w.n_kv_heads * LK // 8
+        d_rows = sum(min(w.sink, n) + n - max(min(w.sink, n), n - w.window) for n in lens_after) * w.n_kv_heads
+        dec_bytes = code_bytes + (union + d_rows) * 2 * w.head_dim * 2
+        hash_rows = int(bench.inp["seq_lens"].sum()) * w.n_kv_heads
+        hash_flops = 2.0 * hash_rows * w.head_dim * LK
+        if HASH_IMPL.startswith("tcgen05"):
+            hash_bound, hash_peak, hash_unit = "tensor", peaks["bf16"], "TFLOP/s"
+        else:  # fp32 FMA pipe: 148 SMs x 128 lanes x 2 flop x max SM clock
+            hash_bound, hash_peak, hash_unit = "alu", 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12, "TFLOP/s"
+        hash_roof = dict(kernel="mp_hash_keys", bound=hash_bound, achieved=hash_flops / (hash_ms / 1e3) / 1e12,
+                         peak=hash_peak, unit=hash_unit, algorithmic=hash_flops, units=f"{hash_rows} key rows",
+                         traffic=traffic_record("hash_keys", w.name))
+        hash_roof["frac"] = hash_roof["achieved"] / hash_roof["peak"]
+        dec_roof = dict(kernel="mp_decode_attend", bound="hbm", achieved=dec_bytes / (decode_ms / 1e3) / 1e9,
+                        peak=peaks["hbm"], unit="GB/s", algorithmic=dec_bytes,
+                        units=f"{int(lens_after.sum())} tokens x {w.n_kv_heads} kv heads; {union} union rows",
+                        traffic=traffic_record("decode", w.name))
+        dec_roof["frac"] = dec_roof["achieved"] / dec_roof["peak"]
+        dominant = hash_roof if hash_ms >= decode_ms else dec_roof
+        roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+        roofline["kernel"] = dominant["kernel"]
+        roofline["peak_source"] = peaks["source"]
+        line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
+                    warmup=args.warmup, ms_per_step=total.item() / args.steps, higher_is_better=True,
+                    scaling="weak", vs_baseline=None, dtype="bf16-in/fp32-acc", data="synthetic",
+                    config=config_of(w), roofline=roofline,
+                    breakdown=dict(hash_ms=hash_ms, append_ms=append_ms, decode_ms=decode_ms,
+                                   hash_roofline=hash_roof, decode_roofline=dec_roof,
+                                   decode_only_tokens_per_s=bench.tokens / (decode_ms / 1e3),
+                                   mean_sampled_per_head=mean_ns, union_rows=union),
+                    gpu_launches=bench.launches_per_step * args.steps, clocks=clk, e2e=e2e)
+        if world == 1 and not args.no_cpu_baseline:
+            v, info = oracle_rate(bench.inp, w, budget_s=10.0)
+            line["cpu_baseline"] = dict(value=v, unit="tokens/s", **info)
+        print(json.dumps(line, default=_jsonable), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

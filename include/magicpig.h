@@ -1,0 +1,158 @@
+/*
+ * magicpig.h - C ABI of the B200 (sm_100a) LSH-sampled decode-attention library.
+ *
+ * Method: MagicPIG, "LSH Sampling for Efficient LLM Generation" (Chen et al.,
+ * 2024).  The GrooveSquid summary page ("Medium Difficulty Summary") describes
+ * it as estimating the attention output by sampling instead of TopK selection;
+ * the sourcepulse project page ("How It Works") says the samples are chosen by
+ * locality-sensitive hashing; the gitdiagram page ("LSH Sampling": LSH kernel,
+ * LSH interface) names a native LSH library under it.  The arithmetic, in the
+ * notation used throughout this library:
+ *
+ *   SimHash.  W holds L*K random hyperplanes of dimension d; row c = l*K + b is
+ *   the hyperplane of bit b of table l.  Bit b of the table-l code of a vector
+ *   x is 1 iff x . W[c] > 0 (exactly 0 gives 0).
+ *   Sampling.  A context token i outside the exact set D is sampled for query
+ *   head h (i in S_h) iff its code equals the query's in at least 2 of the L
+ *   tables.  D = [0, sink) U [N - window, N).
+ *   Estimator.  s_i = q . k_i / sqrt(d); p_i = 1 - arccos(cos(q, k_i)) / pi;
+ *   x_i = p_i^K; u_i = 1 - (1-x_i)^L - L x_i (1-x_i)^(L-1); w_i = exp(s_i) on
+ *   D and exp(s_i - log u_i) on S_h; out = sum w_i v_i / sum w_i over D U S_h;
+ *   lse = log sum w_i (natural log, -log u included).
+ *
+ * Conventions for every call:
+ *   - Tensors are caller-owned device buffers (bf16 is passed as raw 16-bit
+ *     patterns).  The library allocates nothing and keeps no global state
+ *     beyond a per-device cache of function attributes.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) except mp_read_status, which synchronises.
+ *   - Return value: MP_OK or a negative MP_ERR_* from host-side validation
+ *     (nothing is launched then) or from the CUDA launch itself.  Faults found
+ *     on the device (a sequence length past the capacity) never trap: they are
+ *     written to a status word and the offending length is clamped.
+ *   - Every device pointer must be 16-byte aligned.
+ */
+#ifndef MAGICPIG_H
+#define MAGICPIG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MP_OK 0
+#define MP_ERR_ARG (-1)       /* null pointer, negative size, bad value */
+#define MP_ERR_SHAPE (-2)     /* unsupported shape (see mp_shape) */
+#define MP_ERR_ALIGN (-3)     /* a pointer is not 16-byte aligned */
+#define MP_ERR_CAPACITY (-4)  /* a length exceeds the capacity / max_len (device: clamped) */
+#define MP_ERR_WORKSPACE (-5) /* workspace smaller than mp_decode_workspace_bytes */
+#define MP_ERR_CUDA (-6)      /* a CUDA runtime call or launch failed */
+
+/*
+ * Problem shape.  Supported: head_dim == 128; k_bits in {8, 10};
+ * 2 <= n_tables <= 255 with n_tables * k_bits <= 2048; n_q_heads a multiple of
+ * n_kv_heads with group G = n_q_heads / n_kv_heads in {1, 2, 4, 8};
+ * capacity a positive multiple of 128 below 2^24; sink, window >= 0.
+ */
+typedef struct mp_shape {
+    int32_t batch;      /* B */
+    int32_t n_q_heads;  /* Hq */
+    int32_t n_kv_heads; /* Hkv */
+    int32_t head_dim;   /* d */
+    int32_t capacity;   /* Ncap: token slots of the K/V caches and of the codes */
+    int32_t k_bits;     /* K: SimHash bits per table */
+    int32_t n_tables;   /* L: hash tables */
+    int32_t sink;       /* leading tokens of the exact set D */
+    int32_t window;     /* trailing (most recent) tokens of the exact set D */
+} mp_shape;
+
+/*
+ * Key-code layout ("table-major"), per (b, kv head) unit:
+ *   k_bits == 8 : uint8  [B][Hkv][L][Ncap]         one byte per (table, token),
+ *                 bit b of the byte = bit b of the code.
+ *   k_bits == 10: uint32 [B][Hkv][L][K][Ncap/32]   bit planes: bit t of word
+ *                 (l, b, w) = bit b of the table-l code of token 32*w + t.
+ * Both use exactly L*K/8 bytes per token.  mp_codes_bytes gives the size.
+ */
+int mp_codes_bytes(const mp_shape *shape, size_t *bytes);
+
+/*
+ * Key hashing (SimHash of cached keys; the "LSH kernel" / hash-table
+ * construction of the gitdiagram and sourcepulse pages).
+ *   keys   bf16 [B][Hkv][Ncap][d]   rows [0, n_tokens) of every unit are hashed
+ *   W      bf16 [L*K][d]            hyperplanes, row c = l*K + b
+ *   seq_lens  int32 [B] device, nullable: if given, unit (b, .) hashes only
+ *          tokens [0, min(seq_lens[b], n_tokens)) (ragged batches)
+ *   codes  out, layout above; only the hashed tokens are written (for
+ *          k_bits == 10 the last partial 32-token word is rewritten whole).
+ * 0 <= n_tokens <= Ncap (host bound; sizes the grid).  Projections are fp32
+ * sums of exact bf16 products.
+ */
+int mp_hash_keys(const mp_shape *shape, const void *keys, const void *W, const int32_t *seq_lens,
+                 int32_t n_tokens, void *codes, void *stream);
+
+/*
+ * Query hashing: qcodes[b][h][l] (uint16) = table-l SimHash code of q[b][h].
+ *   q bf16 [B][Hq][d]; W as above; qcodes out uint16 [B][Hq][L].
+ */
+int mp_hash_queries(const mp_shape *shape, const void *q, const void *W, uint16_t *qcodes,
+                    void *stream);
+
+/*
+ * Decode-time append of one token per sequence: for every (b, kv head), at
+ * pos = seq_lens[b], writes k_cache/v_cache rows from k_new/v_new, writes the
+ * SimHash codes of k_new into column pos of the codes, then seq_lens[b] += 1.
+ *   k_new, v_new  bf16 [B][Hkv][d]
+ *   k_cache, v_cache  bf16 [B][Hkv][Ncap][d]      codes  layout above
+ *   seq_lens  int32 [B] device, incremented in place
+ *   status    int32 device word (nullable): set to MP_ERR_CAPACITY when some
+ *             seq_lens[b] >= Ncap (that sequence is then left untouched).
+ */
+int mp_append_token(const mp_shape *shape, const void *k_new, const void *v_new, const void *W,
+                    void *k_cache, void *v_cache, void *codes, int32_t *seq_lens,
+                    int32_t *status, void *stream);
+
+/* Test hooks of mp_decode_attend (all nullable). */
+typedef struct mp_decode_debug {
+    const uint16_t *qcodes_in; /* [B][Hq][L]: use these query codes instead of hashing q */
+    uint16_t *qcodes_out;      /* [B][Hq][L]: copy of the query codes used */
+    uint8_t *member_out;       /* [B][Hq][Ncap]: 1 iff token i is in S_h (i < N_b) */
+} mp_decode_debug;
+
+/* Workspace bytes that mp_decode_attend needs for sequences up to max_len. */
+int mp_decode_workspace_bytes(const mp_shape *shape, int32_t max_len, size_t *bytes);
+
+/*
+ * One LSH-sampled decode step (query hashing, collision scan + compaction,
+ * sampled attention with the -log u correction, the exact sink/window set D
+ * and the log-sum-exp merge) for every (b, query head).
+ *   q        bf16 [B][Hq][d]          W bf16 [L*K][d]
+ *   codes    key codes (layout above), valid for tokens [0, seq_lens[b])
+ *   k_cache, v_cache  bf16 [B][Hkv][Ncap][d]
+ *   seq_lens int32 [B] device: N_b; each must be <= max_len (else clamped and
+ *            MP_ERR_CAPACITY is recorded in the status word)
+ *   max_len  host bound on every N_b, 0 <= max_len <= Ncap (sizes the grid)
+ *   out      fp32 [B][Hq][d]           lse fp32 [B][Hq] (-inf when N_b == 0)
+ *   n_sampled int32 [B][Hq]: |S_h|, tokens of D excluded
+ *   workspace device scratch of at least mp_decode_workspace_bytes bytes; its
+ *            first word is the status word (reset by every call)
+ *   debug    nullable test hooks
+ */
+int mp_decode_attend(const mp_shape *shape, const void *q, const void *W, const void *codes,
+                     const void *k_cache, const void *v_cache, const int32_t *seq_lens,
+                     int32_t max_len, float *out, float *lse, int32_t *n_sampled, void *workspace,
+                     size_t workspace_bytes, const mp_decode_debug *debug, void *stream);
+
+/* Synchronises `stream` and reads the status word of a decode workspace. */
+int mp_read_status(const void *workspace, int32_t *status, void *stream);
+
+/* Human-readable name of an MP_* code. */
+const char *mp_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAGICPIG_H */

@@ -1,0 +1,36 @@
+"""B200 (sm_100a) LSH-sampled decode attention (MagicPIG hot path).
+
+The compute lives in ``libmagicpig_b200.so`` (hand-written CUDA kernels behind
+the C ABI of ``include/magicpig.h``); this package is a thin ctypes binding
+that marshals torch tensors (device memory and streams only) into those calls.
+There is no fallback: if the library is missing or cannot load, every call
+raises.
+"""
+from ._binding import (  # noqa: F401
+    MagicPIGError,
+    Shape,
+    append_token,
+    codes_bytes,
+    codes_shape,
+    decode_attend,
+    decode_workspace_bytes,
+    hash_keys,
+    hash_queries,
+    library,
+    library_path,
+    read_status,
+    status_string,
+    MP_OK,
+    MP_ERR_ARG,
+    MP_ERR_SHAPE,
+    MP_ERR_ALIGN,
+    MP_ERR_CAPACITY,
+    MP_ERR_WORKSPACE,
+    MP_ERR_CUDA,
+)
+
+__all__ = [
+    "MagicPIGError", "Shape", "append_token", "codes_bytes", "codes_shape", "decode_attend",
+    "decode_workspace_bytes", "hash_keys", "hash_queries", "library", "library_path", "read_status",
+    "status_string",
+]

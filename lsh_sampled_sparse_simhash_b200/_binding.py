@@ -1,0 +1,166 @@
+"""ctypes binding of include/magicpig.h (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libmagicpig_b200.so")
+
+MP_OK = 0
+MP_ERR_ARG = -1
+MP_ERR_SHAPE = -2
+MP_ERR_ALIGN = -3
+MP_ERR_CAPACITY = -4
+MP_ERR_WORKSPACE = -5
+MP_ERR_CUDA = -6
+
+
+class MagicPIGError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+class _CShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("batch", "n_q_heads", "n_kv_heads", "head_dim", "capacity", "k_bits", "n_tables",
+                 "sink", "window")]
+
+
+class _CDebug(ctypes.Structure):
+    _fields_ = [("qcodes_in", ctypes.c_void_p), ("qcodes_out", ctypes.c_void_p),
+                ("member_out", ctypes.c_void_p)]
+
+
+@dataclasses.dataclass(frozen=True)
+class Shape:
+    """Problem shape (see mp_shape in include/magicpig.h)."""
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    capacity: int
+    k_bits: int
+    n_tables: int
+    sink: int
+    window: int
+
+    def c(self) -> _CShape:
+        return _CShape(*dataclasses.astuple(self))
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Loads the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise MagicPIGError(MP_ERR_CUDA, f"{library_path} not built (run __graft_entry__.build())")
+        lib = ctypes.CDLL(library_path)
+        P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        SP = ctypes.POINTER(_CShape)
+        lib.mp_codes_bytes.argtypes = [SP, ctypes.POINTER(SZ)]
+        lib.mp_hash_keys.argtypes = [SP, P, P, P, I32, P, P]
+        lib.mp_hash_queries.argtypes = [SP, P, P, P, P]
+        lib.mp_append_token.argtypes = [SP, P, P, P, P, P, P, P, P, P]
+        lib.mp_decode_workspace_bytes.argtypes = [SP, I32, ctypes.POINTER(SZ)]
+        lib.mp_decode_attend.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P, SZ,
+                                         ctypes.POINTER(_CDebug), P]
+        lib.mp_read_status.argtypes = [P, ctypes.POINTER(I32), P]
+        lib.mp_status_string.argtypes = [ctypes.c_int]
+        lib.mp_status_string.restype = ctypes.c_char_p
+        for f in ("mp_codes_bytes", "mp_hash_keys", "mp_hash_queries", "mp_append_token",
+                  "mp_decode_workspace_bytes", "mp_decode_attend", "mp_read_status"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    try:
+        return library().mp_status_string(int(code)).decode()
+    except MagicPIGError:
+        return f"status {code}"
+
+
+def _check(code: int, where: str):
+    if code != MP_OK:
+        raise MagicPIGError(code, where)
+
+
+def _ptr(t) -> Optional[int]:
+    """Device pointer of a torch tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def codes_bytes(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    _check(library().mp_codes_bytes(ctypes.byref(shape.c()), ctypes.byref(n)), "mp_codes_bytes")
+    return n.value
+
+
+def codes_shape(shape: Shape):
+    """(dtype name, tensor shape) of the key codes: uint8 [B,Hkv,L,Ncap] for
+    K = 8, int32-bit planes [B,Hkv,L,K,Ncap/32] for K = 10."""
+    B, Hkv, L, K, N = shape.batch, shape.n_kv_heads, shape.n_tables, shape.k_bits, shape.capacity
+    if K == 8:
+        return "uint8", (B, Hkv, L, N)
+    return "int32", (B, Hkv, L, K, N // 32)
+
+
+def decode_workspace_bytes(shape: Shape, max_len: int) -> int:
+    n = ctypes.c_size_t()
+    _check(library().mp_decode_workspace_bytes(ctypes.byref(shape.c()), int(max_len), ctypes.byref(n)),
+           "mp_decode_workspace_bytes")
+    return n.value
+
+
+def hash_keys(shape: Shape, keys, W, n_tokens: int, codes, seq_lens=None, stream=None):
+    _check(library().mp_hash_keys(ctypes.byref(shape.c()), _ptr(keys), _ptr(W), _ptr(seq_lens), int(n_tokens),
+                                  _ptr(codes), _stream(stream)), "mp_hash_keys")
+
+
+def hash_queries(shape: Shape, q, W, qcodes, stream=None):
+    _check(library().mp_hash_queries(ctypes.byref(shape.c()), _ptr(q), _ptr(W), _ptr(qcodes), _stream(stream)),
+           "mp_hash_queries")
+
+
+def append_token(shape: Shape, k_new, v_new, W, k_cache, v_cache, codes, seq_lens, status=None, stream=None):
+    _check(library().mp_append_token(ctypes.byref(shape.c()), _ptr(k_new), _ptr(v_new), _ptr(W),
+                                     _ptr(k_cache), _ptr(v_cache), _ptr(codes), _ptr(seq_lens), _ptr(status),
+                                     _stream(stream)), "mp_append_token")
+
+
+def decode_attend(shape: Shape, q, W, codes, k_cache, v_cache, seq_lens, max_len: int, out, lse, n_sampled,
+                  workspace, qcodes_in=None, qcodes_out=None, member_out=None, stream=None):
+    dbg = None
+    if qcodes_in is not None or qcodes_out is not None or member_out is not None:
+        dbg = ctypes.byref(_CDebug(_ptr(qcodes_in), _ptr(qcodes_out), _ptr(member_out)))
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(library().mp_decode_attend(ctypes.byref(shape.c()), _ptr(q), _ptr(W), _ptr(codes), _ptr(k_cache),
+                                      _ptr(v_cache), _ptr(seq_lens), int(max_len), _ptr(out), _ptr(lse),
+                                      _ptr(n_sampled), _ptr(workspace), nbytes, dbg, _stream(stream)),
+           "mp_decode_attend")
+
+
+def read_status(workspace, stream=None) -> int:
+    v = ctypes.c_int32()
+    _check(library().mp_read_status(_ptr(workspace), ctypes.byref(v), _stream(stream)), "mp_read_status")
+    return v.value

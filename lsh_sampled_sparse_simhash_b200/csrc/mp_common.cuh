@@ -1,0 +1,69 @@
+// Shared device helpers of the sm_100a LSH-sampled decode-attention library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "magicpig.h"
+
+namespace mp {
+
+constexpr int kHeadDim = 128;
+constexpr int kMaxGroup = 8;
+constexpr int kChunkK8 = 2048;   // scan chunk (tokens) for byte codes: 128 threads x 16 tokens
+constexpr int kChunkK10 = 8192;  // scan chunk (tokens) for bit planes: 64 threads x 128 tokens
+constexpr int kScanThreadsK8 = 128;
+constexpr int kScanThreadsK10 = 64;
+
+struct Shape {
+    int B, Hq, Hkv, G, d, Ncap, K, L, LK, sink, window;
+};
+
+inline int chunk_tokens(int K) { return K == 8 ? kChunkK8 : kChunkK10; }
+
+// Device-side status word: the first error wins, later ones are dropped.
+__device__ __forceinline__ void set_status(int32_t *status, int32_t code)
+{
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t packed) { return __uint_as_float(packed << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t packed) { return __uint_as_float(packed & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte global->shared copy; src_bytes = 0 zero-fills the destination.
+__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gmem_src, int src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem_dst)),
+                 "l"(gmem_src), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
+                                            const void *smem_row)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(smem_row)));
+}
+
+// D(16x8, fp32) += A(16x16, bf16, row) * B(16x8, bf16, col)
+__device__ __forceinline__ void mma_bf16_16816(float &d0, float &d1, float &d2, float &d3, uint32_t a0,
+                                               uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+}  // namespace mp

@@ -1,0 +1,106 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports
+every entry point that include/magicpig.h declares, and rejects bad arguments
+on the host (no kernel is launched, no CUDA call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import lsh_sampled_sparse_simhash_b200 as mp
+from lsh_sampled_sparse_simhash_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "magicpig.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__
+    __graft_entry__.build()
+    return mp.library()
+
+
+def good_shape(**kw):
+    d = dict(batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, capacity=1024, k_bits=8, n_tables=75,
+             sink=4, window=64)
+    d.update(kw)
+    return B._CShape(*d.values())
+
+
+def test_exports_every_declared_symbol(lib):
+    decl = re.findall(r"^\s*(?:int|const char \*)\s*(mp_\w+)\s*\(", open(HEADER).read(), re.M)
+    assert len(decl) >= 8
+    for name in decl:
+        assert hasattr(lib, name), name
+    # and nothing undeclared under the mp_ prefix
+    import subprocess
+    syms = subprocess.run(["nm", "-D", "--defined-only", mp.library_path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (mp_\w+)$", syms, re.M))
+    assert exported == set(decl), exported ^ set(decl)
+
+
+def test_library_has_no_driver_link_dependency(lib):
+    import subprocess
+    out = subprocess.run(["ldd", mp.library_path], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libtorch" not in out
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert mp.status_string(code).startswith("MP_")
+
+
+def test_codes_bytes_formula(lib):
+    n = ctypes.c_size_t()
+    for K, L in [(8, 75), (10, 150)]:
+        s = good_shape(k_bits=K, n_tables=L)
+        assert lib.mp_codes_bytes(ctypes.byref(s), ctypes.byref(n)) == 0
+        assert n.value == 2 * 2 * L * K * 1024 // 8
+
+
+@pytest.mark.parametrize("bad", [
+    dict(head_dim=64), dict(k_bits=9), dict(n_tables=1), dict(n_tables=256), dict(n_q_heads=6),
+    dict(n_q_heads=32, n_kv_heads=2), dict(capacity=1000), dict(capacity=0), dict(batch=0),
+    dict(sink=-1), dict(window=-1), dict(n_kv_heads=0)])
+def test_bad_shapes_rejected(lib, bad):
+    n = ctypes.c_size_t()
+    s = good_shape(**bad)
+    assert lib.mp_codes_bytes(ctypes.byref(s), ctypes.byref(n)) == mp.MP_ERR_SHAPE
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, 10, 16, None) == mp.MP_ERR_SHAPE
+    assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 10, ctypes.byref(n)) == mp.MP_ERR_SHAPE
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    s = good_shape()
+    assert lib.mp_hash_keys(ctypes.byref(s), None, 16, None, 10, 16, None) == mp.MP_ERR_ARG
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 18, None, 10, 16, None) == mp.MP_ERR_ALIGN
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, 18, 10, 16, None) == mp.MP_ERR_ALIGN
+    assert lib.mp_hash_queries(ctypes.byref(s), 16, 16, None, None) == mp.MP_ERR_ARG
+    assert lib.mp_append_token(ctypes.byref(s), 16, 16, 16, 16, 16, 16, None, None, None) == mp.MP_ERR_ARG
+    assert lib.mp_append_token(ctypes.byref(s), 16, 16, 16, 16, 16, 16, 16, 18, None) == mp.MP_ERR_ALIGN
+    assert lib.mp_read_status(None, None, None) == mp.MP_ERR_ARG
+
+
+def test_lengths_and_workspace_checked(lib):
+    s = good_shape()
+    n = ctypes.c_size_t()
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, 1025, 16, None) == mp.MP_ERR_CAPACITY
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, -1, 16, None) == mp.MP_ERR_CAPACITY
+    assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 1025, ctypes.byref(n)) == mp.MP_ERR_CAPACITY
+    assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 1000, ctypes.byref(n)) == 0
+    need = n.value
+    args = [16] * 6 + [1000] + [16] * 4
+    assert lib.mp_decode_attend(ctypes.byref(s), *args, need - 1, None, None) == mp.MP_ERR_WORKSPACE
+    args[6] = 2000
+    assert lib.mp_decode_attend(ctypes.byref(s), *args, need, None, None) == mp.MP_ERR_CAPACITY
+
+
+def test_workspace_grows_with_max_len(lib):
+    s = good_shape(capacity=65536)
+    sizes = []
+    for m in (0, 1, 2048, 2049, 65536):
+        n = ctypes.c_size_t()
+        assert lib.mp_decode_workspace_bytes(ctypes.byref(s), m, ctypes.byref(n)) == 0
+        sizes.append(n.value)
+    assert sizes == sorted(sizes) and sizes[1] < sizes[3]

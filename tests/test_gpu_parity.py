@@ -1,0 +1,283 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bars: key/query codes bit-exact except bits whose fp64 projection lies within
+1e-4 |k||w| of zero (those are counted); candidate sets and n_sampled
+bit-exact when both sides get the same codes; out within 2e-3 relative L2 per
+head and lse within 1e-3 of the oracle on the same candidate set.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_harness import (Run, check_outputs, code_mismatch, dev, host, oracle_decode_units,
+                         oracle_query_codes, oracle_unit_codes)
+from workloads import WORKLOADS, f32_to_bf16_bits, make_inputs
+
+import lsh_sampled_sparse_simhash_b200 as mp
+
+pytestmark = pytest.mark.gpu
+
+TINY = WORKLOADS["tiny"]
+SMALL_CASES = {
+    "tiny_g1_k8": TINY,
+    "g4_k8_ragged_tail": TINY.with_(name="g4k8", batch=2, n_q_heads=8, n_kv_heads=2, context=5000,
+                                    n_planted=16, seed=2001),
+    "g4_k10": TINY.with_(name="g4k10", batch=2, n_q_heads=8, n_kv_heads=2, context=9000, k_bits=10,
+                         n_tables=150, n_planted=24, seed=2002),
+    "g2_k10_short": TINY.with_(name="g2k10", batch=1, n_q_heads=4, n_kv_heads=2, context=700, k_bits=10,
+                               n_tables=150, n_planted=4, seed=2003),
+    "g8_k8": TINY.with_(name="g8k8", batch=1, n_q_heads=16, n_kv_heads=2, context=4100, n_planted=8,
+                        seed=2004),
+    "g4_k8_mu_offset": TINY.with_(name="mu", batch=2, n_q_heads=8, n_kv_heads=2, context=6000,
+                                  mu_norm=8.0, n_planted=16, seed=2005),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    import __graft_entry__
+    __graft_entry__.build()
+    assert torch.cuda.is_available()
+
+
+def all_units(w):
+    return [(b, kh) for b in range(w.batch) for kh in range(w.n_kv_heads)]
+
+
+def oracle_codes_all(run):
+    w, inp = run.w, run.inp
+    units = all_units(w)
+    res = [oracle_unit_codes(inp, w, b, kh, int(inp["seq_lens"][b])) for b, kh in units]
+    return units, [c for c, _ in res], [m for _, m in res]
+
+
+@pytest.mark.parametrize("case", list(SMALL_CASES))
+def test_hash_keys_and_queries_match_oracle(case):
+    w = SMALL_CASES[case]
+    run = Run(w)
+    run.hash_keys()
+    torch.cuda.synchronize()
+    units, codes, margins = oracle_codes_all(run)
+    bad = exempt = 0
+    for (b, kh), c, m in zip(units, codes, margins):
+        n = c.shape[0]
+        g = run.codes_logical(b, kh, n)
+        x, e = code_mismatch(g, c, m, w.k_bits)
+        bad += x
+        exempt += e
+    assert bad == 0, f"{bad} key-code bits differ beyond the near-zero tolerance ({exempt} exempt)"
+    qref, qmargin = oracle_query_codes(run.inp, w)
+    x, e = code_mismatch(run.hash_queries(), qref, qmargin, w.k_bits)
+    assert x == 0, f"{x} query-code bits differ ({e} exempt)"
+
+
+@pytest.mark.parametrize("case", list(SMALL_CASES))
+def test_decode_same_codes_matches_oracle(case):
+    """Both sides get the oracle's key and query codes: S_h and n_sampled must
+    be identical, outputs within tolerance."""
+    w = SMALL_CASES[case]
+    run = Run(w)
+    units, codes, _ = oracle_codes_all(run)
+    run.set_codes(codes, units)
+    qref, _ = oracle_query_codes(run.inp, w)
+    gpu = run.decode(qcodes_in=qref)
+    assert gpu["status"] == 0
+    np.testing.assert_array_equal(gpu["qcodes"], qref)
+    ref = oracle_decode_units(run.inp, w, units, codes, qref)
+    worst = check_outputs(gpu, ref, w)
+    print(f"{case}: worst rel-L2 {worst:.2e}, sampled per head {gpu['ns'].mean():.1f}")
+    assert gpu["ns"].sum() > 0 or w.context <= w.sink + w.window
+
+
+@pytest.mark.parametrize("case", ["tiny_g1_k8", "g4_k10", "g8_k8"])
+def test_end_to_end_gpu_codes(case):
+    """GPU hashing feeds the GPU scan.  Where a GPU code equals the oracle's,
+    membership must agree; when every code agrees, so must the outputs."""
+    w = SMALL_CASES[case]
+    run = Run(w)
+    run.hash_keys()
+    gpu = run.decode()
+    units, codes, _ = oracle_codes_all(run)
+    qref, _ = oracle_query_codes(run.inp, w)
+    ref = oracle_decode_units(run.inp, w, units, codes, qref)
+    G = w.group
+    all_same = np.array_equal(gpu["qcodes"], qref)
+    for (b, kh), c in zip(units, codes):
+        n = c.shape[0]
+        same_tok = (run.codes_logical(b, kh, n) == c).all(axis=1)
+        all_same &= bool(same_tok.all())
+        mem = ref[(b, kh)][3]
+        hs = slice(kh * G, (kh + 1) * G)
+        np.testing.assert_array_equal(gpu["member"][b, hs, :n][:, same_tok], mem[:, same_tok])
+    if all_same:
+        check_outputs(gpu, ref, w)
+
+
+def test_short_and_empty_contexts():
+    """N = 0, 1, and N <= sink + window (D covers everything, S is empty)."""
+    w = TINY.with_(name="short", batch=4, n_q_heads=8, n_kv_heads=2, context=300, n_planted=0, seed=2010)
+    inp = make_inputs(w)
+    inp["seq_lens"] = np.array([0, 1, 68, 69], np.int32)
+    run = Run(w, inp)
+    run.alloc_decode(300)
+    run.hash_keys(300)
+    units = all_units(w)
+    codes = [oracle_unit_codes(inp, w, b, kh, int(inp["seq_lens"][b]))[0] for b, kh in units]
+    run.set_codes(codes, units)
+    qref, _ = oracle_query_codes(inp, w)
+    gpu = run.decode(qcodes_in=qref)
+    ref = oracle_decode_units(inp, w, units, codes, qref)
+    check_outputs(gpu, ref, w)
+    assert (gpu["ns"][:3] == 0).all()
+    assert np.isinf(gpu["lse"][0]).all() and not gpu["out"][0].any()
+
+
+def test_every_token_sampled():
+    """All-zero hyperplanes: every projection is exactly 0, every code is 0,
+    every token collides in all L tables and is sampled (u from its angle)."""
+    w = TINY.with_(name="allcand", batch=1, n_q_heads=4, n_kv_heads=1, context=3000, n_planted=0, seed=2011)
+    inp = make_inputs(w)
+    inp["W"] = np.zeros_like(inp["W"])
+    run = Run(w, inp)
+    run.hash_keys()
+    gpu = run.decode()
+    n = int(inp["seq_lens"][0])
+    codes = [np.zeros((n, w.n_tables), np.uint16)]
+    qref = np.zeros((1, 4, w.n_tables), np.uint16)
+    np.testing.assert_array_equal(gpu["qcodes"], qref)
+    assert (run.codes_logical(0, 0, n) == 0).all()
+    ref = oracle_decode_units(inp, w, [(0, 0)], codes, qref)
+    check_outputs(gpu, ref, w)
+    assert (gpu["ns"] == n - w.sink - w.window).all()
+
+
+@pytest.mark.parametrize("K,L", [(8, 75), (10, 150)])
+def test_keys_on_hyperplanes_get_zero_bits(K, L):
+    """Hand-built ties: W[c] = e_j - e_{j+1} and keys with k_j == k_{j+1} have
+    projection exactly 0, which must give bit 0 (strict > 0 rule)."""
+    w = TINY.with_(name="ties", batch=1, n_q_heads=1, n_kv_heads=1, context=256, k_bits=K, n_tables=L,
+                   n_planted=0, seed=2012)
+    inp = make_inputs(w)
+    d = 128
+    Wf = np.zeros((L * K, d), np.float32)
+    for c in range(L * K):
+        Wf[c, c % d] = 1.0
+        Wf[c, (c + 1) % d] = -1.0
+    inp["W"] = f32_to_bf16_bits(Wf)
+    kf = np.random.default_rng(1).standard_normal((256, d)).astype(np.float32)
+    kf[::3, 1::2] = kf[::3, 0::2]  # every third key: k_{2i+1} = k_{2i}
+    inp["K"][0, 0, :256] = f32_to_bf16_bits(kf)
+    run = Run(w, inp)
+    run.hash_keys()
+    torch.cuda.synchronize()
+    ref, margin = oracle_unit_codes(inp, w, 0, 0, 256)
+    assert (margin == 0).any()
+    got = run.codes_logical(0, 0, 256)
+    np.testing.assert_array_equal(got, ref)  # ties must match exactly, not just within tolerance
+
+
+def test_append_then_decode_equals_rehash():
+    for w in (SMALL_CASES["g4_k8_ragged_tail"], SMALL_CASES["g4_k10"]):
+        inp = make_inputs(w)
+        run = Run(w, inp)
+        run.alloc_decode(w.context + 1)
+        run.hash_keys(w.context)
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        mp.append_token(run.shape, run.k_new, run.v_new, run.W, run.K, run.V, run.codes, run.lens, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert (host(run.lens) == w.context + 1).all()
+        kn = inp["k_new"]
+        for b in range(w.batch):
+            for kh in range(w.n_kv_heads):
+                np.testing.assert_array_equal(host(run.K[b, kh, w.context]).view(np.uint16), kn[b, kh])
+                np.testing.assert_array_equal(host(run.V[b, kh, w.context]).view(np.uint16), inp["v_new"][b, kh])
+                ref, margin = oracle_unit_codes({"K": kn[:, :, None], "W": inp["W"]}, w, b, kh, 1)
+                got = run.codes_logical(b, kh, w.context + 1)[-1:]
+                x, _ = code_mismatch(got, ref, margin, w.k_bits)
+                assert x == 0
+        # the appended cache decodes like a cache hashed from scratch
+        inp2 = dict(inp)
+        inp2["K"] = host(run.K).view(np.uint16)
+        inp2["V"] = host(run.V).view(np.uint16)
+        inp2["seq_lens"] = host(run.lens)
+        gpu = run.decode()
+        ref_run = Run(w, inp2)
+        ref_run.alloc_decode(w.context + 1)
+        ref_run.hash_keys(w.context + 1)
+        gpu2 = ref_run.decode()
+        np.testing.assert_array_equal(gpu["member"], gpu2["member"])
+        np.testing.assert_allclose(gpu["out"], gpu2["out"], rtol=0, atol=0)
+
+
+def test_append_past_capacity_sets_status():
+    w = TINY.with_(name="cap", context=255, n_planted=0, seed=2013)  # capacity 256
+    run = Run(w)
+    run.lens.fill_(256)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mp.append_token(run.shape, run.k_new, run.v_new, run.W, run.K, run.V, run.codes, run.lens, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == mp.MP_ERR_CAPACITY
+    assert int(run.lens.item()) == 256
+
+
+def test_overlong_length_is_clamped_and_reported():
+    w = SMALL_CASES["g4_k8_ragged_tail"]
+    run = Run(w)
+    run.hash_keys()
+    ref = run.decode()
+    assert ref["status"] == 0
+    run.lens.add_(50)  # past max_len
+    got = run.decode()
+    assert got["status"] == mp.MP_ERR_CAPACITY
+    np.testing.assert_array_equal(got["out"], ref["out"])
+
+
+# ------------------------------------------------ full-size configurations ----
+
+FULL = ["llama8b_16k", "batch8_64k", "batch4_128k", "ragged16"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_units(name):
+    """The full workload in the benchmark's launch configuration (hash every
+    key, append one token per sequence, decode); two (b, kv head) units are
+    checked against the oracle on the oracle's own codes."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    run = Run(w, inp)
+    run.alloc_decode(run.max_len + 1)
+    run.hash_keys(run.max_len)
+    mp.append_token(run.shape, run.k_new, run.v_new, run.W, run.K, run.V, run.codes, run.lens)
+    torch.cuda.synchronize()
+    new_lens = host(run.lens)
+    assert (new_lens == inp["seq_lens"] + 1).all()
+    # host copy of the post-append cache for the sampled units
+    units = [(0, 0), (w.batch - 1, w.n_kv_heads - 1)]
+    inp2 = dict(inp)
+    inp2["seq_lens"] = new_lens
+    K2 = inp["K"].copy()
+    V2 = inp["V"].copy()
+    for b in range(w.batch):
+        K2[b, :, inp["seq_lens"][b]] = inp["k_new"][b]
+        V2[b, :, inp["seq_lens"][b]] = inp["v_new"][b]
+    inp2["K"], inp2["V"] = K2, V2
+    codes, bad = [], 0
+    rng = np.random.default_rng(0)
+    for b, kh in units:
+        n = int(new_lens[b])
+        c, m = oracle_unit_codes(inp2, w, b, kh, n)
+        codes.append(c)
+        pick = rng.choice(n, size=min(n, 4096), replace=False)
+        x, _ = code_mismatch(run.codes_logical(b, kh, n)[pick], c[pick], m[pick], w.k_bits)
+        bad += x
+    assert bad == 0
+    run.set_codes(codes, units)
+    qref, _ = oracle_query_codes(inp, w)
+    gpu = run.decode(qcodes_in=qref)
+    assert gpu["status"] == 0
+    ref = oracle_decode_units(inp2, w, units, codes, qref)
+    worst = check_outputs(gpu, ref, w)
+    print(f"{name}: worst rel-L2 {worst:.2e}; mean |S_h| {gpu['ns'].mean():.0f}")
