@@ -2,8 +2,8 @@
 """Benchmark of one LSH-sampled decode layer-step (MagicPIG hot path) on B200.
 
 A step = every row of the hot path over one batch of synthetic input:
-  mp_hash_keys   SimHash of every cached key (tcgen05-free SIMT or tensor-core
-                 hash, see the roofline "bound"),
+  mp_hash_keys   SimHash of every cached key (tcgen05 tensor-core GEMM with a
+                 sign-packing epilogue),
   mp_append_token  one new token per sequence (K/V row + codes, length + 1),
   mp_decode_attend query hash, collision scan + compaction, sampled attention
                  with the -log u correction, exact sink/window set, LSE merge.
@@ -34,7 +34,7 @@ sys.path.insert(0, ROOT)
 DEFAULT_WORKLOAD = "llama8b_16k"
 FLUSH_BYTES = 256 << 20  # > 126 MB L2
 METRIC = "decode context-tokens scanned/s per layer-step"
-HASH_IMPL = "simt-fp32"   # implementation of mp_hash_keys in this build
+HASH_IMPL = "tcgen05-bf16"   # implementation of mp_hash_keys in this build
 
 
 def parse():
@@ -57,6 +57,19 @@ def load_peaks():
                     bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                     sm_max_mhz=float(d.get("sm_max_mhz", 1965.0)), source="measured")
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
+
+
+def reduce_over_ranks(total_ms, tokens, device, world):
+    """Whole-job numbers: the slowest rank's device time and the sum of the
+    tokens every rank processed (one replica per rank)."""
+    import torch
+    t = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    n = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return t.item(), n.item()
 
 
 def workload_for_rank(name, rank):
@@ -185,6 +198,15 @@ class Bench:
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
         return ev
 
+    def preroll(self, seconds):
+        torch = self.torch
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            for _ in range(8):
+                self.flush.zero_()
+                self.step()
+            torch.cuda.synchronize()
+
     def run_timed(self, ev):
         for e in ev:
             self.flush.zero_()
@@ -279,16 +301,15 @@ def oracle_rate(inp, w, budget_s):
     units = [(b, kh) for b in range(w.batch) for kh in range(w.n_kv_heads)]
     total_unit_tokens = sum(int(inp["seq_lens"][b]) + 1 for b, _ in units)
     done_tokens, t0, k = 0, time.perf_counter(), 0
-    for b, kh in units:
+    while time.perf_counter() - t0 < budget_s:
+        b, kh = units[k % len(units)]
         done_tokens += oracle_unit_step(inp, w, b, kh)
         k += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
     dt = time.perf_counter() - t0
     est_step = dt * total_unit_tokens / done_tokens
     value = step_tokens(inp["seq_lens"] + 1) / est_step
-    sample = (f"{k} of {len(units)} (b, kv-head) units of one step ({done_tokens} unit-tokens: hash of their "
-              f"keys + collision scan + estimator), scaled to the full step by token count")
+    sample = (f"{k} (b, kv-head) unit-steps of the {len(units)} in one step ({done_tokens} unit-tokens: SimHash "
+              f"of the unit's keys + collision scan + estimator), scaled to the full step by token count")
     return value, dict(kind="oracle", cores=oracle.num_threads(), sample=sample, seconds=round(dt, 2))
 
 
@@ -369,10 +390,11 @@ def main():
             dist.barrier()
 
     ev = bench.timed(args.steps, args.warmup)
-    barrier()
-    torch.cuda.synchronize()
     clocks = ClockSampler(local if world > 1 else 0)
     clocks.start()
+    bench.preroll(0.5)  # untimed steps so the sampler sees the clocks under this load
+    barrier()
+    torch.cuda.synchronize()
     bench.run_timed(ev)
     torch.cuda.synchronize()
     barrier()
@@ -381,13 +403,8 @@ def main():
     hash_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     append_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
-    total = torch.tensor([sum(step_ms)], dtype=torch.float64, device=device)
-    tokens = torch.tensor([bench.tokens * args.steps], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(total, op=dist.ReduceOp.MAX)
-        dist.all_reduce(tokens, op=dist.ReduceOp.SUM)
-    total_s = total.item() / 1e3
-    value = tokens.item() / total_s
+    total_ms, all_tokens = reduce_over_ranks(sum(step_ms), bench.tokens * args.steps, device, world)
+    value = all_tokens / (total_ms / 1e3)
 
     e2e = None
     if not args.no_e2e:
@@ -426,7 +443,7 @@ def main():
         roofline["kernel"] = dominant["kernel"]
         roofline["peak_source"] = peaks["source"]
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
-                    warmup=args.warmup, ms_per_step=total.item() / args.steps, higher_is_better=True,
+                    warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype="bf16-in/fp32-acc", data="synthetic",
                     config=config_of(w), roofline=roofline,
                     breakdown=dict(hash_ms=hash_ms, append_ms=append_ms, decode_ms=decode_ms,

@@ -87,11 +87,14 @@ int mp_codes_bytes(const mp_shape *shape, size_t *bytes);
  *          tokens [0, min(seq_lens[b], n_tokens)) (ragged batches)
  *   codes  out, layout above; only the hashed tokens are written (for
  *          k_bits == 10 the last partial 32-token word is rewritten whole).
- * 0 <= n_tokens <= Ncap (host bound; sizes the grid).  Projections are fp32
- * sums of exact bf16 products.
+ *   status int32 device word (nullable): MP_ERR_CUDA if the kernel's internal
+ *          pipeline stalled (a bounded wait expired; the codes are then
+ *          incomplete).  Never written on success.
+ * 0 <= n_tokens <= Ncap (host bound; sizes the grid).  Projections are bf16
+ * tensor-core products with fp32 accumulation (tcgen05).
  */
 int mp_hash_keys(const mp_shape *shape, const void *keys, const void *W, const int32_t *seq_lens,
-                 int32_t n_tokens, void *codes, void *stream);
+                 int32_t n_tokens, void *codes, int32_t *status, void *stream);
 
 /*
  * Query hashing: qcodes[b][h][l] (uint16) = table-l SimHash code of q[b][h].

@@ -65,7 +65,7 @@ def library() -> ctypes.CDLL:
         P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
         SP = ctypes.POINTER(_CShape)
         lib.mp_codes_bytes.argtypes = [SP, ctypes.POINTER(SZ)]
-        lib.mp_hash_keys.argtypes = [SP, P, P, P, I32, P, P]
+        lib.mp_hash_keys.argtypes = [SP, P, P, P, I32, P, P, P]
         lib.mp_hash_queries.argtypes = [SP, P, P, P, P]
         lib.mp_append_token.argtypes = [SP, P, P, P, P, P, P, P, P, P]
         lib.mp_decode_workspace_bytes.argtypes = [SP, I32, ctypes.POINTER(SZ)]
@@ -132,9 +132,9 @@ def decode_workspace_bytes(shape: Shape, max_len: int) -> int:
     return n.value
 
 
-def hash_keys(shape: Shape, keys, W, n_tokens: int, codes, seq_lens=None, stream=None):
+def hash_keys(shape: Shape, keys, W, n_tokens: int, codes, seq_lens=None, status=None, stream=None):
     _check(library().mp_hash_keys(ctypes.byref(shape.c()), _ptr(keys), _ptr(W), _ptr(seq_lens), int(n_tokens),
-                                  _ptr(codes), _stream(stream)), "mp_hash_keys")
+                                  _ptr(codes), _ptr(status), _stream(stream)), "mp_hash_keys")
 
 
 def hash_queries(shape: Shape, q, W, qcodes, stream=None):

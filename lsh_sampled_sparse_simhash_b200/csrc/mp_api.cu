@@ -89,16 +89,17 @@ int mp_codes_bytes(const mp_shape *shape, size_t *bytes)
 }
 
 int mp_hash_keys(const mp_shape *shape, const void *keys, const void *W, const int32_t *seq_lens,
-                 int32_t n_tokens, void *codes, void *stream)
+                 int32_t n_tokens, void *codes, int32_t *status, void *stream)
 {
     Shape s;
     int r = validate_shape(shape, s);
     if (r) return r;
     if ((r = check_ptrs({keys, W, codes}))) return r;
     if (seq_lens && (reinterpret_cast<uintptr_t>(seq_lens) & 3u)) return MP_ERR_ALIGN;
+    if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return MP_ERR_ALIGN;
     if (n_tokens < 0 || n_tokens > s.Ncap) return MP_ERR_CAPACITY;
-    return cuda_status(launch_hash_keys(s, static_cast<const uint16_t *>(keys), static_cast<const uint16_t *>(W),
-                                        seq_lens, n_tokens, codes, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_hash_keys_tc(s, static_cast<const uint16_t *>(keys), static_cast<const uint16_t *>(W),
+                                           seq_lens, n_tokens, codes, status, static_cast<cudaStream_t>(stream)));
 }
 
 int mp_hash_queries(const mp_shape *shape, const void *q, const void *W, uint16_t *qcodes, void *stream)

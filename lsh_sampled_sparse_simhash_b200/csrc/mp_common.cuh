@@ -10,10 +10,10 @@ namespace mp {
 
 constexpr int kHeadDim = 128;
 constexpr int kMaxGroup = 8;
-constexpr int kChunkK8 = 2048;   // scan chunk (tokens) for byte codes: 128 threads x 16 tokens
-constexpr int kChunkK10 = 8192;  // scan chunk (tokens) for bit planes: 64 threads x 128 tokens
-constexpr int kScanThreadsK8 = 128;
-constexpr int kScanThreadsK10 = 64;
+constexpr int kScanThreads = 256;  // scan block: token groups x table splits
+constexpr int kScanSplits = 4;     // tables l = ts, ts + 4, ... per split
+constexpr int kChunkK8 = 1024;     // scan chunk (tokens) for byte codes: 64 groups x 16 tokens
+constexpr int kChunkK10 = 8192;    // scan chunk (tokens) for bit planes: 64 groups x 128 tokens
 
 struct Shape {
     int B, Hq, Hkv, G, d, Ncap, K, L, LK, sink, window;
@@ -30,6 +30,16 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code)
 __device__ __forceinline__ float bf16_lo(uint32_t packed) { return __uint_as_float(packed << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t packed) { return __uint_as_float(packed & 0xFFFF0000u); }
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+// Programmatic dependent launch: block until the preceding kernel in the
+// stream has completed and its memory is visible, then let the next kernel
+// start launching.  Both are no-ops for a kernel launched without the
+// programmatic-serialization attribute.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {

@@ -16,6 +16,8 @@
 //           n_sampled.
 #include <math.h>
 
+#include <algorithm>
+
 #include "mp_common.cuh"
 #include "mp_kernels.cuh"
 
@@ -40,6 +42,7 @@ __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__r
     const int l0 = blockIdx.x * TB;
     const size_t vec0 = (size_t)b * s.Hq + (size_t)kvh * G;
 
+    grid_dependency_wait();
     if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *status = 0;
 
     if (qcodes_in) {
@@ -167,7 +170,7 @@ __device__ __forceinline__ uint32_t range_mask(int base, int lo, int hi, int wid
 template <int G, int NW, int WIDTH>
 __device__ __forceinline__ void compact_and_store(const Shape &s, int unit, int chunk, int nchunk,
                                                   int chunk_tokens, int t0, int N, int lo, int hi,
-                                                  uint32_t (&hm)[G][NW], const ScanOut &o,
+                                                  uint32_t (&hm)[G][NW], bool owner, const ScanOut &o,
                                                   int *smem_scratch)
 {
     uint32_t any[NW];
@@ -208,7 +211,7 @@ __device__ __forceinline__ void compact_and_store(const Shape &s, int unit, int 
         c = block_sum(c, smem_scratch + 32);
         if (threadIdx.x == 0) cnt[1 + g] = c;
     }
-    if (o.member_out) {
+    if (o.member_out && owner) {
         const int b = unit / s.Hkv, kvh = unit % s.Hkv;
 #pragma unroll
         for (int w = 0; w < NW; w++) {
@@ -223,22 +226,63 @@ __device__ __forceinline__ void compact_and_store(const Shape &s, int unit, int 
     }
 }
 
+// Table-split partial counters: thread (ts, tg) with ts > 0 leaves its two
+// bit-sliced counters (seen >= 1, seen >= 2) for its token group in shared
+// memory; the ts == 0 thread of the same group folds them in:
+//   s2 = s2 | s2' | (s1 & s1'),  s1 = s1 | s1'.
+template <int G, int NW>
+__device__ __forceinline__ void combine_splits(uint32_t (&s1)[G][NW], uint32_t (&s2)[G][NW], uint32_t *part, int ts,
+                                               int tg)
+{
+    constexpr int TG = kScanThreads / kScanSplits;
+    if (ts > 0) {
+#pragma unroll
+        for (int g = 0; g < G; g++)
+#pragma unroll
+            for (int j = 0; j < NW; j++) {
+                part[((g * NW + j) * 2 + 0) * kScanThreads + threadIdx.x] = s1[g][j];
+                part[((g * NW + j) * 2 + 1) * kScanThreads + threadIdx.x] = s2[g][j];
+            }
+    }
+    __syncthreads();
+    if (ts == 0) {
+#pragma unroll 1
+        for (int t = 1; t < kScanSplits; t++) {
+#pragma unroll
+            for (int g = 0; g < G; g++)
+#pragma unroll
+                for (int j = 0; j < NW; j++) {
+                    const uint32_t a1 = part[((g * NW + j) * 2 + 0) * kScanThreads + t * TG + tg];
+                    const uint32_t a2 = part[((g * NW + j) * 2 + 1) * kScanThreads + t * TG + tg];
+                    s2[g][j] |= a2 | (s1[g][j] & a1);
+                    s1[g][j] |= a1;
+                }
+        }
+    }
+}
+
 // ---------------------------------------------------------- scan, K = 8 ----
-// Byte codes [unit][L][Ncap].  Thread = 16 consecutive tokens (one 16-byte
-// load per table); 128 threads = one 2048-token chunk.  Per 4-token word and
+// Byte codes [unit][L][Ncap].  A 1024-token chunk per block of 256 threads:
+// 64 token groups of 16 tokens (one 16-byte load per table) x 4 table splits
+// (tables ts, ts + 4, ...), merged in shared memory.  Per 4-token word and
 // head: x = codes ^ (qcode * 0x01010101); a byte of x is zero iff that token
 // matches.  Zero bytes are found exactly with ((x & 0x7f..) + 0x7f..) | x,
 // whose byte top bit is 1 iff the byte is non-zero.  Two bit-sliced counters
 // (seen >= 1, seen >= 2) live in the byte top bits.
 template <int G>
-__global__ void __launch_bounds__(kScanThreadsK8) scan_k8_kernel(
+__global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
     Shape s, const uint8_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
     const int32_t *__restrict__ seq_lens, int max_len, int nchunk, ScanOut o)
 {
-    extern __shared__ uint32_t rep[];  // [L][G] query code replicated in 4 bytes
+    extern __shared__ uint32_t dyn[];  // rep [L][G] (query code in 4 bytes), then split partials
+    uint32_t *rep = dyn;
+    uint32_t *part = dyn + ((s.L * G + 3) & ~3);
     __shared__ int scratch[64];
+    constexpr int TG = kScanThreads / kScanSplits;
+    const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
     const int unit = blockIdx.y, chunk = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
+    grid_dependency_wait();
     const int N = clamp_len(seq_lens, b, max_len, o.status, chunk == 0 && kvh == 0 && threadIdx.x == 0);
     const int c0 = chunk * kChunkK8;
     if (c0 >= N) return;
@@ -248,7 +292,7 @@ __global__ void __launch_bounds__(kScanThreadsK8) scan_k8_kernel(
     }
     __syncthreads();
 
-    const int t0 = c0 + threadIdx.x * 16;
+    const int t0 = c0 + tg * 16;
     uint32_t s1[G][4], s2[G][4];
 #pragma unroll
     for (int g = 0; g < G; g++)
@@ -258,7 +302,7 @@ __global__ void __launch_bounds__(kScanThreadsK8) scan_k8_kernel(
     if (t0 < N) {
         const uint8_t *base = codes + (size_t)unit * s.L * s.Ncap + t0;
 #pragma unroll 4
-        for (int l = 0; l < s.L; l++) {
+        for (int l = ts; l < s.L; l += kScanSplits) {
             const uint4 w4 = ld_stream_16(base + (size_t)l * s.Ncap);
             const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
@@ -274,6 +318,7 @@ __global__ void __launch_bounds__(kScanThreadsK8) scan_k8_kernel(
             }
         }
     }
+    combine_splits<G, 4>(s1, s2, part, ts, tg);
     // Per-head 16-bit token masks from the byte top bits of the >= 2 counter.
     uint32_t hm[G][1];
 #pragma unroll
@@ -281,28 +326,34 @@ __global__ void __launch_bounds__(kScanThreadsK8) scan_k8_kernel(
         uint32_t m = 0u;
 #pragma unroll
         for (int i = 0; i < 16; i++) m |= ((s2[g][i >> 2] >> (8 * (i & 3) + 7)) & 1u) << i;
-        hm[g][0] = m;
+        hm[g][0] = ts == 0 ? m : 0u;
     }
     // Tokens eligible for S: [sink, N - window) and below N.
     compact_and_store<G, 1, 16>(s, unit, chunk, nchunk, kChunkK8, t0, N, s.sink, min(N - s.window, N), hm,
-                                o, scratch);
+                                ts == 0, o, scratch);
 }
 
 // --------------------------------------------------------- scan, K = 10 ----
-// Bit-plane codes [unit][L][K][Ncap/32] (uint32).  Thread = 128 tokens (one
-// 16-byte load per plane); 64 threads = one 8192-token chunk.  A token
-// mismatches table l for head h iff some plane differs from the query bit:
-// mis = OR_b (plane_b ^ qmask_b), qmask_b = 0 or ~0 from shared memory.
+// Bit-plane codes [unit][L][K][Ncap/32] (uint32).  An 8192-token chunk per
+// block of 256 threads: 64 token groups of 128 tokens (one 16-byte load per
+// plane) x 4 table splits.  A token mismatches table l for head h iff some
+// plane differs from the query bit: mis = OR_b (plane_b ^ qmask_b), with
+// qmask_b = 0 or ~0 from shared memory.
 template <int G>
-__global__ void __launch_bounds__(kScanThreadsK10) scan_k10_kernel(
+__global__ void __launch_bounds__(kScanThreads) scan_k10_kernel(
     Shape s, const uint32_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
     const int32_t *__restrict__ seq_lens, int max_len, int nchunk, ScanOut o)
 {
-    extern __shared__ uint32_t qm[];  // [L][G][12]: qmask of the 10 planes, padded to 12
+    extern __shared__ uint32_t dyn[];  // qm [L][G][12] (qmask of the 10 planes, padded), then split partials
+    uint32_t *qm = dyn;
+    uint32_t *part = dyn + s.L * G * 12;
     __shared__ int scratch[64];
     constexpr int KB = 10;
+    constexpr int TG = kScanThreads / kScanSplits;
+    const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
     const int unit = blockIdx.y, chunk = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
+    grid_dependency_wait();
     const int N = clamp_len(seq_lens, b, max_len, o.status, chunk == 0 && kvh == 0 && threadIdx.x == 0);
     const int c0 = chunk * kChunkK10;
     if (c0 >= N) return;
@@ -313,7 +364,7 @@ __global__ void __launch_bounds__(kScanThreadsK10) scan_k10_kernel(
     }
     __syncthreads();
 
-    const int t0 = c0 + threadIdx.x * 128;
+    const int t0 = c0 + tg * 128;
     const int words = s.Ncap >> 5;
     uint32_t s1[G][4], s2[G][4];
 #pragma unroll
@@ -324,7 +375,7 @@ __global__ void __launch_bounds__(kScanThreadsK10) scan_k10_kernel(
     if (t0 < N) {
         const uint32_t *base = codes + (size_t)unit * s.L * KB * words + (t0 >> 5);
 #pragma unroll 1
-        for (int l = 0; l < s.L; l++) {
+        for (int l = ts; l < s.L; l += kScanSplits) {
             uint4 pl[KB];
 #pragma unroll
             for (int bb = 0; bb < KB; bb++) pl[bb] = ld_stream_16(base + ((size_t)l * KB + bb) * words);
@@ -349,8 +400,15 @@ __global__ void __launch_bounds__(kScanThreadsK10) scan_k10_kernel(
             }
         }
     }
+    combine_splits<G, 4>(s1, s2, part, ts, tg);
+    if (ts != 0) {
+#pragma unroll
+        for (int g = 0; g < G; g++)
+#pragma unroll
+            for (int j = 0; j < 4; j++) s2[g][j] = 0u;
+    }
     compact_and_store<G, 4, 32>(s, unit, chunk, nchunk, kChunkK10, t0, N, s.sink, min(N - s.window, N), s2,
-                                o, scratch);
+                                ts == 0, o, scratch);
 }
 
 // ---------------------------------------------------------------- attend ----
@@ -396,10 +454,11 @@ struct AttendArgs {
     const int32_t *seq_lens;
     int max_len;
     int nchunk;
+    int subs;   // blocks per scan chunk (each takes an equal share of its candidate list)
     int chunk_tokens;
     const uint32_t *cand;
     const int32_t *cnt;
-    float *pm, *pl, *pacc;  // [B*Hq][nchunk+1], [..][..][128]
+    float *pm, *pl, *pacc;  // [B*Hq][nchunk*subs+1], [..][..][128]
     LogU lu;
     float scale;  // 1/sqrt(d)
 };
@@ -412,17 +471,21 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
     __shared__ float nrm[4][16];          // per warp: |k|^2
     __shared__ uint32_t meta[kAttStages][kAttRows];  // headmask | exact << 8
     __shared__ float qinv[G];
+    __shared__ uint8_t upairs[4][16 * G];             // per warp: (row, head) pairs that need log u
 
     const Shape &s = a.s;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int unit = blockIdx.y, split = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
+    grid_dependency_wait();
     int N = a.seq_lens[b];
     N = N < 0 ? 0 : (N > a.max_len ? a.max_len : N);
-    const bool dsplit = split == a.nchunk;
-    if (!dsplit && split * a.chunk_tokens >= N) return;
+    const bool dsplit = split == a.nchunk * a.subs;
+    const int chunk = split / a.subs, sub = split % a.subs;
+    if (!dsplit && chunk * a.chunk_tokens >= N) return;
 
-    // Rows of this split: compacted candidates, or the exact set D.
+    // Rows of this block: its share of a chunk's compacted candidates, or the
+    // exact set D.
     const int n_sink = min(s.sink, N);
     const int win0 = max(n_sink, N - s.window);
     int nrows;
@@ -430,8 +493,11 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
     if (dsplit) {
         nrows = n_sink + (N - win0);
     } else {
-        nrows = a.cnt[((size_t)unit * a.nchunk + split) * 16];
-        list = a.cand + ((size_t)unit * a.nchunk + split) * a.chunk_tokens;
+        const int total = a.cnt[((size_t)unit * a.nchunk + chunk) * 16];
+        const int per = (total + a.subs - 1) / a.subs;
+        const int e0 = min(total, sub * per);
+        nrows = min(total, e0 + per) - e0;
+        list = a.cand + ((size_t)unit * a.nchunk + chunk) * a.chunk_tokens + e0;
     }
     auto row_of = [&](int e, uint32_t &m) -> int {
         if (dsplit) {
@@ -561,20 +627,31 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
         __syncwarp();
 
         // ---- log-weights t = s (exact) or s - log u (sampled), -inf if absent ----
-        for (int p = lane; p < 16 * G; p += 32) {
-            const int r = p / G, h = p % G;
-            const uint32_t m = meta[stage][warp * 16 + r];
-            float tv = -INFINITY;
-            if ((m >> h) & 1u) {
-                const float raw = sc[warp][r][h];
-                tv = raw * a.scale;
-                if (!(m & 0x100u)) {
-                    const float kk = nrm[warp][r];
-                    const float cosv = kk > 0.f ? raw * qinv[h] * rsqrtf(kk) : 0.f;
-                    tv -= log_sampling_prob(cosv, a.lu);
-                }
+        // The (row, head) pairs that need log u are compacted first so that the
+        // transcendental work runs on sampled pairs only.
+        int nu = 0;
+        for (int p0 = 0; p0 < 16 * G; p0 += 32) {
+            const int p = p0 + lane;
+            bool need = false;
+            if (p < 16 * G) {
+                const int r = p / G, h = p % G;
+                const uint32_t m = meta[stage][warp * 16 + r];
+                const bool mem = (m >> h) & 1u;
+                need = mem && !(m & 0x100u);
+                sc[warp][r][h] = mem ? sc[warp][r][h] * a.scale : -INFINITY;
             }
-            sc[warp][r][h] = tv;
+            const uint32_t bal = __ballot_sync(0xffffffffu, need);
+            if (need) upairs[warp][nu + __popc(bal & ((1u << lane) - 1u))] = (uint8_t)p;
+            nu += __popc(bal);
+        }
+        __syncwarp();
+        for (int j = lane; j < nu; j += 32) {
+            const int p = upairs[warp][j];
+            const int r = p / G, h = p % G;
+            const float kk = nrm[warp][r];
+            const float sv = sc[warp][r][h];  // already scaled by 1/sqrt(d)
+            const float cosv = kk > 0.f ? sv * (1.f / a.scale) * qinv[h] * rsqrtf(kk) : 0.f;
+            sc[warp][r][h] = sv - log_sampling_prob(cosv, a.lu);
         }
         __syncwarp();
 
@@ -655,7 +732,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
             }
         }
         const size_t bh = vec0 + g;
-        const size_t pidx = bh * (a.nchunk + 1) + split;
+        const size_t pidx = bh * ((size_t)a.nchunk * a.subs + 1) + split;
         a.pacc[pidx * kHeadDim + dim] = A;
         if (dim == 0) {
             a.pm[pidx] = M;
@@ -667,7 +744,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
 // ----------------------------------------------------------------- merge ----
 template <int G>
 __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t *__restrict__ seq_lens,
-                                                         int max_len, int nchunk, int chunk_tokens,
+                                                         int max_len, int nchunk, int subs, int chunk_tokens,
                                                          const float *__restrict__ pm,
                                                          const float *__restrict__ pl,
                                                          const float *__restrict__ pacc,
@@ -677,14 +754,15 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
     const int bh = blockIdx.x;
     const int b = bh / s.Hq, h = bh % s.Hq, kvh = h / G, g = h % G;
     const int unit = b * s.Hkv + kvh;
+    grid_dependency_wait();
     int N = seq_lens[b];
     N = N < 0 ? 0 : (N > max_len ? max_len : N);
-    const int nch = (N + chunk_tokens - 1) / chunk_tokens;
+    const int nsp = ((N + chunk_tokens - 1) / chunk_tokens) * subs;  // live chunk splits
+    const int dsp = nchunk * subs;                                    // the exact-set split
     const int dim = threadIdx.x;
-    const size_t base = (size_t)bh * (nchunk + 1);
-    float M = -INFINITY;
-    for (int j = 0; j < nch; j++) M = fmaxf(M, pm[base + j]);
-    M = fmaxf(M, pm[base + nchunk]);
+    const size_t base = (size_t)bh * (dsp + 1);
+    float M = pm[base + dsp];
+    for (int j = 0; j < nsp; j++) M = fmaxf(M, pm[base + j]);
     float Ls = 0.f, A = 0.f;
     if (M != -INFINITY) {
         auto add = [&](int j) {
@@ -694,14 +772,14 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
             Ls += pl[base + j] * f;
             A += pacc[(base + j) * kHeadDim + dim] * f;
         };
-        for (int j = 0; j < nch; j++) add(j);
-        add(nchunk);
+        for (int j = 0; j < nsp; j++) add(j);
+        add(dsp);
     }
     out[(size_t)bh * kHeadDim + dim] = Ls > 0.f ? A / Ls : 0.f;
     if (dim == 0) {
         lse[bh] = Ls > 0.f ? M + logf(Ls) : -INFINITY;
         int ns = 0;
-        for (int j = 0; j < nch; j++) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
+        for (int j = 0; j < nsp / subs; j++) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
         n_sampled[bh] = ns;
     }
 }
@@ -718,10 +796,20 @@ struct Workspace {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Attention blocks per scan chunk: enough blocks for two waves on 148 SMs
+// (a fixed count, so the workspace size does not depend on the device).
+static int attend_subs(const Shape &s, int nchunk)
+{
+    const int blocks = nchunk * s.B * s.Hkv;
+    if (blocks == 0) return 1;
+    return std::max(1, std::min(8, (296 + blocks - 1) / blocks));
+}
+
 Workspace workspace_layout(const Shape &s, int max_len, void *base)
 {
     const int C = chunk_tokens(s.K);
     const int nchunk = (max_len + C - 1) / C;
+    const size_t nsplit = (size_t)nchunk * attend_subs(s, nchunk) + 1;
     const size_t units = (size_t)s.B * s.Hkv, bh = (size_t)s.B * s.Hq;
     size_t off = 0;
     Workspace w{};
@@ -735,9 +823,9 @@ Workspace workspace_layout(const Shape &s, int max_len, void *base)
     w.qcodes = reinterpret_cast<uint16_t *>(take(bh * s.L * sizeof(uint16_t)));
     w.cand = reinterpret_cast<uint32_t *>(take(units * nchunk * (size_t)C * sizeof(uint32_t)));
     w.cnt = reinterpret_cast<int32_t *>(take(units * nchunk * 16 * sizeof(int32_t)));
-    w.pm = reinterpret_cast<float *>(take(bh * (nchunk + 1) * sizeof(float)));
-    w.pl = reinterpret_cast<float *>(take(bh * (nchunk + 1) * sizeof(float)));
-    w.pacc = reinterpret_cast<float *>(take(bh * (nchunk + 1) * kHeadDim * sizeof(float)));
+    w.pm = reinterpret_cast<float *>(take(bh * nsplit * sizeof(float)));
+    w.pl = reinterpret_cast<float *>(take(bh * nsplit * sizeof(float)));
+    w.pacc = reinterpret_cast<float *>(take(bh * nsplit * kHeadDim * sizeof(float)));
     w.bytes = off;
     return w;
 }
@@ -765,24 +853,33 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
 {
     const int C = chunk_tokens(s.K);
     const int nchunk = (max_len + C - 1) / C;
+    const int subs = attend_subs(s, nchunk);
     const int units = s.B * s.Hkv;
+    cudaError_t e;
     {
         dim3 grid((s.L + 256 / s.K - 1) / (256 / s.K), units);
-        qhash_kernel<G><<<grid, 256, 0, st>>>(s, q, W, dbg ? dbg->qcodes_in : nullptr, ws.qcodes, ws.status);
+        e = launch_pdl(qhash_kernel<G>, grid, dim3(256), 0, st, s, q, W,
+                       (const uint16_t *)(dbg ? dbg->qcodes_in : nullptr), ws.qcodes, ws.status);
+        if (e != cudaSuccess) return e;
     }
     ScanOut so{ws.cand, ws.cnt, dbg ? dbg->member_out : nullptr, ws.status};
     if (nchunk > 0) {
         dim3 grid(nchunk, units);
+        const size_t part = (size_t)2 * G * 4 * kScanThreads * sizeof(uint32_t);
         if (s.K == 8) {
-            const size_t sm = (size_t)s.L * G * sizeof(uint32_t);
-            scan_k8_kernel<G><<<grid, kScanThreadsK8, sm, st>>>(s, static_cast<const uint8_t *>(codes), ws.qcodes,
-                                                                seq_lens, max_len, nchunk, so);
+            const size_t sm = (size_t)((s.L * G + 3) & ~3) * sizeof(uint32_t) + part;
+            if ((e = ensure_smem(reinterpret_cast<const void *>(scan_k8_kernel<G>), (int)sm)) != cudaSuccess) return e;
+            e = launch_pdl(scan_k8_kernel<G>, grid, dim3(kScanThreads), sm, st, s,
+                           static_cast<const uint8_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
+                           nchunk, so);
         } else {
-            const size_t sm = (size_t)s.L * G * 12 * sizeof(uint32_t);
-            ensure_smem(reinterpret_cast<const void *>(scan_k10_kernel<G>), (int)sm);
-            scan_k10_kernel<G><<<grid, kScanThreadsK10, sm, st>>>(s, static_cast<const uint32_t *>(codes),
-                                                                  ws.qcodes, seq_lens, max_len, nchunk, so);
+            const size_t sm = (size_t)s.L * G * 12 * sizeof(uint32_t) + part;
+            if ((e = ensure_smem(reinterpret_cast<const void *>(scan_k10_kernel<G>), (int)sm)) != cudaSuccess) return e;
+            e = launch_pdl(scan_k10_kernel<G>, grid, dim3(kScanThreads), sm, st, s,
+                           static_cast<const uint32_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
+                           nchunk, so);
         }
+        if (e != cudaSuccess) return e;
     }
     AttendArgs aa;
     aa.s = s;
@@ -792,6 +889,7 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     aa.seq_lens = seq_lens;
     aa.max_len = max_len;
     aa.nchunk = nchunk;
+    aa.subs = subs;
     aa.chunk_tokens = C;
     aa.cand = ws.cand;
     aa.cnt = ws.cnt;
@@ -802,16 +900,18 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     aa.scale = 1.0f / sqrtf((float)s.d);
     {
         const int sm = kAttStages * kStageBytes;
-        ensure_smem(reinterpret_cast<const void *>(attend_kernel<G>), sm);
-        dim3 grid(nchunk + 1, units);
-        attend_kernel<G><<<grid, kAttThreads, sm, st>>>(aa);
+        if ((e = ensure_smem(reinterpret_cast<const void *>(attend_kernel<G>), sm)) != cudaSuccess) return e;
+        dim3 grid(nchunk * subs + 1, units);
+        if ((e = launch_pdl(attend_kernel<G>, grid, dim3(kAttThreads), sm, st, aa)) != cudaSuccess) return e;
     }
-    merge_kernel<G><<<s.B * s.Hq, kHeadDim, 0, st>>>(s, seq_lens, max_len, nchunk, C, ws.pm, ws.pl, ws.pacc,
-                                                     ws.cnt, out, lse, n_sampled);
+    e = launch_pdl(merge_kernel<G>, dim3(s.B * s.Hq), dim3(kHeadDim), 0, st, s, seq_lens, max_len, nchunk, subs, C,
+                   (const float *)ws.pm, (const float *)ws.pl, (const float *)ws.pacc, (const int32_t *)ws.cnt, out,
+                   lse, n_sampled);
+    if (e != cudaSuccess) return e;
     if (dbg && dbg->qcodes_out)
-        cudaMemcpyAsync(dbg->qcodes_out, ws.qcodes, (size_t)s.B * s.Hq * s.L * sizeof(uint16_t),
-                        cudaMemcpyDeviceToDevice, st);
-    return cudaGetLastError();
+        e = cudaMemcpyAsync(dbg->qcodes_out, ws.qcodes, (size_t)s.B * s.Hq * s.L * sizeof(uint16_t),
+                            cudaMemcpyDeviceToDevice, st);
+    return e;
 }
 
 cudaError_t launch_decode(const Shape &s, const uint16_t *q, const uint16_t *W, const void *codes,
@@ -833,14 +933,15 @@ cudaError_t launch_hash_queries(const Shape &s, const uint16_t *q, const uint16_
                                 cudaStream_t st)
 {
     dim3 grid((s.L + 256 / s.K - 1) / (256 / s.K), s.B * s.Hkv);
+    const uint16_t *none = nullptr;
+    int32_t *no_status = nullptr;
     switch (s.G) {
-    case 1: qhash_kernel<1><<<grid, 256, 0, st>>>(s, q, W, nullptr, qcodes, nullptr); break;
-    case 2: qhash_kernel<2><<<grid, 256, 0, st>>>(s, q, W, nullptr, qcodes, nullptr); break;
-    case 4: qhash_kernel<4><<<grid, 256, 0, st>>>(s, q, W, nullptr, qcodes, nullptr); break;
-    case 8: qhash_kernel<8><<<grid, 256, 0, st>>>(s, q, W, nullptr, qcodes, nullptr); break;
+    case 1: return launch_pdl(qhash_kernel<1>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status);
+    case 2: return launch_pdl(qhash_kernel<2>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status);
+    case 4: return launch_pdl(qhash_kernel<4>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status);
+    case 8: return launch_pdl(qhash_kernel<8>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status);
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace mp

@@ -1,6 +1,6 @@
-// SimHash of cached keys and decode-time append (MagicPIG, Chen et al. 2024;
+// Decode-time append: one new token per sequence (MagicPIG, Chen et al. 2024;
 // the gitdiagram page's "LSH Sampling" component: LSH kernel behind an LSH
-// interface; the sourcepulse page's note on optimized hash table construction).
+// interface).  The bulk key hash is the tensor-core kernel in mp_hash_tc.cu.
 //
 // Code layouts (table-major, exactly L*K/8 bytes per token):
 //   K = 8 : uint8  [unit][L][Ncap], bit b of the byte = bit b of the code.
@@ -10,86 +10,11 @@
 
 namespace mp {
 
-// ------------------------------------------------------------ hash keys ----
-// Thread = one key row (fp32 copy in registers); 128 rows per block.  Each
-// hyperplane row of W is read by all threads of a warp at once (a broadcast).
-// Bit = (sum_j k_j w_j > 0) with an fp32 sum of exact bf16 products in
-// ascending j.  K = 10 bit planes come straight from a warp ballot: the 32
-// lanes of a warp are 32 consecutive tokens.
-__global__ void __launch_bounds__(128) hash_keys_simt_kernel(Shape s, const uint16_t *__restrict__ keys,
-                                                             const uint16_t *__restrict__ W,
-                                                             const int32_t *__restrict__ seq_lens, int n_tokens,
-                                                             void *codes)
-{
-    const int unit = blockIdx.y;
-    if (seq_lens) {
-        const int nb = seq_lens[unit / s.Hkv];
-        n_tokens = min(n_tokens, max(nb, 0));
-    }
-    if ((int)blockIdx.x * 128 >= n_tokens) return;
-    const int tok = blockIdx.x * 128 + threadIdx.x;
-    const bool valid = tok < n_tokens;
-    float k[kHeadDim];
-    {
-        const uint4 *kr = reinterpret_cast<const uint4 *>(keys + ((size_t)unit * s.Ncap + tok) * kHeadDim);
-#pragma unroll
-        for (int j8 = 0; j8 < kHeadDim / 8; j8++) {
-            const uint4 v = kr[j8];
-            k[j8 * 8 + 0] = bf16_lo(v.x);
-            k[j8 * 8 + 1] = bf16_hi(v.x);
-            k[j8 * 8 + 2] = bf16_lo(v.y);
-            k[j8 * 8 + 3] = bf16_hi(v.y);
-            k[j8 * 8 + 4] = bf16_lo(v.z);
-            k[j8 * 8 + 5] = bf16_hi(v.z);
-            k[j8 * 8 + 6] = bf16_lo(v.w);
-            k[j8 * 8 + 7] = bf16_hi(v.w);
-        }
-    }
-    const int words = s.Ncap >> 5;
-    for (int l = 0; l < s.L; l++) {
-        unsigned code = 0;
-        for (int bb = 0; bb < s.K; bb++) {
-            const int c = l * s.K + bb;
-            const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)c * kHeadDim);
-            float dot = 0.f;
-#pragma unroll
-            for (int j8 = 0; j8 < kHeadDim / 8; j8++) {
-                const uint4 w = __ldg(wr + j8);
-                dot = fmaf(k[j8 * 8 + 0], bf16_lo(w.x), dot);
-                dot = fmaf(k[j8 * 8 + 1], bf16_hi(w.x), dot);
-                dot = fmaf(k[j8 * 8 + 2], bf16_lo(w.y), dot);
-                dot = fmaf(k[j8 * 8 + 3], bf16_hi(w.y), dot);
-                dot = fmaf(k[j8 * 8 + 4], bf16_lo(w.z), dot);
-                dot = fmaf(k[j8 * 8 + 5], bf16_hi(w.z), dot);
-                dot = fmaf(k[j8 * 8 + 6], bf16_lo(w.w), dot);
-                dot = fmaf(k[j8 * 8 + 7], bf16_hi(w.w), dot);
-            }
-            const bool bit = valid && dot > 0.f;
-            if (s.K == 10) {
-                const uint32_t word = __ballot_sync(0xffffffffu, bit);
-                if ((threadIdx.x & 31) == 0 && tok - (int)(threadIdx.x & 31) < n_tokens)
-                    static_cast<uint32_t *>(codes)[((size_t)unit * s.L * s.K + c) * words + (tok >> 5)] = word;
-            } else {
-                code |= (unsigned)bit << bb;
-            }
-        }
-        if (s.K == 8 && valid) static_cast<uint8_t *>(codes)[((size_t)unit * s.L + l) * s.Ncap + tok] = (uint8_t)code;
-    }
-}
-
-cudaError_t launch_hash_keys(const Shape &s, const uint16_t *keys, const uint16_t *W, const int32_t *seq_lens,
-                             int n_tokens, void *codes, cudaStream_t st)
-{
-    if (n_tokens == 0) return cudaSuccess;
-    dim3 grid((n_tokens + 127) / 128, s.B * s.Hkv);
-    hash_keys_simt_kernel<<<grid, 128, 0, st>>>(s, keys, W, seq_lens, n_tokens, codes);
-    return cudaGetLastError();
-}
-
 // --------------------------------------------------------------- append ----
 // grid (ceil(L / TB), B * Hkv), 256 threads: thread = one hyperplane column of a
-// block of TB = 256 / K whole tables.  Same fp32 ascending-j projection as the
-// key hash, so an appended token gets the codes a full re-hash would give.
+// block of TB = 256 / K whole tables, projection = fp32 sum of exact bf16
+// products in ascending j (bits can differ from the tensor-core hash only where
+// the projection is within fp32 rounding of zero).
 __global__ void __launch_bounds__(256) append_kernel(Shape s, const uint16_t *__restrict__ k_new,
                                                      const uint16_t *__restrict__ v_new,
                                                      const uint16_t *__restrict__ W, uint16_t *kc, uint16_t *vc,
@@ -101,6 +26,7 @@ __global__ void __launch_bounds__(256) append_kernel(Shape s, const uint16_t *__
     const int tid = threadIdx.x;
     const int unit = blockIdx.y;
     const int b = unit / s.Hkv;
+    grid_dependency_wait();
     const int pos = seq_lens[b];
     if (pos < 0 || pos >= s.Ncap) {
         if (blockIdx.x == 0 && unit % s.Hkv == 0 && tid == 0) set_status(status, MP_ERR_CAPACITY);
@@ -158,6 +84,7 @@ __global__ void __launch_bounds__(256) append_kernel(Shape s, const uint16_t *__
 
 __global__ void bump_lengths_kernel(int B, int Ncap, int32_t *seq_lens)
 {
+    grid_dependency_wait();
     for (int b = threadIdx.x; b < B; b += blockDim.x) {
         const int p = seq_lens[b];
         if (p >= 0 && p < Ncap) seq_lens[b] = p + 1;
@@ -170,9 +97,10 @@ cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t 
 {
     const int TB = 256 / s.K;
     dim3 grid((s.L + TB - 1) / TB, s.B * s.Hkv);
-    append_kernel<<<grid, 256, 0, st>>>(s, k_new, v_new, W, kc, vc, codes, seq_lens, status);
-    bump_lengths_kernel<<<1, 256, 0, st>>>(s.B, s.Ncap, seq_lens);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(append_kernel, grid, dim3(256), 0, st, s, k_new, v_new, W, kc, vc, codes,
+                               (const int32_t *)seq_lens, status);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(bump_lengths_kernel, dim3(1), dim3(256), 0, st, s.B, s.Ncap, seq_lens);
 }
 
 }  // namespace mp

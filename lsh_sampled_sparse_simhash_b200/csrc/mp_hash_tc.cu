@@ -1,0 +1,465 @@
+// SimHash of cached keys on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// The projection of every key row onto the L*K hyperplanes of W is a dense
+// bf16 contraction (rows x 128) . (128 x L*K) with fp32 accumulation, so it
+// runs as a persistent, warp-specialised GEMM whose epilogue never writes the
+// fp32 product: it turns each accumulator value into a sign bit (strictly
+// positive -> 1, the SimHash rule of MagicPIG, Chen et al. 2024) and packs the
+// bits straight into the table-major code layout.
+//
+//   warp 0      TMA producer: the W column group (resident in shared memory,
+//               reloaded only when a CTA moves to the next group) and a
+//               2-stage ring of 128-row key tiles, 128B-swizzled.
+//   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, M = 128,
+//               N <= 128, K = 16, into one of four TMEM accumulators.
+//   warp 2      TMEM allocator (512 columns = 4 x 128-column accumulators).
+//   warps 4..11 epilogue, two groups of four warps taking alternate column
+//               tiles: tcgen05.ld 32x32b (thread = key row, registers =
+//               columns, 64 columns per wait), sign test, pack, store.
+//               K = 8: one byte per (table, token); K = 10: one warp ballot
+//               per column gives the 32-token bit-plane word.
+//
+// Column groups: W has L*K rows (hyperplanes); a group of at most 640 rows
+// (608 for K = 8, L = 75) stays resident; K = 10, L = 150 uses 3 groups of
+// <= 512 and re-reads each key tile once per group.
+//
+// Every wait on an mbarrier is bounded (1 s of %globaltimer); on expiry the
+// kernel records MP_ERR_CUDA in the status word, skips the rest of its work,
+// waits (bounded) for its own copies and MMAs in flight, frees TMEM and exits.
+#include <cuda.h>
+
+#include "mp_common.cuh"
+#include "mp_kernels.cuh"
+
+namespace mp {
+namespace tc {
+
+constexpr int kThreads = 384;
+constexpr int kBM = 128;                     // key rows per tile = TMEM lanes
+constexpr int kAccCols = 128;                // columns per accumulator buffer
+constexpr int kAccBufs = 4;                  // 4 x 128 = all 512 TMEM columns
+constexpr int kStages = 2;                   // key-tile ring depth
+constexpr int kHalfBytes = kBM * 128;        // one 64-element (128 B) K half of a tile
+constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KB
+constexpr int kMaxGroupCols = 640;
+constexpr int kWBox = 32;                    // W rows per TMA box
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+struct Params {
+    Shape s;
+    const int32_t *seq_lens;
+    void *codes;
+    int32_t *status;
+    int n_tokens;
+    int n_mt;        // 128-row tiles per unit
+    int ngroups;
+    int gsize;       // columns per group (multiple of 32)
+    int gpad_max;    // padded width of the widest group (multiple of 32)
+    int total_items; // ngroups * units * n_mt
+};
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t a)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase of parity `parity`; false on abort or timeout.
+__device__ __noinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int *abort_flag, int32_t *status)
+{
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(a, parity)) {
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            set_status(status, MP_ERR_CUDA);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// K-major, 128B-swizzled operand: rows of 128 B, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// kind::f16 instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128.
+__device__ __forceinline__ uint32_t idesc_bf16(int n)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum)
+{
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+struct Item {
+    int group, unit, mt, len;
+    bool skip;
+};
+
+__device__ __forceinline__ Item item_of(const Params &p, int it)
+{
+    Item r;
+    const int units = p.s.B * p.s.Hkv;
+    r.group = it / (units * p.n_mt);
+    const int rem = it % (units * p.n_mt);
+    r.unit = rem / p.n_mt;
+    r.mt = rem % p.n_mt;
+    int len = p.n_tokens;
+    if (p.seq_lens) len = min(len, max(p.seq_lens[r.unit / p.s.Hkv], 0));
+    r.len = len;
+    r.skip = r.mt * kBM >= len;
+    return r;
+}
+
+// Columns [c0, c0 + width) of a group; width is a multiple of 32.
+__device__ __forceinline__ void group_cols(const Params &p, int g, int &c0, int &width)
+{
+    c0 = g * p.gsize;
+    const int real = min(p.gsize, p.s.LK - c0);
+    width = (real + 31) & ~31;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    hash_keys_tc_kernel(const __grid_constant__ CUtensorMap tmap_keys, const __grid_constant__ CUtensorMap tmap_w,
+                        const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[16];  // 15 used
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile int abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    grid_dependency_wait();
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t w_half = (uint32_t)p.gpad_max * 128u;  // bytes of one K half of W
+    const uint32_t w_smem = base;
+    const uint32_t a_smem = base + 2u * w_half;
+    // barriers
+    const uint32_t bar0 = smem_u32(&bars[0]);
+    auto full_a = [&](int s) { return bar0 + 8u * s; };            // 0,1
+    auto empty_a = [&](int s) { return bar0 + 8u * (2 + s); };     // 2,3
+    auto tmem_full = [&](int b) { return bar0 + 8u * (4 + b); };   // 4..7
+    auto tmem_empty = [&](int b) { return bar0 + 8u * (8 + b); };  // 8..11
+    const uint32_t w_full = bar0 + 8u * 12, w_empty = bar0 + 8u * 13, final_bar = bar0 + 8u * 14;
+
+    if (tid == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < kStages; s++) {
+            mbar_init(full_a(s), 1);
+            mbar_init(empty_a(s), 1);
+        }
+        for (int b = 0; b < kAccBufs; b++) {
+            mbar_init(tmem_full(b), 1);
+            mbar_init(tmem_empty(b), 128);
+        }
+        mbar_init(w_full, 1);
+        mbar_init(w_empty, 1);
+        mbar_init(final_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
+                     "r"(kAccBufs * kAccCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+    const Shape &s = p.s;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------ producer ----
+        int stage = 0;
+        uint32_t empty_par[kStages] = {0, 0};
+        int last_issued_par[kStages] = {-1, -1};
+        int cur_g = -1, w_loads = 0;
+        for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
+            const Item im = item_of(p, it);
+            if (im.skip) continue;
+            if (im.group != cur_g) {
+                if (cur_g >= 0 && !mbar_wait(w_empty, (w_loads - 1) & 1, &abort_flag, p.status)) break;
+                int c0, width;
+                group_cols(p, im.group, c0, width);
+                mbar_expect_tx(w_full, (uint32_t)width * 256u);
+                for (int rb = 0; rb < width / kWBox; rb++)
+                    for (int kh = 0; kh < 2; kh++)
+                        tma_load_2d(w_smem + kh * w_half + rb * kWBox * 128, &tmap_w, w_full, kh * 64, c0 + rb * kWBox);
+                cur_g = im.group;
+                w_loads++;
+            }
+            if (!mbar_wait(empty_a(stage), empty_par[stage] ^ 1u, &abort_flag, p.status)) break;
+            empty_par[stage] ^= 1u;
+            const int row0 = im.unit * s.Ncap + im.mt * kBM;
+            mbar_expect_tx(full_a(stage), kTileBytes);
+            tma_load_2d(a_smem + stage * kTileBytes, &tmap_keys, full_a(stage), 0, row0);
+            tma_load_2d(a_smem + stage * kTileBytes + kHalfBytes, &tmap_keys, full_a(stage), 64, row0);
+            last_issued_par[stage] = (last_issued_par[stage] + 1) & 1;
+            stage ^= 1;
+        }
+        // our own copies in flight must land before the CTA exits
+        for (int st = 0; st < kStages; st++)
+            if (last_issued_par[st] >= 0) mbar_wait(full_a(st), (uint32_t)last_issued_par[st], &abort_flag, p.status);
+        if (w_loads > 0) mbar_wait(w_full, (w_loads - 1) & 1, &abort_flag, p.status);
+    } else if (warp == 1 && lane == 0) {
+        // ----------------------------------------------------------- MMA ----
+        int stage = 0, acc = 0;
+        uint32_t full_par[kStages] = {0, 0};
+        uint32_t tempty_par[kAccBufs] = {0, 0, 0, 0};
+        int cur_g = -1, w_uses = 0;
+        for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
+            const Item im = item_of(p, it);
+            if (im.skip) continue;
+            if (im.group != cur_g) {
+                if (cur_g >= 0) mma_commit(w_empty);  // W free once the MMAs so far complete
+                if (!mbar_wait(w_full, w_uses & 1, &abort_flag, p.status)) break;
+                cur_g = im.group;
+                w_uses++;
+            }
+            if (!mbar_wait(full_a(stage), full_par[stage], &abort_flag, p.status)) break;
+            full_par[stage] ^= 1u;
+            tc_fence_after();
+            int c0, width;
+            group_cols(p, im.group, c0, width);
+            bool ok = true;
+            for (int n0 = 0; n0 < width; n0 += kAccCols) {
+                const int nw = min(kAccCols, width - n0);
+                if (!mbar_wait(tmem_empty(acc), tempty_par[acc] ^ 1u, &abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tempty_par[acc] ^= 1u;
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(acc * kAccCols);
+                const uint32_t idesc = idesc_bf16(nw);
+#pragma unroll
+                for (int kh = 0; kh < 2; kh++) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ks++) {
+                        const uint64_t ad = sw128_desc(a_smem + stage * kTileBytes + kh * kHalfBytes + ks * 32);
+                        const uint64_t bd = sw128_desc(w_smem + kh * w_half + n0 * 128 + ks * 32);
+                        mma_bf16(d, ad, bd, idesc, (kh | ks) != 0);
+                    }
+                }
+                mma_commit(tmem_full(acc));
+                acc = (acc + 1) & (kAccBufs - 1);
+            }
+            if (!ok) break;
+            mma_commit(empty_a(stage));
+            stage ^= 1;
+        }
+        // every MMA issued so far has completed before TMEM is released
+        mma_commit(final_bar);
+        mbar_wait(final_bar, 0, &abort_flag, p.status);
+    } else if (warp >= 4) {
+        // ------------------------------------------------------ epilogue ----
+        const int q4 = warp & 3;         // TMEM lane quarter of this warp
+        const int eg = (warp - 4) >> 2;  // epilogue group: takes column tiles seq % 2 == eg
+        const int row = q4 * 32 + lane;
+        int seq = 0;                     // column-tile sequence number (all groups)
+        uint32_t tfull_par[kAccBufs] = {0, 0, 0, 0};
+        const int words = s.Ncap >> 5;
+        for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
+            const Item im = item_of(p, it);
+            if (im.skip) continue;
+            int c0, width;
+            group_cols(p, im.group, c0, width);
+            const int tok = im.mt * kBM + row;
+            const bool valid = tok < im.len;
+            const bool warp_live = im.mt * kBM + q4 * 32 < im.len;
+            bool ok = true;
+            for (int n0 = 0; n0 < width; n0 += kAccCols, seq++) {
+                if ((seq & 1) != eg) continue;
+                const int acc = seq & (kAccBufs - 1);
+                const int nw = min(kAccCols, width - n0);
+                if (!mbar_wait(tmem_full(acc), tfull_par[acc], &abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tfull_par[acc] ^= 1u;
+                tc_fence_after();
+                for (int ch = 0; ch < nw; ch += 64) {
+                    uint32_t v[64];
+                    const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kAccCols + ch);
+                    tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                    const bool two = ch + 32 < nw;
+                    if (two) tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int half = 0; half < 2; half++) {
+                        if (half == 1 && !two) break;
+                        const uint32_t *vv = v + 32 * half;
+                        const int col0 = c0 + n0 + ch + 32 * half;  // first global column of these 32
+                        if (s.K == 8) {
+#pragma unroll
+                            for (int t = 0; t < 4; t++) {
+                                uint32_t byte = 0;
+#pragma unroll
+                                for (int bb = 0; bb < 8; bb++)
+                                    byte |= (__uint_as_float(vv[8 * t + bb]) > 0.f ? 1u : 0u) << bb;
+                                const int l = (col0 >> 3) + t;
+                                if (valid && l < s.L)
+                                    static_cast<uint8_t *>(p.codes)[((size_t)im.unit * s.L + l) * s.Ncap + tok] =
+                                        (uint8_t)byte;
+                            }
+                        } else {
+                            uint32_t mine = 0;
+#pragma unroll
+                            for (int j = 0; j < 32; j++) {
+                                const uint32_t wv = __ballot_sync(0xffffffffu, valid && __uint_as_float(vv[j]) > 0.f);
+                                if (lane == j) mine = wv;
+                            }
+                            const int c = col0 + lane;
+                            if (warp_live && c < s.LK)
+                                static_cast<uint32_t *>(p.codes)[((size_t)im.unit * s.L * s.K + c) * words +
+                                                                 ((im.mt * kBM + q4 * 32) >> 5)] = mine;
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(tmem_empty(acc));
+            }
+            if (!ok) break;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kAccBufs * kAccCols));
+    }
+}
+
+// ------------------------------------------------------------------ host ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 2-D bf16 row-major [rows][128] view, box = 64 elements x box_rows, 128B swizzle.
+static bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int num_sms()
+{
+    int dev = 0, n = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+}  // namespace tc
+
+cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint16_t *W, const int32_t *seq_lens,
+                                int n_tokens, void *codes, int32_t *status, cudaStream_t st)
+{
+    using namespace tc;
+    if (n_tokens == 0) return cudaSuccess;
+    Params p;
+    p.s = s;
+    p.seq_lens = seq_lens;
+    p.codes = codes;
+    p.status = status;
+    p.n_tokens = n_tokens;
+    p.n_mt = (n_tokens + kBM - 1) / kBM;
+    p.ngroups = (s.LK + kMaxGroupCols - 1) / kMaxGroupCols;
+    p.gsize = (((s.LK + p.ngroups - 1) / p.ngroups) + 31) & ~31;
+    p.gpad_max = p.gsize;
+    p.total_items = p.ngroups * s.B * s.Hkv * p.n_mt;
+    CUtensorMap mk, mw;
+    if (!make_map(&mk, keys, (uint64_t)s.B * s.Hkv * s.Ncap, kBM)) return cudaErrorInvalidValue;
+    if (!make_map(&mw, W, (uint64_t)s.LK, kWBox)) return cudaErrorInvalidValue;
+    const int smem = 1024 + 2 * p.gpad_max * 128 + kStages * kTileBytes;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(hash_keys_tc_kernel), smem);
+    if (e != cudaSuccess) return e;
+    const int grid = min(num_sms(), p.total_items);
+    return launch_pdl(hash_keys_tc_kernel, dim3(grid), dim3(kThreads), smem, st, mk, mw, p);
+}
+
+}  // namespace mp

@@ -6,8 +6,8 @@
 
 namespace mp {
 
-cudaError_t launch_hash_keys(const Shape &s, const uint16_t *keys, const uint16_t *W, const int32_t *seq_lens,
-                             int n_tokens, void *codes, cudaStream_t st);
+cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint16_t *W, const int32_t *seq_lens,
+                                int n_tokens, void *codes, int32_t *status, cudaStream_t st);
 cudaError_t launch_hash_queries(const Shape &s, const uint16_t *q, const uint16_t *W, uint16_t *qcodes,
                                 cudaStream_t st);
 cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t *v_new, const uint16_t *W,
@@ -21,5 +21,26 @@ size_t decode_workspace_bytes(const Shape &s, int max_len);
 
 // Raises the dynamic shared-memory limit of `func` on the current device once.
 cudaError_t ensure_smem(const void *func, int bytes);
+
+// Launches with programmatic stream serialization: the kernel may be
+// scheduled while its predecessor in the stream is still running; every
+// kernel of this library calls grid_dependency_wait() before touching
+// memory, so ordering is unchanged and only the launch latency is hidden.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 }  // namespace mp

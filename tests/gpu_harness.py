@@ -68,8 +68,12 @@ class Run:
         self.ns = torch.empty((w.batch, w.n_q_heads), dtype=torch.int32, device="cuda")
 
     # ---- library calls ----
-    def hash_keys(self, n_tokens: Optional[int] = None):
-        mp.hash_keys(self.shape, self.K, self.W, self.max_len if n_tokens is None else n_tokens, self.codes)
+    def hash_keys(self, n_tokens: Optional[int] = None, seq_lens=None):
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        mp.hash_keys(self.shape, self.K, self.W, self.max_len if n_tokens is None else n_tokens, self.codes,
+                     seq_lens=seq_lens, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, "hash kernel reported a stalled pipeline"
 
     def hash_queries(self) -> np.ndarray:
         qc = torch.zeros((self.w.batch, self.w.n_q_heads, self.w.n_tables), dtype=torch.int16, device="cuda")

@@ -67,15 +67,16 @@ def test_bad_shapes_rejected(lib, bad):
     n = ctypes.c_size_t()
     s = good_shape(**bad)
     assert lib.mp_codes_bytes(ctypes.byref(s), ctypes.byref(n)) == mp.MP_ERR_SHAPE
-    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, 10, 16, None) == mp.MP_ERR_SHAPE
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, 10, 16, None, None) == mp.MP_ERR_SHAPE
     assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 10, ctypes.byref(n)) == mp.MP_ERR_SHAPE
 
 
 def test_null_and_misaligned_pointers_rejected(lib):
     s = good_shape()
-    assert lib.mp_hash_keys(ctypes.byref(s), None, 16, None, 10, 16, None) == mp.MP_ERR_ARG
-    assert lib.mp_hash_keys(ctypes.byref(s), 16, 18, None, 10, 16, None) == mp.MP_ERR_ALIGN
-    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, 18, 10, 16, None) == mp.MP_ERR_ALIGN
+    assert lib.mp_hash_keys(ctypes.byref(s), None, 16, None, 10, 16, None, None) == mp.MP_ERR_ARG
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 18, None, 10, 16, None, None) == mp.MP_ERR_ALIGN
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, 18, 10, 16, None, None) == mp.MP_ERR_ALIGN
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, 10, 16, 18, None) == mp.MP_ERR_ALIGN
     assert lib.mp_hash_queries(ctypes.byref(s), 16, 16, None, None) == mp.MP_ERR_ARG
     assert lib.mp_append_token(ctypes.byref(s), 16, 16, 16, 16, 16, 16, None, None, None) == mp.MP_ERR_ARG
     assert lib.mp_append_token(ctypes.byref(s), 16, 16, 16, 16, 16, 16, 16, 18, None) == mp.MP_ERR_ALIGN
@@ -85,8 +86,8 @@ def test_null_and_misaligned_pointers_rejected(lib):
 def test_lengths_and_workspace_checked(lib):
     s = good_shape()
     n = ctypes.c_size_t()
-    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, 1025, 16, None) == mp.MP_ERR_CAPACITY
-    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, -1, 16, None) == mp.MP_ERR_CAPACITY
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, 1025, 16, None, None) == mp.MP_ERR_CAPACITY
+    assert lib.mp_hash_keys(ctypes.byref(s), 16, 16, None, -1, 16, None, None) == mp.MP_ERR_CAPACITY
     assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 1025, ctypes.byref(n)) == mp.MP_ERR_CAPACITY
     assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 1000, ctypes.byref(n)) == 0
     need = n.value
