@@ -49,6 +49,7 @@ extern "C" {
 #define MP_ERR_CAPACITY (-4)  /* a length exceeds the capacity / max_len (device: clamped) */
 #define MP_ERR_WORKSPACE (-5) /* workspace smaller than mp_decode_workspace_bytes */
 #define MP_ERR_CUDA (-6)      /* a CUDA runtime call or launch failed */
+#define MP_ERR_TOO_LARGE (-7) /* beyond the fixed scratch of mp_decode_attend_noalloc */
 
 /*
  * Problem shape.  Supported: head_dim == 128; k_bits in {8, 10};
@@ -147,6 +148,34 @@ int mp_decode_attend(const mp_shape *shape, const void *q, const void *W, const 
                      const void *k_cache, const void *v_cache, const int32_t *seq_lens,
                      int32_t max_len, float *out, float *lse, int32_t *n_sampled, void *workspace,
                      size_t workspace_bytes, const mp_decode_debug *debug, void *stream);
+
+/*
+ * mp_decode_attend without a caller-provided workspace.  The method has no
+ * counterpart of this call: it exists for callers that cannot allocate device
+ * memory where they decode — code inside a CUDA-graph capture region, runtimes
+ * whose memory pools are sealed after start-up, plugins that only receive
+ * tensors from a host framework.  Same arguments, results and device checks as
+ * mp_decode_attend, minus the workspace and the test hooks.
+ *   - Scratch is one fixed array of 16 MiB compiled into the library; every
+ *     GPU that loads the library holds it until the process exits.
+ *   - Problems whose workspace (mp_decode_workspace_bytes) exceeds 16 MiB are
+ *     rejected with MP_ERR_TOO_LARGE before anything is launched (a single
+ *     128k-token sequence with 8 kv heads and K = 8 fits).
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it: make that first call before any
+ *     stream capture begins.
+ *   - Every call shares the array: calls whose executions overlap on the GPU
+ *     (several streams or host threads on one device) race and must be
+ *     serialised by the caller.  The array's contents carry over between calls;
+ *     nothing in it needs to start at zero.
+ *   - status: int32 device word (nullable) that receives this call's status
+ *     word (MP_OK or MP_ERR_CAPACITY), copied asynchronously on `stream`.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+int mp_decode_attend_noalloc(const mp_shape *shape, const void *q, const void *W, const void *codes,
+                             const void *k_cache, const void *v_cache, const int32_t *seq_lens,
+                             int32_t max_len, float *out, float *lse, int32_t *n_sampled,
+                             int32_t *status, void *stream);
 
 /* Synchronises `stream` and reads the status word of a decode workspace. */
 int mp_read_status(const void *workspace, int32_t *status, void *stream);

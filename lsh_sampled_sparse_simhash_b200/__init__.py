@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     codes_bytes,
     codes_shape,
     decode_attend,
+    decode_attend_noalloc,
     decode_workspace_bytes,
     hash_keys,
     hash_queries,
@@ -27,10 +28,12 @@ from ._binding import (  # noqa: F401
     MP_ERR_CAPACITY,
     MP_ERR_WORKSPACE,
     MP_ERR_CUDA,
+    MP_ERR_TOO_LARGE,
 )
 
 __all__ = [
     "MagicPIGError", "Shape", "append_token", "codes_bytes", "codes_shape", "decode_attend",
+    "decode_attend_noalloc",
     "decode_workspace_bytes", "hash_keys", "hash_queries", "library", "library_path", "read_status",
     "status_string",
 ]

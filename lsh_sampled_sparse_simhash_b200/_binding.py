@@ -16,6 +16,7 @@ MP_ERR_ALIGN = -3
 MP_ERR_CAPACITY = -4
 MP_ERR_WORKSPACE = -5
 MP_ERR_CUDA = -6
+MP_ERR_TOO_LARGE = -7
 
 
 class MagicPIGError(RuntimeError):
@@ -71,11 +72,13 @@ def library() -> ctypes.CDLL:
         lib.mp_decode_workspace_bytes.argtypes = [SP, I32, ctypes.POINTER(SZ)]
         lib.mp_decode_attend.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P, SZ,
                                          ctypes.POINTER(_CDebug), P]
+        lib.mp_decode_attend_noalloc.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P, P]
         lib.mp_read_status.argtypes = [P, ctypes.POINTER(I32), P]
         lib.mp_status_string.argtypes = [ctypes.c_int]
         lib.mp_status_string.restype = ctypes.c_char_p
         for f in ("mp_codes_bytes", "mp_hash_keys", "mp_hash_queries", "mp_append_token",
-                  "mp_decode_workspace_bytes", "mp_decode_attend", "mp_read_status"):
+                  "mp_decode_workspace_bytes", "mp_decode_attend", "mp_decode_attend_noalloc",
+                  "mp_read_status"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -158,6 +161,16 @@ def decode_attend(shape: Shape, q, W, codes, k_cache, v_cache, seq_lens, max_len
                                       _ptr(v_cache), _ptr(seq_lens), int(max_len), _ptr(out), _ptr(lse),
                                       _ptr(n_sampled), _ptr(workspace), nbytes, dbg, _stream(stream)),
            "mp_decode_attend")
+
+
+def decode_attend_noalloc(shape: Shape, q, W, codes, k_cache, v_cache, seq_lens, max_len: int, out, lse,
+                          n_sampled, status=None, stream=None):
+    """mp_decode_attend with the library's fixed scratch array instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    _check(library().mp_decode_attend_noalloc(ctypes.byref(shape.c()), _ptr(q), _ptr(W), _ptr(codes),
+                                              _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), int(max_len),
+                                              _ptr(out), _ptr(lse), _ptr(n_sampled), _ptr(status),
+                                              _stream(stream)), "mp_decode_attend_noalloc")
 
 
 def read_status(workspace, stream=None) -> int:

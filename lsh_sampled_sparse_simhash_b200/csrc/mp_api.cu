@@ -11,7 +11,7 @@
 
 namespace mp {
 
-static int validate_shape(const mp_shape *in, Shape &s)
+int validate_shape(const mp_shape *in, Shape &s)
 {
     if (!in) return MP_ERR_ARG;
     s.B = in->batch;
@@ -36,9 +36,9 @@ static int validate_shape(const mp_shape *in, Shape &s)
     return MP_OK;
 }
 
-static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static int check_ptrs(std::initializer_list<const void *> ptrs)
+int check_ptrs(std::initializer_list<const void *> ptrs)
 {
     for (const void *p : ptrs) {
         if (!p) return MP_ERR_ARG;
@@ -47,7 +47,7 @@ static int check_ptrs(std::initializer_list<const void *> ptrs)
     return MP_OK;
 }
 
-static int cuda_status(cudaError_t e) { return e == cudaSuccess ? MP_OK : MP_ERR_CUDA; }
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MP_OK : MP_ERR_CUDA; }
 
 static size_t codes_bytes(const Shape &s) { return (size_t)s.B * s.Hkv * s.L * s.K * (size_t)s.Ncap / 8; }
 
@@ -177,6 +177,7 @@ const char *mp_status_string(int code)
     case MP_ERR_CAPACITY: return "MP_ERR_CAPACITY: length exceeds capacity or max_len";
     case MP_ERR_WORKSPACE: return "MP_ERR_WORKSPACE: workspace too small";
     case MP_ERR_CUDA: return "MP_ERR_CUDA: CUDA runtime error";
+    case MP_ERR_TOO_LARGE: return "MP_ERR_TOO_LARGE: problem needs more scratch than the fixed array of mp_decode_attend_noalloc";
     default: return "MP_ERR_UNKNOWN";
     }
 }

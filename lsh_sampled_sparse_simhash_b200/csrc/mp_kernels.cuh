@@ -2,9 +2,17 @@
 // argument validation).  All launch asynchronously on `st`.
 #pragma once
 
+#include <initializer_list>
+
 #include "mp_common.cuh"
 
 namespace mp {
+
+// Host-side argument checks shared by the C entry points (mp_api.cu).
+int validate_shape(const mp_shape *in, Shape &s);
+bool aligned16(const void *p);
+int check_ptrs(std::initializer_list<const void *> ptrs);
+int cuda_status(cudaError_t e);
 
 cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint16_t *W, const int32_t *seq_lens,
                                 int n_tokens, void *codes, int32_t *status, cudaStream_t st);

@@ -47,7 +47,7 @@ def test_library_has_no_driver_link_dependency(lib):
 
 
 def test_status_strings(lib):
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert mp.status_string(code).startswith("MP_")
 
 
