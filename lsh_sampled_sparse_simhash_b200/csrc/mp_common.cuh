@@ -11,8 +11,9 @@ namespace mp {
 constexpr int kHeadDim = 128;
 constexpr int kMaxGroup = 8;
 constexpr int kScanThreads = 256;  // scan block: token groups x table splits
-constexpr int kScanSplits = 4;     // tables l = ts, ts + 4, ... per split
-constexpr int kChunkK8 = 1024;     // scan chunk (tokens) for byte codes: 64 groups x 16 tokens
+constexpr int kSplitsK8 = 8;       // byte codes: tables l = ts, ts + 8, ... per split
+constexpr int kSplitsK10 = 4;      // bit planes: tables l = ts, ts + 4, ...
+constexpr int kChunkK8 = 512;      // scan chunk (tokens) for byte codes: 32 groups x 16 tokens
 constexpr int kChunkK10 = 8192;    // scan chunk (tokens) for bit planes: 64 groups x 128 tokens
 
 struct Shape {

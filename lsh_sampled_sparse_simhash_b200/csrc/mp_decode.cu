@@ -230,11 +230,11 @@ __device__ __forceinline__ void compact_and_store(const Shape &s, int unit, int 
 // bit-sliced counters (seen >= 1, seen >= 2) for its token group in shared
 // memory; the ts == 0 thread of the same group folds them in:
 //   s2 = s2 | s2' | (s1 & s1'),  s1 = s1 | s1'.
-template <int G, int NW>
+template <int G, int NW, int TS>
 __device__ __forceinline__ void combine_splits(uint32_t (&s1)[G][NW], uint32_t (&s2)[G][NW], uint32_t *part, int ts,
                                                int tg)
 {
-    constexpr int TG = kScanThreads / kScanSplits;
+    constexpr int TG = kScanThreads / TS;
     if (ts > 0) {
 #pragma unroll
         for (int g = 0; g < G; g++)
@@ -247,7 +247,7 @@ __device__ __forceinline__ void combine_splits(uint32_t (&s1)[G][NW], uint32_t (
     __syncthreads();
     if (ts == 0) {
 #pragma unroll 1
-        for (int t = 1; t < kScanSplits; t++) {
+        for (int t = 1; t < TS; t++) {
 #pragma unroll
             for (int g = 0; g < G; g++)
 #pragma unroll
@@ -262,9 +262,10 @@ __device__ __forceinline__ void combine_splits(uint32_t (&s1)[G][NW], uint32_t (
 }
 
 // ---------------------------------------------------------- scan, K = 8 ----
-// Byte codes [unit][L][Ncap].  A 1024-token chunk per block of 256 threads:
-// 64 token groups of 16 tokens (one 16-byte load per table) x 4 table splits
-// (tables ts, ts + 4, ...), merged in shared memory.  Per 4-token word and
+// Byte codes [unit][L][Ncap].  A 512-token chunk per block of 256 threads:
+// 32 token groups of 16 tokens (one 16-byte load per table) x 8 table splits
+// (tables ts, ts + 8, ...; up to 8 loads in flight per thread), merged in
+// shared memory.  Per 4-token word and
 // head: x = codes ^ (qcode * 0x01010101); a byte of x is zero iff that token
 // matches.  Zero bytes are found exactly with ((x & 0x7f..) + 0x7f..) | x,
 // whose byte top bit is 1 iff the byte is non-zero.  Two bit-sliced counters
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
     uint32_t *rep = dyn;
     uint32_t *part = dyn + ((s.L * G + 3) & ~3);
     __shared__ int scratch[64];
-    constexpr int TG = kScanThreads / kScanSplits;
+    constexpr int TS = kSplitsK8, TG = kScanThreads / TS, NB = 8;
     const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
     const int unit = blockIdx.y, chunk = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
@@ -301,24 +302,33 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
 
     if (t0 < N) {
         const uint8_t *base = codes + (size_t)unit * s.L * s.Ncap + t0;
-#pragma unroll 4
-        for (int l = ts; l < s.L; l += kScanSplits) {
-            const uint4 w4 = ld_stream_16(base + (size_t)l * s.Ncap);
-            const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+        for (int lb = ts; lb < s.L; lb += NB * TS) {
+            uint4 wv[NB];
 #pragma unroll
-            for (int g = 0; g < G; g++) {
-                const uint32_t r = rep[l * G + g];
+            for (int i = 0; i < NB; i++) {
+                const int l = lb + i * TS;
+                wv[i] = l < s.L ? ld_stream_16(base + (size_t)l * s.Ncap) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const uint32_t x = w[j] ^ r;
-                    const uint32_t nz = ((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x;
-                    s2[g][j] |= s1[g][j] & ~nz;
-                    s1[g][j] |= ~nz;
+            for (int i = 0; i < NB; i++) {
+                const int l = lb + i * TS;
+                if (l >= s.L) break;
+                const uint32_t w[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+#pragma unroll
+                for (int g = 0; g < G; g++) {
+                    const uint32_t r = rep[l * G + g];
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const uint32_t x = w[j] ^ r;
+                        const uint32_t nz = ((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x;
+                        s2[g][j] |= s1[g][j] & ~nz;
+                        s1[g][j] |= ~nz;
+                    }
                 }
             }
         }
     }
-    combine_splits<G, 4>(s1, s2, part, ts, tg);
+    combine_splits<G, 4, TS>(s1, s2, part, ts, tg);
     // Per-head 16-bit token masks from the byte top bits of the >= 2 counter.
     uint32_t hm[G][1];
 #pragma unroll
@@ -349,7 +359,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_k10_kernel(
     uint32_t *part = dyn + s.L * G * 12;
     __shared__ int scratch[64];
     constexpr int KB = 10;
-    constexpr int TG = kScanThreads / kScanSplits;
+    constexpr int TS = kSplitsK10, TG = kScanThreads / TS;
     const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
     const int unit = blockIdx.y, chunk = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
@@ -375,7 +385,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_k10_kernel(
     if (t0 < N) {
         const uint32_t *base = codes + (size_t)unit * s.L * KB * words + (t0 >> 5);
 #pragma unroll 1
-        for (int l = ts; l < s.L; l += kScanSplits) {
+        for (int l = ts; l < s.L; l += TS) {
             uint4 pl[KB];
 #pragma unroll
             for (int bb = 0; bb < KB; bb++) pl[bb] = ld_stream_16(base + ((size_t)l * KB + bb) * words);
@@ -400,7 +410,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_k10_kernel(
             }
         }
     }
-    combine_splits<G, 4>(s1, s2, part, ts, tg);
+    combine_splits<G, 4, TS>(s1, s2, part, ts, tg);
     if (ts != 0) {
 #pragma unroll
         for (int g = 0; g < G; g++)
@@ -440,6 +450,7 @@ __device__ __forceinline__ float log_sampling_prob(float c, const LogU &u)
 }
 
 constexpr int kAttThreads = 128;
+constexpr int kMaxSpan = 64;                // scan chunks per attention block, at most
 constexpr int kAttRows = 64;                // rows per tile (4 warps x 16)
 constexpr int kAttStages = 3;               // cp.async ring depth
 constexpr int kRowBytes = kHeadDim * 2;     // 256
@@ -454,24 +465,57 @@ struct AttendArgs {
     const int32_t *seq_lens;
     int max_len;
     int nchunk;
-    int subs;   // blocks per scan chunk (each takes an equal share of its candidate list)
+    int span;   // scan chunks per attention block (their candidate lists are concatenated)
+    int subs;   // blocks per span (each takes an equal share of the span's candidates)
+    int ngroups;  // ceil(nchunk / span)
     int chunk_tokens;
     const uint32_t *cand;
     const int32_t *cnt;
-    float *pm, *pl, *pacc;  // [B*Hq][nchunk*subs+1], [..][..][128]
+    float *pm, *pl, *pacc;  // [B*Hq][ngroups*subs+1], [..][..][128]
     LogU lu;
     float scale;  // 1/sqrt(d)
 };
 
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
+                                                  const void *smem_row)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(smem_row)));
+}
+
+// Transposes an 8x8 b16 matrix held one row-pair per thread (mma fragment layout).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
+{
+    uint32_t r;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(r) : "r"(x));
+    return r;
+}
+
+// {lo, hi} -> bf16x2 (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// One block = 4 warps; a warp owns 16 rows of every 64-row tile.
+//   scores  S^T (16 rows x 8 heads) = K rows . Q^T with bf16 mma.sync, fp32 acc;
+//           |k|^2 from the same A fragments.  Lane (g, t) holds rows g, g+8 for
+//           heads 2t, 2t+1 and keeps the online-softmax state of those heads.
+//   log u   only for the (row, head) pairs that are sampled, compacted per warp.
+//   P.V     O^T (128 dims x 8 heads) += V^T . P^T on the tensor cores: P is
+//           split into bf16 hi + lo parts (error ~2^-17 relative), transposed
+//           into B fragments with movmatrix, V^T comes from ldmatrix.trans.
 template <int G>
 __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ float sc[4][16][G];        // per warp: raw scores, then t, then p
-    __shared__ float nrm[4][16];          // per warp: |k|^2
     __shared__ uint32_t meta[kAttStages][kAttRows];  // headmask | exact << 8
+    __shared__ float ucos[4][16 * G];                // per warp: cos of pairs needing log u
+    __shared__ float uval[4][16 * G];                // per warp: their log u
     __shared__ float qinv[G];
-    __shared__ uint8_t upairs[4][16 * G];             // per warp: (row, head) pairs that need log u
 
     const Shape &s = a.s;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -480,105 +524,137 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
     grid_dependency_wait();
     int N = a.seq_lens[b];
     N = N < 0 ? 0 : (N > a.max_len ? a.max_len : N);
-    const bool dsplit = split == a.nchunk * a.subs;
-    const int chunk = split / a.subs, sub = split % a.subs;
-    if (!dsplit && chunk * a.chunk_tokens >= N) return;
+    const bool dsplit = split == a.ngroups * a.subs;
+    const int grp = split / a.subs, sub = split % a.subs;
+    const int c_begin = grp * a.span;
+    const int nch = (N + a.chunk_tokens - 1) / a.chunk_tokens;
+    if (!dsplit && c_begin >= nch) return;
 
-    // Rows of this block: its share of a chunk's compacted candidates, or the
-    // exact set D.
+    // Rows of this block: its share of the concatenated candidate lists of
+    // chunks [c_begin, c_end), or the exact set D.
+    __shared__ int cpre[kMaxSpan + 1];  // prefix sums of the chunks' candidate counts
     const int n_sink = min(s.sink, N);
     const int win0 = max(n_sink, N - s.window);
-    int nrows;
-    const uint32_t *list = nullptr;
+    const int nc = dsplit ? 0 : min(a.span, nch - c_begin);
+    int nrows, e0 = 0;
+    const uint32_t *lists = a.cand + ((size_t)unit * a.nchunk + c_begin) * a.chunk_tokens;
     if (dsplit) {
         nrows = n_sink + (N - win0);
     } else {
-        const int total = a.cnt[((size_t)unit * a.nchunk + chunk) * 16];
-        const int per = (total + a.subs - 1) / a.subs;
-        const int e0 = min(total, sub * per);
-        nrows = min(total, e0 + per) - e0;
-        list = a.cand + ((size_t)unit * a.nchunk + chunk) * a.chunk_tokens + e0;
-    }
-    auto row_of = [&](int e, uint32_t &m) -> int {
-        if (dsplit) {
-            m = ((1u << G) - 1u) | 0x100u;
-            return e < n_sink ? e : win0 + (e - n_sink);
+        if (warp == 0) {
+            int run = 0;
+            for (int j0 = 0; j0 < nc; j0 += 32) {
+                const int j = j0 + lane;
+                const int v = j < nc ? a.cnt[((size_t)unit * a.nchunk + c_begin + j) * 16] : 0;
+                int incl = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                if (j < nc) cpre[j + 1] = run + incl;
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) cpre[0] = 0;
         }
-        const uint32_t v = list[e];
-        m = v >> 24;
-        return (int)(v & 0xFFFFFFu);
-    };
+        __syncthreads();
+        const int total = cpre[nc];
+        const int per = (total + a.subs - 1) / a.subs;
+        e0 = min(total, sub * per);
+        nrows = min(total, e0 + per) - e0;
+    }
+    const uint32_t dmeta = ((1u << G) - 1u) | 0x100u;
 
     const size_t vec0 = (size_t)b * s.Hq + (size_t)kvh * G;
+    const int gq = lane >> 2, tq = lane & 3;
     // B fragments of Q^T (k = head_dim, n = head), 8 k-steps x 2 registers.
     uint32_t qb[8][2];
-    {
-        const int gq = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int ks = 0; ks < 8; ks++) {
-            if (gq < G) {
-                const uint32_t *qp = reinterpret_cast<const uint32_t *>(a.q + (vec0 + gq) * kHeadDim);
-                qb[ks][0] = qp[(ks * 16 + 2 * t) >> 1];
-                qb[ks][1] = qp[(ks * 16 + 2 * t + 8) >> 1];
-            } else {
-                qb[ks][0] = qb[ks][1] = 0u;
-            }
+    for (int ks = 0; ks < 8; ks++) {
+        if (gq < G) {
+            const uint32_t *qp = reinterpret_cast<const uint32_t *>(a.q + (vec0 + gq) * kHeadDim);
+            qb[ks][0] = qp[(ks * 16 + 2 * tq) >> 1];
+            qb[ks][1] = qp[(ks * 16 + 2 * tq + 8) >> 1];
+        } else {
+            qb[ks][0] = qb[ks][1] = 0u;
         }
     }
-    if (tid < G) {
-        float qq = 0.f;
-        const uint16_t *qp = a.q + (vec0 + tid) * kHeadDim;
-        for (int j = 0; j < kHeadDim; j++) {
-            float v = bf16_to_f32(qp[j]);
-            qq = fmaf(v, v, qq);
-        }
-        qinv[tid] = qq > 0.f ? rsqrtf(qq) : 0.f;
+    for (int h = warp; h < G; h += 4) {
+        const uint2 qv = reinterpret_cast<const uint2 *>(a.q + (vec0 + h) * kHeadDim)[lane];
+        float x0 = bf16_lo(qv.x), x1 = bf16_hi(qv.x), x2 = bf16_lo(qv.y), x3 = bf16_hi(qv.y);
+        float qq = x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) qq += __shfl_xor_sync(0xffffffffu, qq, o);
+        if (lane == 0) qinv[h] = qq > 0.f ? rsqrtf(qq) : 0.f;
     }
 
     const uint16_t *kbase = a.kc + (size_t)unit * s.Ncap * kHeadDim;
     const uint16_t *vbase = a.vc + (size_t)unit * s.Ncap * kHeadDim;
     const int ntiles = (nrows + kAttRows - 1) / kAttRows;
 
-    // Tile loader: thread = 16-byte column (tid % 16) of rows tid/16 + 8 i.
-    auto load_tile = [&](int tile, int stage) {
+    // Candidate entries of a tile for this thread's rows (tid/16 + 8 i); the
+    // list is read one tile ahead of the copies so its latency is hidden.
+    int jc = 0;  // chunk of this thread's next candidate (rows are visited in increasing order)
+    auto fetch = [&](int tile, uint32_t (&ent)[8]) {
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const int e = tile * kAttRows + (tid >> 4) + 8 * i;
+            if (e >= nrows) {
+                ent[i] = 0xFFFFFFFFu;
+            } else if (dsplit) {
+                ent[i] = (uint32_t)(e < n_sink ? e : win0 + (e - n_sink));
+            } else {
+                const int r = e0 + e;
+                while (cpre[jc + 1] <= r) jc++;
+                ent[i] = lists[(size_t)jc * a.chunk_tokens + (r - cpre[jc])];
+            }
+        }
+    };
+    auto issue = [&](const uint32_t (&ent)[8], int stage) {
         uint8_t *ks_ = smem + stage * kStageBytes;
         uint8_t *vs_ = ks_ + kAttRows * kRowStride;
         const int col = tid & 15;
 #pragma unroll
-        for (int i = 0; i < kAttRows / 8; i++) {
+        for (int i = 0; i < 8; i++) {
             const int r = (tid >> 4) + 8 * i;
-            const int e = tile * kAttRows + r;
-            uint32_t m = 0;
-            int tok = 0;
-            const bool ok = e < nrows;
-            if (ok) tok = row_of(e, m);
+            const bool ok = ent[i] != 0xFFFFFFFFu;
+            const int tok = ok ? (int)(ent[i] & 0xFFFFFFu) : 0;
             const size_t off = (size_t)tok * kHeadDim + col * 8;
             cp_async_16(ks_ + r * kRowStride + col * 16, kbase + off, ok ? 16 : 0);
             cp_async_16(vs_ + r * kRowStride + col * 16, vbase + off, ok ? 16 : 0);
-            if (col == 0) meta[stage][r] = ok ? m : 0u;
+            if (col == 0) meta[stage][r] = ok ? (dsplit ? dmeta : (ent[i] >> 24)) : 0u;
         }
     };
 
-    float m_run[G], l_run[G], acc[G][4];
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2t, 2t+1 of this lane
+    float acc[8][4];
 #pragma unroll
-    for (int g = 0; g < G; g++) {
-        m_run[g] = -INFINITY;
-        l_run[g] = 0.f;
+    for (int mt = 0; mt < 8; mt++)
 #pragma unroll
-        for (int e = 0; e < 4; e++) acc[g][e] = 0.f;
-    }
+        for (int e = 0; e < 4; e++) acc[mt][e] = 0.f;
 
+    uint32_t nxt[8];
 #pragma unroll
     for (int st = 0; st < kAttStages - 1; st++) {
-        if (st < ntiles) load_tile(st, st);
+        if (st < ntiles) {
+            fetch(st, nxt);
+            issue(nxt, st);
+        }
         cp_async_commit();
     }
+    if (kAttStages - 1 < ntiles) fetch(kAttStages - 1, nxt);
     __syncthreads();  // qinv
+    const int h0 = 2 * tq, h1 = 2 * tq + 1;
+    const float qi0 = h0 < G ? qinv[h0] : 0.f, qi1 = h1 < G ? qinv[h1] : 0.f;
+    const float inv_scale = 1.f / a.scale;
 
     for (int tile = 0; tile < ntiles; tile++) {
         {
             const int nt = tile + kAttStages - 1;
-            if (nt < ntiles) load_tile(nt, nt % kAttStages);
+            if (nt < ntiles) {
+                issue(nxt, nt % kAttStages);
+                if (nt + 1 < ntiles) fetch(nt + 1, nxt);
+            }
             cp_async_commit();
         }
         cp_async_wait<kAttStages - 1>();
@@ -587,15 +663,16 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
         const uint8_t *ks_ = smem + stage * kStageBytes;
         const uint8_t *vs_ = ks_ + kAttRows * kRowStride;
 
-        // ---- S^T (16 rows x 8 heads) = K rows . Q^T, plus |k|^2 ----
-        float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f, na = 0.f, nb = 0.f;
+        // ---- S^T = K rows . Q^T and |k|^2 ----
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        float na = 0.f, nb = 0.f;
         {
             const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStride + (lane >> 4) * 16;
 #pragma unroll
             for (int kst = 0; kst < 8; kst++) {
                 uint32_t a0, a1, a2, a3;
                 ldmatrix_x4(a0, a1, a2, a3, arow + kst * 32);
-                mma_bf16_16816(c0, c1, c2, c3, a0, a1, a2, a3, qb[kst][0], qb[kst][1]);
+                mma_bf16_16816(c[0], c[1], c[2], c[3], a0, a1, a2, a3, qb[kst][0], qb[kst][1]);
                 float x;
                 x = bf16_lo(a0); na = fmaf(x, x, na);
                 x = bf16_hi(a0); na = fmaf(x, x, na);
@@ -610,93 +687,83 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
             na += __shfl_xor_sync(0xffffffffu, na, 2);
             nb += __shfl_xor_sync(0xffffffffu, nb, 1);
             nb += __shfl_xor_sync(0xffffffffu, nb, 2);
-            const int gr = lane >> 2, t = lane & 3;
-            if (2 * t < G) {
-                sc[warp][gr][2 * t] = c0;
-                sc[warp][gr + 8][2 * t] = c2;
-            }
-            if (2 * t + 1 < G) {
-                sc[warp][gr][2 * t + 1] = c1;
-                sc[warp][gr + 8][2 * t + 1] = c3;
-            }
-            if (t == 0) {
-                nrm[warp][gr] = na;
-                nrm[warp][gr + 8] = nb;
-            }
         }
-        __syncwarp();
 
-        // ---- log-weights t = s (exact) or s - log u (sampled), -inf if absent ----
-        // The (row, head) pairs that need log u are compacted first so that the
-        // transcendental work runs on sampled pairs only.
-        int nu = 0;
-        for (int p0 = 0; p0 < 16 * G; p0 += 32) {
-            const int p = p0 + lane;
-            bool need = false;
-            if (p < 16 * G) {
-                const int r = p / G, h = p % G;
-                const uint32_t m = meta[stage][warp * 16 + r];
-                const bool mem = (m >> h) & 1u;
-                need = mem && !(m & 0x100u);
-                sc[warp][r][h] = mem ? sc[warp][r][h] * a.scale : -INFINITY;
+        // ---- log-weights: s (exact) or s - log u (sampled), -inf if absent ----
+        const uint32_t mg = meta[stage][warp * 16 + gq], mg8 = meta[stage][warp * 16 + gq + 8];
+        float tv[4];
+        bool need[4];
+        int pos[4];
+        {
+            const uint32_t mrow[4] = {mg, mg, mg8, mg8};
+            const int hh[4] = {h0, h1, h0, h1};
+            const float kinv_g = na > 0.f ? rsqrtf(na) : 0.f, kinv_g8 = nb > 0.f ? rsqrtf(nb) : 0.f;
+            const float kin[4] = {kinv_g, kinv_g, kinv_g8, kinv_g8};
+            const float qin[4] = {qi0, qi1, qi0, qi1};
+            int base = 0;
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const bool mem = hh[j] < G && ((mrow[j] >> hh[j]) & 1u);
+                need[j] = mem && !(mrow[j] & 0x100u);
+                tv[j] = mem ? c[j] * a.scale : -INFINITY;
+                const uint32_t bal = __ballot_sync(0xffffffffu, need[j]);
+                pos[j] = base + __popc(bal & ((1u << lane) - 1u));
+                if (need[j]) ucos[warp][pos[j]] = c[j] * qin[j] * kin[j];
+                base += __popc(bal);
             }
-            const uint32_t bal = __ballot_sync(0xffffffffu, need);
-            if (need) upairs[warp][nu + __popc(bal & ((1u << lane) - 1u))] = (uint8_t)p;
-            nu += __popc(bal);
+            __syncwarp();
+            for (int i = lane; i < base; i += 32) uval[warp][i] = log_sampling_prob(ucos[warp][i], a.lu);
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                if (need[j]) tv[j] -= uval[warp][pos[j]];
         }
-        __syncwarp();
-        for (int j = lane; j < nu; j += 32) {
-            const int p = upairs[warp][j];
-            const int r = p / G, h = p % G;
-            const float kk = nrm[warp][r];
-            const float sv = sc[warp][r][h];  // already scaled by 1/sqrt(d)
-            const float cosv = kk > 0.f ? sv * (1.f / a.scale) * qinv[h] * rsqrtf(kk) : 0.f;
-            sc[warp][r][h] = sv - log_sampling_prob(cosv, a.lu);
-        }
-        __syncwarp();
+        (void)inv_scale;
 
-        // ---- online softmax update (per warp state) ----
-        float alpha[G], mnew[G];
+        // ---- online softmax over this warp's rows (lanes with equal t share heads) ----
+        float mt0 = fmaxf(tv[0], tv[2]), mt1 = fmaxf(tv[1], tv[3]);
 #pragma unroll
-        for (int g = 0; g < G; g++) {
-            float mt = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < 16; r++) mt = fmaxf(mt, sc[warp][r][g]);
-            mnew[g] = fmaxf(m_run[g], mt);
-            alpha[g] = mnew[g] == -INFINITY ? 1.f : expf(m_run[g] - mnew[g]);
+        for (int o = 4; o < 32; o <<= 1) {
+            mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, o));
+            mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, o));
         }
-        __syncwarp();
-        for (int p = lane; p < 16 * G; p += 32) {
-            const int r = p / G, h = p % G;
-            const float tv = sc[warp][r][h];
-            sc[warp][r][h] = tv == -INFINITY ? 0.f : expf(tv - mnew[h]);
+        const float mn0 = fmaxf(m0, mt0), mn1 = fmaxf(m1, mt1);
+        const float al0 = mn0 == -INFINITY ? 1.f : expf(m0 - mn0);
+        const float al1 = mn1 == -INFINITY ? 1.f : expf(m1 - mn1);
+        float p[4];
+        p[0] = tv[0] == -INFINITY ? 0.f : expf(tv[0] - mn0);
+        p[1] = tv[1] == -INFINITY ? 0.f : expf(tv[1] - mn1);
+        p[2] = tv[2] == -INFINITY ? 0.f : expf(tv[2] - mn0);
+        p[3] = tv[3] == -INFINITY ? 0.f : expf(tv[3] - mn1);
+        l0 = l0 * al0 + p[0] + p[2];
+        l1 = l1 * al1 + p[1] + p[3];
+        m0 = mn0;
+        m1 = mn1;
+#pragma unroll
+        for (int mt = 0; mt < 8; mt++) {
+            acc[mt][0] *= al0;
+            acc[mt][1] *= al1;
+            acc[mt][2] *= al0;
+            acc[mt][3] *= al1;
         }
-        __syncwarp();
-        float lsum[G];
+
+        // ---- O^T += V^T . P^T (P split into bf16 hi + lo) ----
+        const uint32_t hi_g = pack_bf16x2(p[0], p[1]), hi_g8 = pack_bf16x2(p[2], p[3]);
+        const uint32_t lo_g = pack_bf16x2(p[0] - bf16_lo(hi_g), p[1] - bf16_hi(hi_g));
+        const uint32_t lo_g8 = pack_bf16x2(p[2] - bf16_lo(hi_g8), p[3] - bf16_hi(hi_g8));
+        const uint32_t bh0 = movmatrix_trans(hi_g), bh1 = movmatrix_trans(hi_g8);
+        const uint32_t bl0 = movmatrix_trans(lo_g), bl1 = movmatrix_trans(lo_g8);
+        {
+            const int mrow = lane >> 3;
+            const uint8_t *vrow =
+                vs_ + (warp * 16 + (mrow >> 1) * 8 + (lane & 7)) * kRowStride + (mrow & 1) * 16;
 #pragma unroll
-        for (int g = 0; g < G; g++) {
-            lsum[g] = 0.f;
-#pragma unroll
-            for (int e = 0; e < 4; e++) acc[g][e] *= alpha[g];
-        }
-#pragma unroll 4
-        for (int r = 0; r < 16; r++) {
-            const uint2 vv = *reinterpret_cast<const uint2 *>(vs_ + (warp * 16 + r) * kRowStride + lane * 8);
-            const float v0 = bf16_lo(vv.x), v1 = bf16_hi(vv.x), v2 = bf16_lo(vv.y), v3 = bf16_hi(vv.y);
-#pragma unroll
-            for (int g = 0; g < G; g++) {
-                const float pw = sc[warp][r][g];
-                lsum[g] += pw;
-                acc[g][0] = fmaf(pw, v0, acc[g][0]);
-                acc[g][1] = fmaf(pw, v1, acc[g][1]);
-                acc[g][2] = fmaf(pw, v2, acc[g][2]);
-                acc[g][3] = fmaf(pw, v3, acc[g][3]);
+            for (int mt = 0; mt < 8; mt++) {
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4_trans(a0, a1, a2, a3, vrow + mt * 32);
+                mma_bf16_16816(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3], a0, a1, a2, a3, bh0, bh1);
+                mma_bf16_16816(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3], a0, a1, a2, a3, bl0, bl1);
             }
-        }
-#pragma unroll
-        for (int g = 0; g < G; g++) {
-            l_run[g] = l_run[g] * alpha[g] + lsum[g];
-            m_run[g] = mnew[g];
         }
         __syncthreads();  // stage may be refilled next iteration
     }
@@ -704,16 +771,33 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
     __syncthreads();
 
     // ---- merge the 4 warps' states, write this split's partial ----
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
     float *red = reinterpret_cast<float *>(smem);  // [4][G][128] acc, then m, l
     float *redm = red + 4 * G * kHeadDim;
     float *redl = redm + 4 * G;
 #pragma unroll
-    for (int g = 0; g < G; g++) {
-#pragma unroll
-        for (int e = 0; e < 4; e++) red[(warp * G + g) * kHeadDim + lane * 4 + e] = acc[g][e];
-        if (lane == 0) {
-            redm[warp * G + g] = m_run[g];
-            redl[warp * G + g] = l_run[g];
+    for (int mt = 0; mt < 8; mt++) {
+        if (h0 < G) {
+            red[(warp * G + h0) * kHeadDim + mt * 16 + gq] = acc[mt][0];
+            red[(warp * G + h0) * kHeadDim + mt * 16 + gq + 8] = acc[mt][2];
+        }
+        if (h1 < G) {
+            red[(warp * G + h1) * kHeadDim + mt * 16 + gq] = acc[mt][1];
+            red[(warp * G + h1) * kHeadDim + mt * 16 + gq + 8] = acc[mt][3];
+        }
+    }
+    if (gq == 0) {
+        if (h0 < G) {
+            redm[warp * G + h0] = m0;
+            redl[warp * G + h0] = l0;
+        }
+        if (h1 < G) {
+            redm[warp * G + h1] = m1;
+            redl[warp * G + h1] = l1;
         }
     }
     __syncthreads();
@@ -732,7 +816,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
             }
         }
         const size_t bh = vec0 + g;
-        const size_t pidx = bh * ((size_t)a.nchunk * a.subs + 1) + split;
+        const size_t pidx = bh * ((size_t)a.ngroups * a.subs + 1) + split;
         a.pacc[pidx * kHeadDim + dim] = A;
         if (dim == 0) {
             a.pm[pidx] = M;
@@ -742,45 +826,95 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
 }
 
 // ----------------------------------------------------------------- merge ----
+// One block of 128 threads per (b, q head).  Pass 1: the global maximum of
+// the split maxima (threads stride over splits).  Pass 2: warp w folds splits
+// w, w + 4, ... with exp(m_j - M) weights (lane = 4 output dims, independent
+// loads unrolled), then the four warps are summed in shared memory.
 template <int G>
 __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t *__restrict__ seq_lens,
-                                                         int max_len, int nchunk, int subs, int chunk_tokens,
+                                                         int max_len, int nchunk, int span, int subs,
+                                                         int ngroups, int chunk_tokens,
                                                          const float *__restrict__ pm,
                                                          const float *__restrict__ pl,
                                                          const float *__restrict__ pacc,
                                                          const int32_t *__restrict__ cnt, float *out,
                                                          float *lse, int32_t *n_sampled)
 {
+    __shared__ float red_m[4], red_l[4];
+    __shared__ int red_n[4];
+    __shared__ float4 red_acc[4][32];
     const int bh = blockIdx.x;
     const int b = bh / s.Hq, h = bh % s.Hq, kvh = h / G, g = h % G;
     const int unit = b * s.Hkv + kvh;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     grid_dependency_wait();
     int N = seq_lens[b];
     N = N < 0 ? 0 : (N > max_len ? max_len : N);
-    const int nsp = ((N + chunk_tokens - 1) / chunk_tokens) * subs;  // live chunk splits
-    const int dsp = nchunk * subs;                                    // the exact-set split
-    const int dim = threadIdx.x;
+    const int nch = (N + chunk_tokens - 1) / chunk_tokens;
+    const int nsp = ((nch + span - 1) / span) * subs;  // live chunk splits
+    const int dsp = ngroups * subs;                     // the exact-set split
     const size_t base = (size_t)bh * (dsp + 1);
-    float M = pm[base + dsp];
-    for (int j = 0; j < nsp; j++) M = fmaxf(M, pm[base + j]);
-    float Ls = 0.f, A = 0.f;
-    if (M != -INFINITY) {
-        auto add = [&](int j) {
-            const float mj = pm[base + j];
-            if (mj == -INFINITY) return;
-            const float f = expf(mj - M);
-            Ls += pl[base + j] * f;
-            A += pacc[(base + j) * kHeadDim + dim] * f;
-        };
-        for (int j = 0; j < nsp; j++) add(j);
-        add(dsp);
+    auto split_index = [&](int j) { return j < nsp ? j : dsp; };  // j in [0, nsp]
+
+    // pass 1: M = max over live splits and D; sampled count
+    float m = -INFINITY;
+    int ns = 0;
+    for (int j = tid; j <= nsp; j += blockDim.x) m = fmaxf(m, pm[base + split_index(j)]);
+    for (int j = tid; j < nch; j += blockDim.x) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        ns += __shfl_xor_sync(0xffffffffu, ns, o);
     }
-    out[(size_t)bh * kHeadDim + dim] = Ls > 0.f ? A / Ls : 0.f;
-    if (dim == 0) {
-        lse[bh] = Ls > 0.f ? M + logf(Ls) : -INFINITY;
-        int ns = 0;
-        for (int j = 0; j < nsp / subs; j++) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
-        n_sampled[bh] = ns;
+    if (lane == 0) {
+        red_m[warp] = m;
+        red_n[warp] = ns;
+    }
+    __syncthreads();
+    const float M = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+
+    // pass 2
+    float Ls = 0.f;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+#pragma unroll 4
+        for (int j = warp; j <= nsp; j += 4) {
+            const size_t sp = base + split_index(j);
+            const float mj = pm[sp];
+            const float f = mj == -INFINITY ? 0.f : expf(mj - M);
+            const float lj = pl[sp];
+            const float4 aj = reinterpret_cast<const float4 *>(pacc + sp * kHeadDim)[lane];
+            Ls = fmaf(lj, f, Ls);
+            A.x = fmaf(aj.x, f, A.x);
+            A.y = fmaf(aj.y, f, A.y);
+            A.z = fmaf(aj.z, f, A.z);
+            A.w = fmaf(aj.w, f, A.w);
+        }
+    }
+    red_acc[warp][lane] = A;
+    if (lane == 0) red_l[warp] = Ls;
+    __syncthreads();
+    if (warp == 0) {
+        const float Lt = red_l[0] + red_l[1] + red_l[2] + red_l[3];
+        float4 o = red_acc[0][lane];
+#pragma unroll
+        for (int w = 1; w < 4; w++) {
+            const float4 t = red_acc[w][lane];
+            o.x += t.x;
+            o.y += t.y;
+            o.z += t.z;
+            o.w += t.w;
+        }
+        const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+        o.x *= inv;
+        o.y *= inv;
+        o.z *= inv;
+        o.w *= inv;
+        reinterpret_cast<float4 *>(out + (size_t)bh * kHeadDim)[lane] = o;
+        if (lane == 0) {
+            lse[bh] = Lt > 0.f ? M + logf(Lt) : -INFINITY;
+            n_sampled[bh] = red_n[0] + red_n[1] + red_n[2] + red_n[3];
+        }
     }
 }
 
@@ -796,20 +930,40 @@ struct Workspace {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Attention blocks per scan chunk: enough blocks for two waves on 148 SMs
-// (a fixed count, so the workspace size does not depend on the device).
-static int attend_subs(const Shape &s, int nchunk)
+// How attention blocks cover the scan chunks.  Many chunks: each block takes
+// `span` consecutive chunks (about 600 blocks in all, so that the per-block
+// set-up is amortised and the merge sees few partials).  Few chunks: each
+// chunk's list is shared by `subs` blocks so that about 296 blocks (two per
+// SM on 148 SMs) run.  Fixed counts, so the workspace size does not depend on
+// the device.
+struct SplitPlan {
+    int nchunk, span, subs, ngroups, nsplit;
+};
+
+static SplitPlan split_plan(const Shape &s, int max_len)
 {
-    const int blocks = nchunk * s.B * s.Hkv;
-    if (blocks == 0) return 1;
-    return std::max(1, std::min(8, (296 + blocks - 1) / blocks));
+    SplitPlan p;
+    const int C = chunk_tokens(s.K);
+    p.nchunk = (max_len + C - 1) / C;
+    const int blocks = p.nchunk * s.B * s.Hkv;
+    if (blocks >= 600) {
+        p.span = std::min(kMaxSpan, blocks / 600);
+        p.subs = 1;
+    } else {
+        p.span = 1;
+        p.subs = blocks > 0 ? std::max(1, std::min(8, 296 / blocks)) : 1;
+    }
+    p.ngroups = (p.nchunk + p.span - 1) / p.span;
+    p.nsplit = p.ngroups * p.subs + 1;
+    return p;
 }
 
 Workspace workspace_layout(const Shape &s, int max_len, void *base)
 {
     const int C = chunk_tokens(s.K);
-    const int nchunk = (max_len + C - 1) / C;
-    const size_t nsplit = (size_t)nchunk * attend_subs(s, nchunk) + 1;
+    const SplitPlan sp = split_plan(s, max_len);
+    const int nchunk = sp.nchunk;
+    const size_t nsplit = (size_t)sp.nsplit;
     const size_t units = (size_t)s.B * s.Hkv, bh = (size_t)s.B * s.Hq;
     size_t off = 0;
     Workspace w{};
@@ -852,8 +1006,8 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
                                    const Workspace &ws, const mp_decode_debug *dbg, cudaStream_t st)
 {
     const int C = chunk_tokens(s.K);
-    const int nchunk = (max_len + C - 1) / C;
-    const int subs = attend_subs(s, nchunk);
+    const SplitPlan sp = split_plan(s, max_len);
+    const int nchunk = sp.nchunk;
     const int units = s.B * s.Hkv;
     cudaError_t e;
     {
@@ -889,7 +1043,9 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     aa.seq_lens = seq_lens;
     aa.max_len = max_len;
     aa.nchunk = nchunk;
-    aa.subs = subs;
+    aa.span = sp.span;
+    aa.subs = sp.subs;
+    aa.ngroups = sp.ngroups;
     aa.chunk_tokens = C;
     aa.cand = ws.cand;
     aa.cnt = ws.cnt;
@@ -901,10 +1057,11 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     {
         const int sm = kAttStages * kStageBytes;
         if ((e = ensure_smem(reinterpret_cast<const void *>(attend_kernel<G>), sm)) != cudaSuccess) return e;
-        dim3 grid(nchunk * subs + 1, units);
+        dim3 grid(sp.nsplit, units);
         if ((e = launch_pdl(attend_kernel<G>, grid, dim3(kAttThreads), sm, st, aa)) != cudaSuccess) return e;
     }
-    e = launch_pdl(merge_kernel<G>, dim3(s.B * s.Hq), dim3(kHeadDim), 0, st, s, seq_lens, max_len, nchunk, subs, C,
+    e = launch_pdl(merge_kernel<G>, dim3(s.B * s.Hq), dim3(kHeadDim), 0, st, s, seq_lens, max_len, nchunk, sp.span,
+                   sp.subs, sp.ngroups, C,
                    (const float *)ws.pm, (const float *)ws.pl, (const float *)ws.pacc, (const int32_t *)ws.cnt, out,
                    lse, n_sampled);
     if (e != cudaSuccess) return e;

@@ -11,10 +11,12 @@
 //               reloaded only when a CTA moves to the next group) and a
 //               2-stage ring of 128-row key tiles, 128B-swizzled.
 //   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, M = 128,
-//               N <= 128, K = 16, into one of four TMEM accumulators.
-//   warp 2      TMEM allocator (512 columns = 4 x 128-column accumulators).
-//   warps 4..11 epilogue, two groups of four warps taking alternate column
-//               tiles: tcgen05.ld 32x32b (thread = key row, registers =
+//               N <= 256, K = 16, into one of two TMEM accumulators (N = 256
+//               keeps the operand traffic per flop within shared-memory
+//               bandwidth).
+//   warp 2      TMEM allocator (512 columns = 2 x 256-column accumulators).
+//   warps 4..11 epilogue, two groups of four warps taking column tiles in
+//               turn: tcgen05.ld 32x32b (thread = key row, registers =
 //               columns, 64 columns per wait), sign test, pack, store.
 //               K = 8: one byte per (table, token); K = 10: one warp ballot
 //               per column gives the 32-token bit-plane word.
@@ -34,10 +36,12 @@
 namespace mp {
 namespace tc {
 
-constexpr int kThreads = 384;
+constexpr int kEpiGroups = 2;                // epilogue groups of 4 warps
+constexpr int kThreads = 128 + 128 * kEpiGroups;
 constexpr int kBM = 128;                     // key rows per tile = TMEM lanes
-constexpr int kAccCols = 128;                // columns per accumulator buffer
-constexpr int kAccBufs = 4;                  // 4 x 128 = all 512 TMEM columns
+constexpr int kAccCols = 256;                // columns per accumulator buffer
+constexpr int kAccBufs = 2;                  // 2 x 256 = all 512 TMEM columns
+constexpr int kLensCache = 256;              // sequence lengths kept in shared memory
 constexpr int kStages = 2;                   // key-tile ring depth
 constexpr int kHalfBytes = kBM * 128;        // one 64-element (128 B) K half of a tile
 constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KB
@@ -152,12 +156,39 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// All ones iff the fp32 value with these bits is > 0 (so +0, -0 and NaN -> 0).
+__device__ __forceinline__ uint32_t positive_mask(uint32_t bits)
+{
+    uint32_t m;
+    asm("set.gt.u32.f32 %0, %1, 0f00000000;" : "=r"(m) : "f"(__uint_as_float(bits)));
+    return m;
+}
+
+// [x > 0] as 1.0f / 0.0f on the FMA pipe: the first saturating product sends
+// every positive normal to 1 and keeps positive subnormals above 2^-23, the
+// second sends those to 1 as well; zero, negatives and NaN give 0.
+__device__ __forceinline__ float positive_unit(uint32_t bits)
+{
+    return __saturatef(__saturatef(__uint_as_float(bits) * 0x1p126f) * 0x1p126f);
+}
+
+// Byte whose bit b is [v[b] > 0], built with FMA-pipe arithmetic: the sum
+// sum_b [v_b > 0] 2^b is exact in fp32, and adding 2^23 puts it in the low
+// byte of the float's bit pattern.
+__device__ __forceinline__ uint32_t pack_positive_byte(const uint32_t *v)
+{
+    float acc = positive_unit(v[7]);
+#pragma unroll
+    for (int b = 6; b >= 0; b--) acc = fmaf(acc, 2.f, positive_unit(v[b]));
+    return __float_as_uint(acc + 8388608.f);
+}
+
 struct Item {
     int group, unit, mt, len;
     bool skip;
 };
 
-__device__ __forceinline__ Item item_of(const Params &p, int it)
+__device__ __forceinline__ Item item_of(const Params &p, int it, const int *lens_sh)
 {
     Item r;
     const int units = p.s.B * p.s.Hkv;
@@ -166,7 +197,10 @@ __device__ __forceinline__ Item item_of(const Params &p, int it)
     r.unit = rem / p.n_mt;
     r.mt = rem % p.n_mt;
     int len = p.n_tokens;
-    if (p.seq_lens) len = min(len, max(p.seq_lens[r.unit / p.s.Hkv], 0));
+    if (p.seq_lens) {
+        const int b = r.unit / p.s.Hkv;
+        len = min(len, max(b < kLensCache ? lens_sh[b] : p.seq_lens[b], 0));
+    }
     r.len = len;
     r.skip = r.mt * kBM >= len;
     return r;
@@ -188,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ __align__(8) uint64_t bars[16];  // 15 used
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_flag;
+    __shared__ int lens_sh[kLensCache];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     grid_dependency_wait();
@@ -213,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(tmem_full(b), 1);
             mbar_init(tmem_empty(b), 128);
         }
+        static_assert(kAccBufs * kAccCols == 512, "TMEM holds 512 columns");
         mbar_init(w_full, 1);
         mbar_init(w_empty, 1);
         mbar_init(final_bar, 1);
@@ -223,6 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                      "r"(kAccBufs * kAccCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
+    if (p.seq_lens)
+        for (int i = tid; i < p.s.B && i < kLensCache; i += blockDim.x) lens_sh[i] = p.seq_lens[i];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -236,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int last_issued_par[kStages] = {-1, -1};
         int cur_g = -1, w_loads = 0;
         for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
-            const Item im = item_of(p, it);
+            const Item im = item_of(p, it, lens_sh);
             if (im.skip) continue;
             if (im.group != cur_g) {
                 if (cur_g >= 0 && !mbar_wait(w_empty, (w_loads - 1) & 1, &abort_flag, p.status)) break;
@@ -264,12 +302,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w_loads > 0) mbar_wait(w_full, (w_loads - 1) & 1, &abort_flag, p.status);
     } else if (warp == 1 && lane == 0) {
         // ----------------------------------------------------------- MMA ----
-        int stage = 0, acc = 0;
+        int stage = 0, seq = 0;  // seq: column-tile sequence number; buffer seq % 4, use seq / 4
         uint32_t full_par[kStages] = {0, 0};
-        uint32_t tempty_par[kAccBufs] = {0, 0, 0, 0};
         int cur_g = -1, w_uses = 0;
         for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
-            const Item im = item_of(p, it);
+            const Item im = item_of(p, it, lens_sh);
             if (im.skip) continue;
             if (im.group != cur_g) {
                 if (cur_g >= 0) mma_commit(w_empty);  // W free once the MMAs so far complete
@@ -283,13 +320,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             int c0, width;
             group_cols(p, im.group, c0, width);
             bool ok = true;
-            for (int n0 = 0; n0 < width; n0 += kAccCols) {
+            for (int n0 = 0; n0 < width; n0 += kAccCols, seq++) {
                 const int nw = min(kAccCols, width - n0);
-                if (!mbar_wait(tmem_empty(acc), tempty_par[acc] ^ 1u, &abort_flag, p.status)) {
+                const int acc = seq & (kAccBufs - 1);
+                // wait for the epilogue to release use (seq / 4 - 1) of this buffer
+                if (!mbar_wait(tmem_empty(acc), ((seq / kAccBufs) & 1) ^ 1u, &abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
-                tempty_par[acc] ^= 1u;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(acc * kAccCols);
                 const uint32_t idesc = idesc_bf16(nw);
@@ -303,7 +341,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 mma_commit(tmem_full(acc));
-                acc = (acc + 1) & (kAccBufs - 1);
             }
             if (!ok) break;
             mma_commit(empty_a(stage));
@@ -315,13 +352,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 4) {
         // ------------------------------------------------------ epilogue ----
         const int q4 = warp & 3;         // TMEM lane quarter of this warp
-        const int eg = (warp - 4) >> 2;  // epilogue group: takes column tiles seq % 2 == eg
+        const int eg = (warp - 4) >> 2;  // epilogue group: takes column tiles seq % kEpiGroups == eg
         const int row = q4 * 32 + lane;
         int seq = 0;                     // column-tile sequence number (all groups)
-        uint32_t tfull_par[kAccBufs] = {0, 0, 0, 0};
         const int words = s.Ncap >> 5;
         for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
-            const Item im = item_of(p, it);
+            const Item im = item_of(p, it, lens_sh);
             if (im.skip) continue;
             int c0, width;
             group_cols(p, im.group, c0, width);
@@ -330,14 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool warp_live = im.mt * kBM + q4 * 32 < im.len;
             bool ok = true;
             for (int n0 = 0; n0 < width; n0 += kAccCols, seq++) {
-                if ((seq & 1) != eg) continue;
+                if (seq % kEpiGroups != eg) continue;
                 const int acc = seq & (kAccBufs - 1);
                 const int nw = min(kAccCols, width - n0);
-                if (!mbar_wait(tmem_full(acc), tfull_par[acc], &abort_flag, p.status)) {
+                if (!mbar_wait(tmem_full(acc), (seq / kAccBufs) & 1, &abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
-                tfull_par[acc] ^= 1u;
                 tc_fence_after();
                 for (int ch = 0; ch < nw; ch += 64) {
                     uint32_t v[64];
@@ -354,10 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (s.K == 8) {
 #pragma unroll
                             for (int t = 0; t < 4; t++) {
-                                uint32_t byte = 0;
-#pragma unroll
-                                for (int bb = 0; bb < 8; bb++)
-                                    byte |= (__uint_as_float(vv[8 * t + bb]) > 0.f ? 1u : 0u) << bb;
+                                const uint32_t byte = pack_positive_byte(vv + 8 * t);
                                 const int l = (col0 >> 3) + t;
                                 if (valid && l < s.L)
                                     static_cast<uint8_t *>(p.codes)[((size_t)im.unit * s.L + l) * s.Ncap + tok] =

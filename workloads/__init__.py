@@ -98,6 +98,11 @@ WORKLOADS = {
         seed=1005,
         description="batch 16, lengths U[32768,131072], K=8, L=75, keys = mu_h (|mu_h|=8) + N(0,1), "
                     "128 needles per kv head"),
+    "ragged4": Workload(
+        "ragged4", 4, 32, 8, 128, 131072, 8, 75, n_planted=128, ragged_min=32768, mu_norm=8.0,
+        seed=1006,
+        description="the ragged workload at batch 4 (about 2 GB of cache): the profiling case for the "
+                    "K=8 scan and the sampled-attention kernel"),
 }
 
 
