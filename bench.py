@@ -208,6 +208,20 @@ class Bench:
             torch.cuda.synchronize()
 
     def run_timed(self, ev):
+        """K steps, one event pair per step (no events between the calls, which
+        would serialise the programmatic launch chain)."""
+        for e in ev:
+            self.flush.zero_()
+            self.lens.copy_(self.lens0, non_blocking=True)
+            e[0].record()
+            self.hash()
+            self.append()
+            self.decode()
+            e[1].record()
+
+    def run_breakdown(self, ev):
+        """K more steps with an event between every call: per-call device time
+        for the roofline of each kernel."""
         for e in ev:
             self.flush.zero_()
             self.lens.copy_(self.lens0, non_blocking=True)
@@ -399,10 +413,13 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
-    hash_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    append_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    evb = bench.timed(args.steps, 0)
+    bench.run_breakdown(evb)
+    torch.cuda.synchronize()
+    hash_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evb)
+    append_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evb)
+    decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evb)
     total_ms, all_tokens = reduce_over_ranks(sum(step_ms), bench.tokens * args.steps, device, world)
     value = all_tokens / (total_ms / 1e3)
 

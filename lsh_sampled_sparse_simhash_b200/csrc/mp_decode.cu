@@ -153,7 +153,17 @@ struct ScanOut {
     int32_t *cnt;        // [B*Hkv][nchunk][16]: [0] union count, [1+g] per-head count
     uint8_t *member_out; // nullable [B][Hq][Ncap]
     int32_t *status;
+    uint32_t one;        // 1, opaque to the compiler (see add_fma)
 };
+
+// a + c computed as a * one + c: an integer multiply-add runs on the FMA pipe,
+// leaving the ALU pipe to the logic operations of the byte scan.
+__device__ __forceinline__ uint32_t add_fma(uint32_t a, uint32_t one, uint32_t c)
+{
+    uint32_t r;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(one), "r"(c));
+    return r;
+}
 
 // Bits [lo - base, hi - base) of a `width`-bit token word starting at token `base`.
 __device__ __forceinline__ uint32_t range_mask(int base, int lo, int hi, int width)
@@ -268,8 +278,9 @@ __device__ __forceinline__ void combine_splits(uint32_t (&s1)[G][NW], uint32_t (
 // shared memory.  Per 4-token word and
 // head: x = codes ^ (qcode * 0x01010101); a byte of x is zero iff that token
 // matches.  Zero bytes are found exactly with ((x & 0x7f..) + 0x7f..) | x,
-// whose byte top bit is 1 iff the byte is non-zero.  Two bit-sliced counters
-// (seen >= 1, seen >= 2) live in the byte top bits.
+// whose byte top bit is 1 iff the byte is non-zero (the add runs on the FMA
+// pipe).  Two bit-sliced counters (seen >= 1, seen >= 2) live in the byte top
+// bits.
 template <int G>
 __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
     Shape s, const uint8_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
@@ -320,7 +331,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
                         const uint32_t x = w[j] ^ r;
-                        const uint32_t nz = ((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x;
+                        const uint32_t nz = add_fma(x & 0x7F7F7F7Fu, o.one, 0x7F7F7F7Fu) | x;
                         s2[g][j] |= s1[g][j] & ~nz;
                         s1[g][j] |= ~nz;
                     }
@@ -1016,7 +1027,7 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
                        (const uint16_t *)(dbg ? dbg->qcodes_in : nullptr), ws.qcodes, ws.status);
         if (e != cudaSuccess) return e;
     }
-    ScanOut so{ws.cand, ws.cnt, dbg ? dbg->member_out : nullptr, ws.status};
+    ScanOut so{ws.cand, ws.cnt, dbg ? dbg->member_out : nullptr, ws.status, 1u};
     if (nchunk > 0) {
         dim3 grid(nchunk, units);
         const size_t part = (size_t)2 * G * 4 * kScanThreads * sizeof(uint32_t);
@@ -1052,6 +1063,7 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     aa.pm = ws.pm;
     aa.pl = ws.pl;
     aa.pacc = ws.pacc;
+
     aa.lu = make_logu(s);
     aa.scale = 1.0f / sqrtf((float)s.d);
     {
@@ -1061,9 +1073,8 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
         if ((e = launch_pdl(attend_kernel<G>, grid, dim3(kAttThreads), sm, st, aa)) != cudaSuccess) return e;
     }
     e = launch_pdl(merge_kernel<G>, dim3(s.B * s.Hq), dim3(kHeadDim), 0, st, s, seq_lens, max_len, nchunk, sp.span,
-                   sp.subs, sp.ngroups, C,
-                   (const float *)ws.pm, (const float *)ws.pl, (const float *)ws.pacc, (const int32_t *)ws.cnt, out,
-                   lse, n_sampled);
+                   sp.subs, sp.ngroups, C, (const float *)ws.pm, (const float *)ws.pl, (const float *)ws.pacc,
+                   (const int32_t *)ws.cnt, out, lse, n_sampled);
     if (e != cudaSuccess) return e;
     if (dbg && dbg->qcodes_out)
         e = cudaMemcpyAsync(dbg->qcodes_out, ws.qcodes, (size_t)s.B * s.Hq * s.L * sizeof(uint16_t),

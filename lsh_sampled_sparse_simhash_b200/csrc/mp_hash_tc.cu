@@ -15,9 +15,10 @@
 //               keeps the operand traffic per flop within shared-memory
 //               bandwidth).
 //   warp 2      TMEM allocator (512 columns = 2 x 256-column accumulators).
-//   warps 4..11 epilogue, two groups of four warps taking column tiles in
-//               turn: tcgen05.ld 32x32b (thread = key row, registers =
-//               columns, 64 columns per wait), sign test, pack, store.
+//   warps 4..19 epilogue, four groups of four warps, each group one 64-column
+//               slice of every column tile: tcgen05.ld 32x32b (thread = key
+//               row, registers = columns), release of the accumulator, then
+//               sign test, pack, store off the MMA's critical path.
 //               K = 8: one byte per (table, token); K = 10: one warp ballot
 //               per column gives the 32-token bit-plane word.
 //
@@ -36,13 +37,18 @@
 namespace mp {
 namespace tc {
 
-constexpr int kEpiGroups = 2;                // epilogue groups of 4 warps
+#ifndef MP_HASH_EPI_GROUPS
+#define MP_HASH_EPI_GROUPS 4
+#endif
+constexpr int kEpiGroups = MP_HASH_EPI_GROUPS;  // epilogue groups of 4 warps, one column slice each
 constexpr int kThreads = 128 + 128 * kEpiGroups;
 constexpr int kBM = 128;                     // key rows per tile = TMEM lanes
 constexpr int kAccCols = 256;                // columns per accumulator buffer
 constexpr int kAccBufs = 2;                  // 2 x 256 = all 512 TMEM columns
 constexpr int kLensCache = 256;              // sequence lengths kept in shared memory
+constexpr int kSliceCols = kAccCols / kEpiGroups;  // columns of a tile per epilogue group
 constexpr int kStages = 2;                   // key-tile ring depth
+constexpr int kPrefetchAhead = 3;            // key tiles (of this block) kept in flight to L2
 constexpr int kHalfBytes = kBM * 128;        // one 64-element (128 B) K half of a tile
 constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KB
 constexpr int kMaxGroupCols = 640;
@@ -116,6 +122,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// Pulls a future key tile into L2 (no shared memory, no completion tracking),
+// so that the ring's real load later finds it there.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
 // K-major, 128B-swizzled operand: rows of 128 B, 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
 {
@@ -183,6 +198,47 @@ __device__ __forceinline__ uint32_t pack_positive_byte(const uint32_t *v)
     return __float_as_uint(acc + 8388608.f);
 }
 
+// 32-bit word whose bit c is [v[c] > 0]: two exact 16-bit FMA-pipe sums.
+__device__ __forceinline__ uint32_t pack_positive_word(const uint32_t *v)
+{
+    float lo = positive_unit(v[15]), hi = positive_unit(v[31]);
+#pragma unroll
+    for (int b = 14; b >= 0; b--) {
+        lo = fmaf(lo, 2.f, positive_unit(v[b]));
+        hi = fmaf(hi, 2.f, positive_unit(v[16 + b]));
+    }
+    return __byte_perm(__float_as_uint(lo + 8388608.f), __float_as_uint(hi + 8388608.f), 0x5410);
+}
+
+// Within each group of 4 lanes, transposes the 4x4 byte matrix whose row r
+// (lane r of the group) is the word x: afterwards lane r holds byte r of every
+// lane of its group, in lane order.
+__device__ __forceinline__ uint32_t quad_transpose(uint32_t x, int lane)
+{
+    uint32_t y = __shfl_xor_sync(0xffffffffu, x, 1);
+    x = __byte_perm(x, y, (lane & 1) ? 0x3715 : 0x6240);
+    y = __shfl_xor_sync(0xffffffffu, x, 2);
+    return __byte_perm(x, y, (lane & 2) ? 0x3276 : 0x5410);
+}
+
+// 32x32 bit-matrix transpose across a warp: lane t holds row t; afterwards
+// lane c holds column c (bit t of the result = bit c of lane t's input).
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane)
+{
+    const uint32_t masks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+    for (int k = 0; k < 5; k++) {
+        const int j = 16 >> k;
+        const uint32_t m = masks[k];
+        const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+        if (lane & j)
+            x = (x & ~m) | ((y >> j) & m);   // take the partner's high half into our low positions
+        else
+            x = (x & m) | ((y << j) & ~m);   // take the partner's low half into our high positions
+    }
+    return x;
+}
+
 struct Item {
     int group, unit, mt, len;
     bool skip;
@@ -246,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < kAccBufs; b++) {
             mbar_init(tmem_full(b), 1);
-            mbar_init(tmem_empty(b), 128);
+            mbar_init(tmem_empty(b), 128 * kEpiGroups);
         }
         static_assert(kAccBufs * kAccCols == 512, "TMEM holds 512 columns");
         mbar_init(w_full, 1);
@@ -273,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t empty_par[kStages] = {0, 0};
         int last_issued_par[kStages] = {-1, -1};
         int cur_g = -1, w_loads = 0;
+        bool first_pass = true;
         for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
             const Item im = item_of(p, it, lens_sh);
             if (im.skip) continue;
@@ -290,6 +347,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(empty_a(stage), empty_par[stage] ^ 1u, &abort_flag, p.status)) break;
             empty_par[stage] ^= 1u;
             const int row0 = im.unit * s.Ncap + im.mt * kBM;
+            // later tiles of this block into L2: the first pass covers 2..kPrefetchAhead
+            // items ahead, every later pass the one newly kPrefetchAhead ahead
+            for (int ahead = first_pass ? 2 : kPrefetchAhead; ahead <= kPrefetchAhead; ahead++) {
+                const int it2 = it + ahead * (int)gridDim.x;
+                if (it2 < p.total_items) {
+                    const Item i2 = item_of(p, it2, lens_sh);
+                    if (!i2.skip) {
+                        const int r2 = i2.unit * s.Ncap + i2.mt * kBM;
+                        tma_prefetch_l2_2d(&tmap_keys, 0, r2);
+                        tma_prefetch_l2_2d(&tmap_keys, 64, r2);
+                    }
+                }
+            }
+            first_pass = false;
             mbar_expect_tx(full_a(stage), kTileBytes);
             tma_load_2d(a_smem + stage * kTileBytes, &tmap_keys, full_a(stage), 0, row0);
             tma_load_2d(a_smem + stage * kTileBytes + kHalfBytes, &tmap_keys, full_a(stage), 64, row0);
@@ -351,10 +422,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(final_bar, 0, &abort_flag, p.status);
     } else if (warp >= 4) {
         // ------------------------------------------------------ epilogue ----
+        // Every epilogue warp takes part in every column tile: group eg owns
+        // columns [64 eg, 64 eg + 64) of the tile, warp quarter q4 owns rows
+        // [32 q4, 32 q4 + 32).  The accumulator is released as soon as its
+        // values are in registers, so packing and storing overlap the next MMAs.
         const int q4 = warp & 3;         // TMEM lane quarter of this warp
-        const int eg = (warp - 4) >> 2;  // epilogue group: takes column tiles seq % kEpiGroups == eg
+        const int eg = (warp - 4) >> 2;  // column slice of every tile
         const int row = q4 * 32 + lane;
-        int seq = 0;                     // column-tile sequence number (all groups)
+        int seq = 0;                     // column-tile sequence number
         const int words = s.Ncap >> 5;
         for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
             const Item im = item_of(p, it, lens_sh);
@@ -366,51 +441,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool warp_live = im.mt * kBM + q4 * 32 < im.len;
             bool ok = true;
             for (int n0 = 0; n0 < width; n0 += kAccCols, seq++) {
-                if (seq % kEpiGroups != eg) continue;
                 const int acc = seq & (kAccBufs - 1);
                 const int nw = min(kAccCols, width - n0);
+                const int ch = eg * kSliceCols;              // this group's slice of the tile
+                const int sw = max(0, min(kSliceCols, nw - ch));  // a multiple of 32
                 if (!mbar_wait(tmem_full(acc), (seq / kAccBufs) & 1, &abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                for (int ch = 0; ch < nw; ch += 64) {
-                    uint32_t v[64];
-                    const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kAccCols + ch);
-                    tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                    const bool two = ch + 32 < nw;
-                    if (two) tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-                    tmem_wait_ld();
+                uint32_t v[kSliceCols];
+                const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kAccCols + ch);
 #pragma unroll
-                    for (int half = 0; half < 2; half++) {
-                        if (half == 1 && !two) break;
-                        const uint32_t *vv = v + 32 * half;
-                        const int col0 = c0 + n0 + ch + 32 * half;  // first global column of these 32
-                        if (s.K == 8) {
+                for (int q = 0; q < kSliceCols / 32; q++)
+                    if (32 * q < sw) tmem_ld32(ta + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * q]));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(tmem_empty(acc));  // values are in registers: free the accumulator
 #pragma unroll
-                            for (int t = 0; t < 4; t++) {
-                                const uint32_t byte = pack_positive_byte(vv + 8 * t);
-                                const int l = (col0 >> 3) + t;
-                                if (valid && l < s.L)
-                                    static_cast<uint8_t *>(p.codes)[((size_t)im.unit * s.L + l) * s.Ncap + tok] =
-                                        (uint8_t)byte;
+                for (int half = 0; half < kSliceCols / 32; half++) {
+                    if (32 * half >= sw) break;
+                    const uint32_t *vv = v + 32 * half;
+                    const int col0 = c0 + n0 + ch + 32 * half;  // first global column of these 32
+                    if (s.K == 8) {
+                        // 4 table bytes of this token -> 4 tokens of one table per lane
+                        const uint32_t b0 = pack_positive_byte(vv), b1 = pack_positive_byte(vv + 8);
+                        const uint32_t b2 = pack_positive_byte(vv + 16), b3 = pack_positive_byte(vv + 24);
+                        const uint32_t w = quad_transpose(
+                            __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410), lane);
+                        const int l = (col0 >> 3) + (lane & 3);
+                        const int t4 = im.mt * kBM + q4 * 32 + (lane & ~3);  // first of this lane's 4 tokens
+                        if (l < s.L) {
+                            uint8_t *dst = static_cast<uint8_t *>(p.codes) + ((size_t)im.unit * s.L + l) * s.Ncap + t4;
+                            if (t4 + 3 < im.len) {
+                                *reinterpret_cast<uint32_t *>(dst) = w;
+                            } else {
+                                for (int k = 0; k < 4 && t4 + k < im.len; k++) dst[k] = (uint8_t)(w >> (8 * k));
                             }
-                        } else {
-                            uint32_t mine = 0;
-#pragma unroll
-                            for (int j = 0; j < 32; j++) {
-                                const uint32_t wv = __ballot_sync(0xffffffffu, valid && __uint_as_float(vv[j]) > 0.f);
-                                if (lane == j) mine = wv;
-                            }
-                            const int c = col0 + lane;
-                            if (warp_live && c < s.LK)
-                                static_cast<uint32_t *>(p.codes)[((size_t)im.unit * s.L * s.K + c) * words +
-                                                                 ((im.mt * kBM + q4 * 32) >> 5)] = mine;
                         }
+                    } else {
+                        // row word (bit c = column col0 + c) -> column word (bit t = token t)
+                        const uint32_t rw = valid ? pack_positive_word(vv) : 0u;
+                        const uint32_t mine = warp_transpose32(rw, lane);
+                        const int c = col0 + lane;
+                        if (warp_live && c < s.LK)
+                            static_cast<uint32_t *>(p.codes)[((size_t)im.unit * s.L * s.K + c) * words +
+                                                             ((im.mt * kBM + q4 * 32) >> 5)] = mine;
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(tmem_empty(acc));
             }
             if (!ok) break;
         }
