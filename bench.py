@@ -46,6 +46,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--code-layout", default=None, choices=["auto", "bytes", "planes"],
+                   help="key-code layout (default: the workload's, i.e. bytes for K=8, planes for K=10)")
     return p.parse_args()
 
 
@@ -72,9 +74,11 @@ def reduce_over_ranks(total_ms, tokens, device, world):
     return t.item(), n.item()
 
 
-def workload_for_rank(name, rank):
+def workload_for_rank(name, rank, code_layout=None):
     import workloads
     w = workloads.get(name)
+    if code_layout:
+        w = w.with_(code_layout=code_layout)
     return w.with_(seed=w.seed + 7919 * rank) if rank else w
 
 
@@ -139,7 +143,9 @@ class Bench:
         inp = make_inputs(w)
         self.inp = inp
         self.shape = mp.Shape(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.capacity, w.k_bits,
-                              w.n_tables, w.sink, w.window)
+                              w.n_tables, w.sink, w.window,
+                              {"auto": mp.MP_CODES_AUTO, "bytes": mp.MP_CODES_BYTES,
+                               "planes": mp.MP_CODES_PLANES}[w.code_layout])
 
         def dev(a):
             return torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a)).to(device)
@@ -370,6 +376,7 @@ def config_of(w):
     return dict(workload=w.name, batch=w.batch, q_heads=w.n_q_heads, kv_heads=w.n_kv_heads,
                 head_dim=w.head_dim, context=w.context, ragged_min=w.ragged_min or None, k_bits=w.k_bits,
                 n_tables=w.n_tables, sink=w.sink, window=w.window, planted_per_kv_head=w.n_planted,
+                code_layout=w.code_layout if w.code_layout != "auto" else ("bytes" if w.k_bits == 8 else "planes"),
                 step="hash all cached keys + append 1 token/sequence + LSH-sampled decode",
                 l2="flushed between timed steps (256 MiB write)", parallelism="replicas (1 rank = 1 GPU)")
 
@@ -395,7 +402,7 @@ def main():
     device = torch.device("cuda", local if world > 1 else 0)
     import __graft_entry__
     __graft_entry__.build()
-    w = workload_for_rank(args.workload, rank)
+    w = workload_for_rank(args.workload, rank, args.code_layout)
     bench = Bench(w, device)
     union, mean_ns = bench.union_rows()
 

@@ -51,6 +51,11 @@ extern "C" {
 #define MP_ERR_CUDA (-6)      /* a CUDA runtime call or launch failed */
 #define MP_ERR_TOO_LARGE (-7) /* beyond the fixed scratch of mp_decode_attend_noalloc */
 
+/* Key-code layouts (mp_shape.code_layout). */
+#define MP_CODES_AUTO 0   /* k_bits == 8: MP_CODES_BYTES; k_bits == 10: MP_CODES_PLANES */
+#define MP_CODES_BYTES 1  /* one byte per (table, token); k_bits == 8 only */
+#define MP_CODES_PLANES 2 /* bit planes of 32 tokens; any supported k_bits */
+
 /*
  * Problem shape.  Supported: head_dim == 128; k_bits in {8, 10};
  * 2 <= n_tables <= 255 with n_tables * k_bits <= 2048; n_q_heads a multiple of
@@ -67,15 +72,20 @@ typedef struct mp_shape {
     int32_t n_tables;   /* L: hash tables */
     int32_t sink;       /* leading tokens of the exact set D */
     int32_t window;     /* trailing (most recent) tokens of the exact set D */
+    int32_t code_layout; /* MP_CODES_AUTO, MP_CODES_BYTES or MP_CODES_PLANES */
 } mp_shape;
 
 /*
- * Key-code layout ("table-major"), per (b, kv head) unit:
- *   k_bits == 8 : uint8  [B][Hkv][L][Ncap]         one byte per (table, token),
- *                 bit b of the byte = bit b of the code.
- *   k_bits == 10: uint32 [B][Hkv][L][K][Ncap/32]   bit planes: bit t of word
- *                 (l, b, w) = bit b of the table-l code of token 32*w + t.
- * Both use exactly L*K/8 bytes per token.  mp_codes_bytes gives the size.
+ * Key-code layouts ("table-major"), per (b, kv head) unit:
+ *   MP_CODES_BYTES  (k_bits == 8): uint8 [B][Hkv][L][Ncap], one byte per
+ *                   (table, token), bit b of the byte = bit b of the code.
+ *   MP_CODES_PLANES: uint32 [B][Hkv][L][Ncap/32][K] bit planes: bit t of word
+ *                   (l, w, b) = bit b of the table-l code of token 32*w + t
+ *                   (the K planes of each 32-token group are adjacent).
+ * Both use exactly L*K/8 bytes per token; mp_codes_bytes gives the size.  The
+ * byte layout is the default for k_bits == 8; the plane layout lets the
+ * collision scan compare 32 tokens per logical operation (about 4x fewer
+ * integer operations than byte compares for K = 8).
  */
 int mp_codes_bytes(const mp_shape *shape, size_t *bytes);
 

@@ -29,6 +29,9 @@ from ._binding import (  # noqa: F401
     MP_ERR_WORKSPACE,
     MP_ERR_CUDA,
     MP_ERR_TOO_LARGE,
+    MP_CODES_AUTO,
+    MP_CODES_BYTES,
+    MP_CODES_PLANES,
 )
 
 __all__ = [

@@ -17,6 +17,9 @@ MP_ERR_CAPACITY = -4
 MP_ERR_WORKSPACE = -5
 MP_ERR_CUDA = -6
 MP_ERR_TOO_LARGE = -7
+MP_CODES_AUTO = 0
+MP_CODES_BYTES = 1
+MP_CODES_PLANES = 2
 
 
 class MagicPIGError(RuntimeError):
@@ -28,7 +31,7 @@ class MagicPIGError(RuntimeError):
 class _CShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("batch", "n_q_heads", "n_kv_heads", "head_dim", "capacity", "k_bits", "n_tables",
-                 "sink", "window")]
+                 "sink", "window", "code_layout")]
 
 
 class _CDebug(ctypes.Structure):
@@ -48,6 +51,11 @@ class Shape:
     n_tables: int
     sink: int
     window: int
+    code_layout: int = 0  # MP_CODES_AUTO
+
+    @property
+    def planes(self) -> bool:
+        return self.code_layout == MP_CODES_PLANES or (self.code_layout == MP_CODES_AUTO and self.k_bits != 8)
 
     def c(self) -> _CShape:
         return _CShape(*dataclasses.astuple(self))
@@ -121,11 +129,11 @@ def codes_bytes(shape: Shape) -> int:
 
 def codes_shape(shape: Shape):
     """(dtype name, tensor shape) of the key codes: uint8 [B,Hkv,L,Ncap] for
-    K = 8, int32-bit planes [B,Hkv,L,K,Ncap/32] for K = 10."""
+    byte codes, int32 bit planes [B,Hkv,L,Ncap/32,K] for plane codes."""
     B, Hkv, L, K, N = shape.batch, shape.n_kv_heads, shape.n_tables, shape.k_bits, shape.capacity
-    if K == 8:
+    if not shape.planes:
         return "uint8", (B, Hkv, L, N)
-    return "int32", (B, Hkv, L, K, N // 32)
+    return "int32", (B, Hkv, L, N // 32, K)
 
 
 def decode_workspace_bytes(shape: Shape, max_len: int) -> int:

@@ -23,9 +23,18 @@ int validate_shape(const mp_shape *in, Shape &s)
     s.L = in->n_tables;
     s.sink = in->sink;
     s.window = in->window;
+    if (in->code_layout == MP_CODES_AUTO)
+        s.planes = in->k_bits != 8;
+    else if (in->code_layout == MP_CODES_BYTES)
+        s.planes = 0;
+    else if (in->code_layout == MP_CODES_PLANES)
+        s.planes = 1;
+    else
+        return MP_ERR_SHAPE;
     if (s.B < 1 || s.Hq < 1 || s.Hkv < 1 || s.sink < 0 || s.window < 0) return MP_ERR_SHAPE;
     if (s.d != kHeadDim) return MP_ERR_SHAPE;
     if (s.K != 8 && s.K != 10) return MP_ERR_SHAPE;
+    if (!s.planes && s.K != 8) return MP_ERR_SHAPE;
     if (s.L < 2 || s.L > 255 || s.L * s.K > 2048) return MP_ERR_SHAPE;
     if (s.Hq % s.Hkv != 0) return MP_ERR_SHAPE;
     s.G = s.Hq / s.Hkv;

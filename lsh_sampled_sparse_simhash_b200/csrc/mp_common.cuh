@@ -13,14 +13,15 @@ constexpr int kMaxGroup = 8;
 constexpr int kScanThreads = 256;  // scan block: token groups x table splits
 constexpr int kSplitsK8 = 8;       // byte codes: tables l = ts, ts + 8, ... per split
 constexpr int kSplitsK10 = 4;      // bit planes: tables l = ts, ts + 4, ...
-constexpr int kChunkK8 = 512;      // scan chunk (tokens) for byte codes: 32 groups x 16 tokens
-constexpr int kChunkK10 = 8192;    // scan chunk (tokens) for bit planes: 64 groups x 128 tokens
+constexpr int kChunkBytes = 512;   // scan chunk (tokens) for byte codes: 32 groups x 16 tokens
+constexpr int kChunkPlanes = 8192; // scan chunk (tokens) for bit planes: 64 groups x 128 tokens
 
 struct Shape {
     int B, Hq, Hkv, G, d, Ncap, K, L, LK, sink, window;
+    int planes;  // 1: bit-plane codes, 0: one byte per (table, token)
 };
 
-inline int chunk_tokens(int K) { return K == 8 ? kChunkK8 : kChunkK10; }
+inline int chunk_tokens(const Shape &s) { return s.planes ? kChunkPlanes : kChunkBytes; }
 
 // Device-side status word: the first error wins, later ones are dropped.
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code)

@@ -24,21 +24,26 @@
 namespace mp {
 
 // ------------------------------------------------------------------ qhash ---
-// grid (ceil(L / TB), B * Hkv), 256 threads; thread = one hyperplane column of
-// a table-aligned block of TB = 256 / K tables; the G query heads of one kv
-// head share the W row loads.
+// grid (ceil(L / TB), B * Hkv), 256 threads.  A block covers TB = 64 / K whole
+// tables (64 or 60 hyperplane columns); four lanes share a column, each summing
+// 32 of the 128 products for all G heads of the kv group (one W load serves G
+// heads), then two shuffles finish the sums.
+constexpr int kQhashCols = 64;
+
+inline int qhash_tables_per_block(int K) { return kQhashCols / K; }
+
 template <int G>
 __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__restrict__ q,
                                                     const uint16_t *__restrict__ W,
                                                     const uint16_t *__restrict__ qcodes_in,
                                                     uint16_t *__restrict__ qcodes, int32_t *status)
 {
-    __shared__ float qs[G][kHeadDim];
-    __shared__ uint8_t bits[G][256];
+    __shared__ float qs[G][kHeadDim + 4];  // element d at d + d / 32: the 4 quarters hit distinct banks
+    __shared__ uint8_t bits[G][kQhashCols];
     const int tid = threadIdx.x;
     const int unit = blockIdx.y;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
-    const int TB = 256 / s.K;
+    const int TB = kQhashCols / s.K;
     const int l0 = blockIdx.x * TB;
     const size_t vec0 = (size_t)b * s.Hq + (size_t)kvh * G;
 
@@ -52,34 +57,47 @@ __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__r
         }
         return;
     }
-    for (int i = tid; i < G * kHeadDim; i += blockDim.x)
-        qs[i / kHeadDim][i % kHeadDim] = bf16_to_f32(q[(vec0 + i / kHeadDim) * kHeadDim + i % kHeadDim]);
+    for (int i = tid; i < G * kHeadDim; i += blockDim.x) {
+        const int d = i % kHeadDim;
+        qs[i / kHeadDim][d + (d >> 5)] = bf16_to_f32(q[(vec0 + i / kHeadDim) * kHeadDim + d]);
+    }
     __syncthreads();
 
-    const int c = l0 * s.K + tid;
-    const bool valid = tid < TB * s.K && c < s.LK;
+    const int cl = tid >> 2, part = tid & 3;  // column within the block, quarter of the dims
+    const int c = l0 * s.K + cl;
+    const bool valid = cl < TB * s.K && c < s.LK;
     float acc[G];
 #pragma unroll
     for (int g = 0; g < G; g++) acc[g] = 0.f;
     if (valid) {
-        const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)c * kHeadDim);
-#pragma unroll 4
-        for (int j8 = 0; j8 < kHeadDim / 8; j8++) {
-            uint4 w = __ldg(wr + j8);
-            uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+        const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)c * kHeadDim + part * 32);
+        uint4 w4[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) w4[j] = __ldg(wr + j);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const uint32_t wv[4] = {w4[j].x, w4[j].y, w4[j].z, w4[j].w};
 #pragma unroll
             for (int e = 0; e < 4; e++) {
-                float w0 = bf16_lo(wv[e]), w1 = bf16_hi(wv[e]);
+                const int dd = part * 33 + j * 8 + 2 * e;  // padded index of dim part * 32 + j * 8 + 2 e
+                const float w0 = bf16_lo(wv[e]), w1 = bf16_hi(wv[e]);
 #pragma unroll
                 for (int g = 0; g < G; g++) {
-                    acc[g] = fmaf(w0, qs[g][j8 * 8 + 2 * e], acc[g]);
-                    acc[g] = fmaf(w1, qs[g][j8 * 8 + 2 * e + 1], acc[g]);
+                    acc[g] = fmaf(w0, qs[g][dd], acc[g]);
+                    acc[g] = fmaf(w1, qs[g][dd + 1], acc[g]);
                 }
             }
         }
     }
 #pragma unroll
-    for (int g = 0; g < G; g++) bits[g][tid] = valid && acc[g] > 0.f;
+    for (int g = 0; g < G; g++) {
+        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
+        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 2);
+    }
+    if (part == 0) {
+#pragma unroll
+        for (int g = 0; g < G; g++) bits[g][cl] = valid && acc[g] > 0.f;
+    }
     __syncthreads();
     if (tid < G * TB) {
         const int g = tid / TB, tl = tid % TB, l = l0 + tl;
@@ -136,6 +154,17 @@ __device__ __forceinline__ int block_sum(int v, int *scratch)
     int t = 0;
     for (int w = 0; w < nwarp; w++) t += scratch[w];
     return t;
+}
+
+// 16-byte read-only load that allocates in L1 (the plane scan touches each
+// 32-byte sector with two consecutive loads).
+__device__ __forceinline__ uint4 ld_cached_16(const void *p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
 }
 
 // Streaming 16-byte load that does not allocate in L1.
@@ -271,7 +300,7 @@ __device__ __forceinline__ void combine_splits(uint32_t (&s1)[G][NW], uint32_t (
     }
 }
 
-// ---------------------------------------------------------- scan, K = 8 ----
+// -------------------------------------------------- scan, byte codes (K = 8) ----
 // Byte codes [unit][L][Ncap].  A 512-token chunk per block of 256 threads:
 // 32 token groups of 16 tokens (one 16-byte load per table) x 8 table splits
 // (tables ts, ts + 8, ...; up to 8 loads in flight per thread), merged in
@@ -296,7 +325,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
     grid_dependency_wait();
     const int N = clamp_len(seq_lens, b, max_len, o.status, chunk == 0 && kvh == 0 && threadIdx.x == 0);
-    const int c0 = chunk * kChunkK8;
+    const int c0 = chunk * kChunkBytes;
     if (c0 >= N) return;
     for (int i = threadIdx.x; i < s.L * G; i += blockDim.x) {
         const int l = i / G, g = i % G;
@@ -350,36 +379,38 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
         hm[g][0] = ts == 0 ? m : 0u;
     }
     // Tokens eligible for S: [sink, N - window) and below N.
-    compact_and_store<G, 1, 16>(s, unit, chunk, nchunk, kChunkK8, t0, N, s.sink, min(N - s.window, N), hm,
+    compact_and_store<G, 1, 16>(s, unit, chunk, nchunk, kChunkBytes, t0, N, s.sink, min(N - s.window, N), hm,
                                 ts == 0, o, scratch);
 }
 
-// --------------------------------------------------------- scan, K = 10 ----
-// Bit-plane codes [unit][L][K][Ncap/32] (uint32).  An 8192-token chunk per
-// block of 256 threads: 64 token groups of 128 tokens (one 16-byte load per
-// plane) x 4 table splits.  A token mismatches table l for head h iff some
+// ------------------------------------------------------ scan, bit planes ----
+// Bit-plane codes [unit][L][Ncap/32][K] (uint32).  An 8192-token chunk per
+// block of 256 threads: 64 token groups of 128 tokens (4 words x K planes,
+// 16 K contiguous bytes per table, so a warp streams 512 K contiguous bytes)
+// x 4 table splits.  A token mismatches table l for head h iff some
 // plane differs from the query bit: mis = OR_b (plane_b ^ qmask_b), with
-// qmask_b = 0 or ~0 from shared memory.
-template <int G>
-__global__ void __launch_bounds__(kScanThreads) scan_k10_kernel(
+// qmask_b = 0 or ~0 from shared memory (KB + 2 logic operations per 32
+// tokens per table and head).
+template <int G, int KB>
+__global__ void __launch_bounds__(kScanThreads) scan_planes_kernel(
     Shape s, const uint32_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
     const int32_t *__restrict__ seq_lens, int max_len, int nchunk, ScanOut o)
 {
-    extern __shared__ uint32_t dyn[];  // qm [L][G][12] (qmask of the 10 planes, padded), then split partials
+    constexpr int QW = (KB + 3) & ~3;  // query masks per (table, head), padded to whole uint4s
+    extern __shared__ uint32_t dyn[];  // qm [L][G][QW] (qmask of the KB planes), then split partials
     uint32_t *qm = dyn;
-    uint32_t *part = dyn + s.L * G * 12;
+    uint32_t *part = dyn + s.L * G * QW;
     __shared__ int scratch[64];
-    constexpr int KB = 10;
     constexpr int TS = kSplitsK10, TG = kScanThreads / TS;
     const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
     const int unit = blockIdx.y, chunk = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
     grid_dependency_wait();
     const int N = clamp_len(seq_lens, b, max_len, o.status, chunk == 0 && kvh == 0 && threadIdx.x == 0);
-    const int c0 = chunk * kChunkK10;
+    const int c0 = chunk * kChunkPlanes;
     if (c0 >= N) return;
-    for (int i = threadIdx.x; i < s.L * G * 12; i += blockDim.x) {
-        const int l = i / (G * 12), g = (i / 12) % G, bb = i % 12;
+    for (int i = threadIdx.x; i < s.L * G * QW; i += blockDim.x) {
+        const int l = i / (G * QW), g = (i / QW) % G, bb = i % QW;
         const unsigned code = qcodes[((size_t)b * s.Hq + kvh * G + g) * s.L + l];
         qm[i] = bb < KB ? 0u - ((code >> bb) & 1u) : 0u;
     }
@@ -394,24 +425,37 @@ __global__ void __launch_bounds__(kScanThreads) scan_k10_kernel(
         for (int j = 0; j < 4; j++) s1[g][j] = s2[g][j] = 0u;
 
     if (t0 < N) {
-        const uint32_t *base = codes + (size_t)unit * s.L * KB * words + (t0 >> 5);
+        // this thread's 4 words x KB planes of one table: 16 * KB contiguous bytes
+        const uint32_t *base = codes + ((size_t)unit * s.L * words + (t0 >> 5)) * KB;
 #pragma unroll 1
         for (int l = ts; l < s.L; l += TS) {
-            uint4 pl[KB];
+            const uint4 *src = reinterpret_cast<const uint4 *>(base + (size_t)l * words * KB);
+            uint32_t pw[4 * KB];  // pw[j * KB + b] = plane b of token word j
 #pragma unroll
-            for (int bb = 0; bb < KB; bb++) pl[bb] = ld_stream_16(base + ((size_t)l * KB + bb) * words);
+            for (int q = 0; q < KB; q++) {
+                const uint4 v = ld_cached_16(src + q);
+                pw[4 * q] = v.x;
+                pw[4 * q + 1] = v.y;
+                pw[4 * q + 2] = v.z;
+                pw[4 * q + 3] = v.w;
+            }
 #pragma unroll
             for (int g = 0; g < G; g++) {
-                const uint4 *m4 = reinterpret_cast<const uint4 *>(qm + (l * G + g) * 12);
-                const uint4 ma = m4[0], mb = m4[1], mc = m4[2];
-                const uint32_t msk[KB] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w, mc.x, mc.y};
+                const uint4 *m4 = reinterpret_cast<const uint4 *>(qm + (l * G + g) * QW);
+                uint32_t msk[QW];
+#pragma unroll
+                for (int q = 0; q < QW / 4; q++) {
+                    const uint4 mq = m4[q];
+                    msk[4 * q] = mq.x;
+                    msk[4 * q + 1] = mq.y;
+                    msk[4 * q + 2] = mq.z;
+                    msk[4 * q + 3] = mq.w;
+                }
                 uint32_t mis[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                 for (int bb = 0; bb < KB; bb++) {
-                    mis[0] |= pl[bb].x ^ msk[bb];
-                    mis[1] |= pl[bb].y ^ msk[bb];
-                    mis[2] |= pl[bb].z ^ msk[bb];
-                    mis[3] |= pl[bb].w ^ msk[bb];
+#pragma unroll
+                    for (int j = 0; j < 4; j++) mis[j] |= pw[j * KB + bb] ^ msk[bb];
                 }
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
@@ -428,7 +472,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_k10_kernel(
 #pragma unroll
             for (int j = 0; j < 4; j++) s2[g][j] = 0u;
     }
-    compact_and_store<G, 4, 32>(s, unit, chunk, nchunk, kChunkK10, t0, N, s.sink, min(N - s.window, N), s2,
+    compact_and_store<G, 4, 32>(s, unit, chunk, nchunk, kChunkPlanes, t0, N, s.sink, min(N - s.window, N), s2,
                                 ts == 0, o, scratch);
 }
 
@@ -463,7 +507,7 @@ __device__ __forceinline__ float log_sampling_prob(float c, const LogU &u)
 constexpr int kAttThreads = 128;
 constexpr int kMaxSpan = 64;                // scan chunks per attention block, at most
 constexpr int kAttRows = 64;                // rows per tile (4 warps x 16)
-constexpr int kAttStages = 3;               // cp.async ring depth
+constexpr int kAttStages = 2;               // cp.async ring depth (3 blocks fit per SM)
 constexpr int kRowBytes = kHeadDim * 2;     // 256
 constexpr int kRowStride = kRowBytes + 16;  // padded: conflict-free ldmatrix / 8-byte reads
 constexpr int kStageBytes = kAttRows * kRowStride * 2;  // K rows then V rows
@@ -520,7 +564,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 //           split into bf16 hi + lo parts (error ~2^-17 relative), transposed
 //           into B fragments with movmatrix, V^T comes from ldmatrix.trans.
 template <int G>
-__global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
+__global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ uint32_t meta[kAttStages][kAttRows];  // headmask | exact << 8
@@ -675,29 +719,28 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a)
         const uint8_t *vs_ = ks_ + kAttRows * kRowStride;
 
         // ---- S^T = K rows . Q^T and |k|^2 ----
+        // The A fragments of K double as B fragments of K^T, so two more MMAs
+        // per k-step give the 16x16 Gram matrix K K^T, whose diagonal is |k|^2.
         float c[4] = {0.f, 0.f, 0.f, 0.f};
-        float na = 0.f, nb = 0.f;
+        float na, nb;
         {
+            float g0[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f};
             const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStride + (lane >> 4) * 16;
 #pragma unroll
             for (int kst = 0; kst < 8; kst++) {
                 uint32_t a0, a1, a2, a3;
                 ldmatrix_x4(a0, a1, a2, a3, arow + kst * 32);
                 mma_bf16_16816(c[0], c[1], c[2], c[3], a0, a1, a2, a3, qb[kst][0], qb[kst][1]);
-                float x;
-                x = bf16_lo(a0); na = fmaf(x, x, na);
-                x = bf16_hi(a0); na = fmaf(x, x, na);
-                x = bf16_lo(a2); na = fmaf(x, x, na);
-                x = bf16_hi(a2); na = fmaf(x, x, na);
-                x = bf16_lo(a1); nb = fmaf(x, x, nb);
-                x = bf16_hi(a1); nb = fmaf(x, x, nb);
-                x = bf16_lo(a3); nb = fmaf(x, x, nb);
-                x = bf16_hi(a3); nb = fmaf(x, x, nb);
+                mma_bf16_16816(g0[0], g0[1], g0[2], g0[3], a0, a1, a2, a3, a0, a2);  // columns: rows 0-7
+                mma_bf16_16816(g1[0], g1[1], g1[2], g1[3], a0, a1, a2, a3, a1, a3);  // columns: rows 8-15
             }
-            na += __shfl_xor_sync(0xffffffffu, na, 1);
-            na += __shfl_xor_sync(0xffffffffu, na, 2);
-            nb += __shfl_xor_sync(0xffffffffu, nb, 1);
-            nb += __shfl_xor_sync(0xffffffffu, nb, 2);
+            // |k_r|^2 = Gram[r][r]: row gq sits in lane 4 gq + gq/2 (g0, element gq & 1),
+            // row gq + 8 in the same lane (g1, element 2 + (gq & 1)).
+            const int src = 4 * gq + (gq >> 1);
+            const float d0 = (gq & 1) ? g0[1] : g0[0];
+            const float d1 = (gq & 1) ? g1[3] : g1[2];
+            na = __shfl_sync(0xffffffffu, d0, src);
+            nb = __shfl_sync(0xffffffffu, d1, src);
         }
 
         // ---- log-weights: s (exact) or s - log u (sampled), -inf if absent ----
@@ -943,10 +986,9 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // How attention blocks cover the scan chunks.  Many chunks: each block takes
 // `span` consecutive chunks (about 600 blocks in all, so that the per-block
-// set-up is amortised and the merge sees few partials).  Few chunks: each
-// chunk's list is shared by `subs` blocks so that about 296 blocks (two per
-// SM on 148 SMs) run.  Fixed counts, so the workspace size does not depend on
-// the device.
+// set-up is amortised and the merge sees few partials).  Few, large chunks:
+// each chunk's list is shared by `subs` blocks.  Fixed counts, so the
+// workspace size does not depend on the device.
 struct SplitPlan {
     int nchunk, span, subs, ngroups, nsplit;
 };
@@ -954,15 +996,18 @@ struct SplitPlan {
 static SplitPlan split_plan(const Shape &s, int max_len)
 {
     SplitPlan p;
-    const int C = chunk_tokens(s.K);
+    const int C = chunk_tokens(s);
     p.nchunk = (max_len + C - 1) / C;
     const int blocks = p.nchunk * s.B * s.Hkv;
     if (blocks >= 600) {
         p.span = std::min(kMaxSpan, blocks / 600);
         p.subs = 1;
     } else {
+        // few chunks: split each chunk's list so that about 1200 blocks run,
+        // but give every block at least ~1024 tokens' worth of candidates
         p.span = 1;
-        p.subs = blocks > 0 ? std::max(1, std::min(8, 296 / blocks)) : 1;
+        const int by_count = blocks > 0 ? (1200 + blocks - 1) / blocks : 1;
+        p.subs = std::max(1, std::min({8, by_count, C / 1024}));
     }
     p.ngroups = (p.nchunk + p.span - 1) / p.span;
     p.nsplit = p.ngroups * p.subs + 1;
@@ -971,7 +1016,7 @@ static SplitPlan split_plan(const Shape &s, int max_len)
 
 Workspace workspace_layout(const Shape &s, int max_len, void *base)
 {
-    const int C = chunk_tokens(s.K);
+    const int C = chunk_tokens(s);
     const SplitPlan sp = split_plan(s, max_len);
     const int nchunk = sp.nchunk;
     const size_t nsplit = (size_t)sp.nsplit;
@@ -1016,13 +1061,14 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
                                    int max_len, float *out, float *lse, int32_t *n_sampled,
                                    const Workspace &ws, const mp_decode_debug *dbg, cudaStream_t st)
 {
-    const int C = chunk_tokens(s.K);
+    const int C = chunk_tokens(s);
     const SplitPlan sp = split_plan(s, max_len);
     const int nchunk = sp.nchunk;
     const int units = s.B * s.Hkv;
     cudaError_t e;
     {
-        dim3 grid((s.L + 256 / s.K - 1) / (256 / s.K), units);
+        const int TB = qhash_tables_per_block(s.K);
+        dim3 grid((s.L + TB - 1) / TB, units);
         e = launch_pdl(qhash_kernel<G>, grid, dim3(256), 0, st, s, q, W,
                        (const uint16_t *)(dbg ? dbg->qcodes_in : nullptr), ws.qcodes, ws.status);
         if (e != cudaSuccess) return e;
@@ -1031,16 +1077,24 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     if (nchunk > 0) {
         dim3 grid(nchunk, units);
         const size_t part = (size_t)2 * G * 4 * kScanThreads * sizeof(uint32_t);
-        if (s.K == 8) {
+        if (!s.planes) {
             const size_t sm = (size_t)((s.L * G + 3) & ~3) * sizeof(uint32_t) + part;
             if ((e = ensure_smem(reinterpret_cast<const void *>(scan_k8_kernel<G>), (int)sm)) != cudaSuccess) return e;
             e = launch_pdl(scan_k8_kernel<G>, grid, dim3(kScanThreads), sm, st, s,
                            static_cast<const uint8_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
                            nchunk, so);
+        } else if (s.K == 8) {
+            const size_t sm = (size_t)s.L * G * 8 * sizeof(uint32_t) + part;
+            if ((e = ensure_smem(reinterpret_cast<const void *>(scan_planes_kernel<G, 8>), (int)sm)) != cudaSuccess)
+                return e;
+            e = launch_pdl(scan_planes_kernel<G, 8>, grid, dim3(kScanThreads), sm, st, s,
+                           static_cast<const uint32_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
+                           nchunk, so);
         } else {
             const size_t sm = (size_t)s.L * G * 12 * sizeof(uint32_t) + part;
-            if ((e = ensure_smem(reinterpret_cast<const void *>(scan_k10_kernel<G>), (int)sm)) != cudaSuccess) return e;
-            e = launch_pdl(scan_k10_kernel<G>, grid, dim3(kScanThreads), sm, st, s,
+            if ((e = ensure_smem(reinterpret_cast<const void *>(scan_planes_kernel<G, 10>), (int)sm)) != cudaSuccess)
+                return e;
+            e = launch_pdl(scan_planes_kernel<G, 10>, grid, dim3(kScanThreads), sm, st, s,
                            static_cast<const uint32_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
                            nchunk, so);
         }
@@ -1100,7 +1154,8 @@ cudaError_t launch_decode(const Shape &s, const uint16_t *q, const uint16_t *W, 
 cudaError_t launch_hash_queries(const Shape &s, const uint16_t *q, const uint16_t *W, uint16_t *qcodes,
                                 cudaStream_t st)
 {
-    dim3 grid((s.L + 256 / s.K - 1) / (256 / s.K), s.B * s.Hkv);
+    const int TB = qhash_tables_per_block(s.K);
+    dim3 grid((s.L + TB - 1) / TB, s.B * s.Hkv);
     const uint16_t *none = nullptr;
     int32_t *no_status = nullptr;
     switch (s.G) {

@@ -3,8 +3,9 @@
 // interface).  The bulk key hash is the tensor-core kernel in mp_hash_tc.cu.
 //
 // Code layouts (table-major, exactly L*K/8 bytes per token):
-//   K = 8 : uint8  [unit][L][Ncap], bit b of the byte = bit b of the code.
-//   K = 10: uint32 [unit][L][K][Ncap/32], bit t of word w = token 32 w + t.
+//   bytes : uint8  [unit][L][Ncap], bit b of the byte = bit b of the code.
+//   planes: uint32 [unit][L][Ncap/32][K], bit t of word (w, b) = bit b of the
+//           code of token 32 w + t.
 #include "mp_common.cuh"
 #include "mp_kernels.cuh"
 
@@ -63,7 +64,7 @@ __global__ void __launch_bounds__(256) append_kernel(Shape s, const uint16_t *__
         }
         bit = dot > 0.f;
     }
-    if (s.K == 8) {
+    if (!s.planes) {
         bits[tid] = bit;
         __syncthreads();
         if (tid < TB && l0 + tid < s.L) {
@@ -72,8 +73,9 @@ __global__ void __launch_bounds__(256) append_kernel(Shape s, const uint16_t *__
             static_cast<uint8_t *>(codes)[((size_t)unit * s.L + l0 + tid) * s.Ncap + pos] = (uint8_t)code;
         }
     } else if (valid) {
+        const int l = c / s.K, bb = c - l * s.K;
         unsigned int *word =
-            static_cast<unsigned int *>(codes) + ((size_t)unit * s.L * s.K + c) * (s.Ncap >> 5) + (pos >> 5);
+            static_cast<unsigned int *>(codes) + (((size_t)unit * s.L + l) * (s.Ncap >> 5) + (pos >> 5)) * s.K + bb;
         const unsigned int m = 1u << (pos & 31);
         if (bit)
             atomicOr(word, m);

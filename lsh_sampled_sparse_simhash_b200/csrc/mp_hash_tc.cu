@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (32 * half >= sw) break;
                     const uint32_t *vv = v + 32 * half;
                     const int col0 = c0 + n0 + ch + 32 * half;  // first global column of these 32
-                    if (s.K == 8) {
+                    if (!s.planes) {
                         // 4 table bytes of this token -> 4 tokens of one table per lane
                         const uint32_t b0 = pack_positive_byte(vv), b1 = pack_positive_byte(vv + 8);
                         const uint32_t b2 = pack_positive_byte(vv + 16), b3 = pack_positive_byte(vv + 24);
@@ -484,9 +484,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t rw = valid ? pack_positive_word(vv) : 0u;
                         const uint32_t mine = warp_transpose32(rw, lane);
                         const int c = col0 + lane;
-                        if (warp_live && c < s.LK)
-                            static_cast<uint32_t *>(p.codes)[((size_t)im.unit * s.L * s.K + c) * words +
-                                                             ((im.mt * kBM + q4 * 32) >> 5)] = mine;
+                        if (warp_live && c < s.LK) {
+                            const int l = c / s.K, b = c - l * s.K;
+                            static_cast<uint32_t *>(p.codes)[(((size_t)im.unit * s.L + l) * words +
+                                                              ((im.mt * kBM + q4 * 32) >> 5)) * s.K + b] = mine;
+                        }
                     }
                 }
             }

@@ -34,9 +34,12 @@ def host(t: torch.Tensor, dtype=None) -> np.ndarray:
     return a
 
 
+LAYOUTS = {"auto": 0, "bytes": 1, "planes": 2}
+
+
 def shape_of(w: Workload) -> mp.Shape:
     return mp.Shape(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.capacity, w.k_bits, w.n_tables,
-                    w.sink, w.window)
+                    w.sink, w.window, LAYOUTS[w.code_layout])
 
 
 class Run:
@@ -84,19 +87,20 @@ class Run:
     def set_codes(self, logical: np.ndarray, units: Optional[Sequence] = None):
         """Writes oracle codes (logical [B,Hkv,N,L] or, with units, [n][N,L])."""
         w = self.w
+        planes = self.shape.planes
         if units is None:
-            packed = pack_codes(logical, w.k_bits, w.capacity)
+            packed = pack_codes(logical, w.k_bits, w.capacity, planes)
             self.codes.copy_(dev(packed).view(self.codes.dtype))
         else:
             for (b, kh), lg in zip(units, logical):
-                packed = pack_codes(lg, w.k_bits, w.capacity)
+                packed = pack_codes(lg, w.k_bits, w.capacity, planes)
                 self.codes[b, kh].copy_(dev(packed).view(self.codes.dtype))
 
     def codes_logical(self, b: int, kh: int, n: int) -> np.ndarray:
         a = host(self.codes[b, kh])
-        if self.w.k_bits == 10:
+        if self.shape.planes:
             a = a.view(np.uint32)
-        return unpack_codes(a, self.w.k_bits, self.w.n_tables, n)
+        return unpack_codes(a, self.w.k_bits, self.w.n_tables, n, self.shape.planes)
 
     def decode(self, qcodes_in: Optional[np.ndarray] = None, member: bool = True):
         w = self.w

@@ -23,7 +23,7 @@ def lib():
 
 def good_shape(**kw):
     d = dict(batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, capacity=1024, k_bits=8, n_tables=75,
-             sink=4, window=64)
+             sink=4, window=64, code_layout=0)
     d.update(kw)
     return B._CShape(*d.values())
 
@@ -53,8 +53,8 @@ def test_status_strings(lib):
 
 def test_codes_bytes_formula(lib):
     n = ctypes.c_size_t()
-    for K, L in [(8, 75), (10, 150)]:
-        s = good_shape(k_bits=K, n_tables=L)
+    for K, L, lay in [(8, 75, 0), (10, 150, 0), (8, 75, 2), (8, 75, 1), (10, 150, 2)]:
+        s = good_shape(k_bits=K, n_tables=L, code_layout=lay)
         assert lib.mp_codes_bytes(ctypes.byref(s), ctypes.byref(n)) == 0
         assert n.value == 2 * 2 * L * K * 1024 // 8
 
@@ -62,7 +62,8 @@ def test_codes_bytes_formula(lib):
 @pytest.mark.parametrize("bad", [
     dict(head_dim=64), dict(k_bits=9), dict(n_tables=1), dict(n_tables=256), dict(n_q_heads=6),
     dict(n_q_heads=32, n_kv_heads=2), dict(capacity=1000), dict(capacity=0), dict(batch=0),
-    dict(sink=-1), dict(window=-1), dict(n_kv_heads=0)])
+    dict(sink=-1), dict(window=-1), dict(n_kv_heads=0), dict(code_layout=3), dict(code_layout=-1),
+    dict(k_bits=10, n_tables=150, code_layout=1)])
 def test_bad_shapes_rejected(lib, bad):
     n = ctypes.c_size_t()
     s = good_shape(**bad)

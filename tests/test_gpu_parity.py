@@ -32,6 +32,9 @@ SMALL_CASES = {
                         seed=2004),
     "g4_k8_mu_offset": TINY.with_(name="mu", batch=2, n_q_heads=8, n_kv_heads=2, context=6000,
                                   mu_norm=8.0, n_planted=16, seed=2005),
+    "g4_k8_planes": TINY.with_(name="k8p", batch=2, n_q_heads=8, n_kv_heads=2, context=9100, n_planted=16,
+                               seed=2006, code_layout="planes"),
+    "g1_k8_planes_short": TINY.with_(name="k8p1", context=1000, n_planted=8, seed=2007, code_layout="planes"),
 }
 
 
@@ -91,7 +94,7 @@ def test_decode_same_codes_matches_oracle(case):
     assert gpu["ns"].sum() > 0 or w.context <= w.sink + w.window
 
 
-@pytest.mark.parametrize("case", ["tiny_g1_k8", "g4_k10", "g8_k8"])
+@pytest.mark.parametrize("case", ["tiny_g1_k8", "g4_k10", "g8_k8", "g4_k8_planes"])
 def test_end_to_end_gpu_codes(case):
     """GPU hashing feeds the GPU scan.  Where a GPU code equals the oracle's,
     membership must agree; when every code agrees, so must the outputs."""
@@ -118,11 +121,12 @@ def test_end_to_end_gpu_codes(case):
 def test_hash_respects_per_sequence_lengths():
     """With seq_lens, tokens at and past each sequence's length keep their old codes."""
     w = SMALL_CASES["g4_k8_ragged_tail"].with_(batch=3)
-    for K, L in [(8, 75), (10, 150)]:
-        wk = w.with_(k_bits=K, n_tables=L)
+    for K, L, layout in [(8, 75, "auto"), (10, 150, "auto"), (8, 75, "planes")]:
+        wk = w.with_(k_bits=K, n_tables=L, code_layout=layout)
         inp = make_inputs(wk)
         run = Run(wk, inp)
-        sentinel = 0x5A if K == 8 else 0x5A5A5A5A
+        planes = layout == "planes" or K == 10
+        sentinel = 0x5A5A5A5A if planes else 0x5A
         run.codes.fill_(sentinel)
         lens = torch.tensor([0, 1000, 4099], dtype=torch.int32, device="cuda")
         run.hash_keys(wk.context, seq_lens=lens)
@@ -132,8 +136,8 @@ def test_hash_respects_per_sequence_lengths():
                 if n:
                     ref, margin = oracle_unit_codes(inp, wk, b, kh, n)
                     assert code_mismatch(run.codes_logical(b, kh, n), ref, margin, K)[0] == 0
-                tail = codes_h[b, kh][..., (n + 31) // 32 + 1:] if K == 10 else codes_h[b, kh][..., n:]
-                assert (tail.view(np.uint32 if K == 10 else np.uint8) == sentinel).all()
+                tail = codes_h[b, kh][..., (n + 31) // 32 + 1:] if planes else codes_h[b, kh][..., n:]
+                assert (tail.view(np.uint32 if planes else np.uint8) == sentinel).all()
 
 
 def test_short_and_empty_contexts():
@@ -174,12 +178,12 @@ def test_every_token_sampled():
     assert (gpu["ns"] == n - w.sink - w.window).all()
 
 
-@pytest.mark.parametrize("K,L", [(8, 75), (10, 150)])
-def test_keys_on_hyperplanes_get_zero_bits(K, L):
+@pytest.mark.parametrize("K,L,layout", [(8, 75, "auto"), (10, 150, "auto"), (8, 75, "planes")])
+def test_keys_on_hyperplanes_get_zero_bits(K, L, layout):
     """Hand-built ties: W[c] = e_j - e_{j+1} and keys with k_j == k_{j+1} have
     projection exactly 0, which must give bit 0 (strict > 0 rule)."""
     w = TINY.with_(name="ties", batch=1, n_q_heads=1, n_kv_heads=1, context=256, k_bits=K, n_tables=L,
-                   n_planted=0, seed=2012)
+                   n_planted=0, seed=2012, code_layout=layout)
     inp = make_inputs(w)
     d = 128
     Wf = np.zeros((L * K, d), np.float32)
@@ -200,7 +204,7 @@ def test_keys_on_hyperplanes_get_zero_bits(K, L):
 
 
 def test_append_then_decode_equals_rehash():
-    for w in (SMALL_CASES["g4_k8_ragged_tail"], SMALL_CASES["g4_k10"]):
+    for w in (SMALL_CASES["g4_k8_ragged_tail"], SMALL_CASES["g4_k10"], SMALL_CASES["g4_k8_planes"]):
         inp = make_inputs(w)
         run = Run(w, inp)
         run.alloc_decode(w.context + 1)
@@ -271,7 +275,7 @@ def test_overlong_length_is_clamped_and_reported():
 
 # ------------------------------------------------ full-size configurations ----
 
-FULL = ["llama8b_16k", "batch8_64k", "batch4_128k", "ragged16"]
+FULL = ["llama8b_16k", "batch8_64k", "batch4_128k", "ragged16", "ragged16_planes"]
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -279,7 +283,7 @@ def test_full_size_sampled_units(name):
     """The full workload in the benchmark's launch configuration (hash every
     key, append one token per sequence, decode); two (b, kv head) units are
     checked against the oracle on the oracle's own codes."""
-    w = WORKLOADS[name]
+    w = WORKLOADS[name] if name in WORKLOADS else WORKLOADS[name.rsplit("_", 1)[0]].with_(code_layout="planes")
     inp = make_inputs(w)
     run = Run(w, inp)
     run.alloc_decode(run.max_len + 1)

@@ -39,7 +39,6 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(case):
     import __graft_entry__
     __graft_entry__.build()
     import lsh_sampled_sparse_simhash_b200 as mp
-    from lsh_sampled_sparse_simhash_b200._binding import _CShape
     from workloads import make_inputs
 
     assert torch.cuda.is_available()
@@ -70,8 +69,7 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(case):
     assert mp.read_status(ws) == 0
 
     lib = mp.library()
-    cs = _CShape(*[getattr(shape, f) for f in ("batch", "n_q_heads", "n_kv_heads", "head_dim", "capacity",
-                                                "k_bits", "n_tables", "sink", "window")])
+    cs = shape.c()
     stream = torch.cuda.current_stream().cuda_stream
     for call in range(2):  # consecutive calls share (and inherit) the scratch contents
         out, lse, ns = outputs()
@@ -100,7 +98,7 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     __graft_entry__.build()
     import lsh_sampled_sparse_simhash_b200 as mp
     from lsh_sampled_sparse_simhash_b200._binding import _CShape
-    big = _CShape(16, 32, 8, 128, 131200, 8, 75, 4, 64)  # the ragged 16 x 128k batch
+    big = _CShape(16, 32, 8, 128, 131200, 8, 75, 4, 64, 0)  # the ragged 16 x 128k batch
     n = ctypes.c_size_t()
     assert mp.library().mp_decode_workspace_bytes(ctypes.byref(big), 131073, ctypes.byref(n)) == 0
     assert n.value > 16 << 20

@@ -66,6 +66,7 @@ class Workload:
     mu_norm: float = 0.0          # >0: keys offset by a per-kv-head mean of this norm
     seed: int = 0
     description: str = ""
+    code_layout: str = "auto"     # key-code layout: "auto", "bytes" (K = 8) or "planes"
 
     @property
     def group(self) -> int:
