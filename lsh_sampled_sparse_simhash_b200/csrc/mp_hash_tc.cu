@@ -66,6 +66,8 @@ struct Params {
     int gsize;       // columns per group (multiple of 32)
     int gpad_max;    // padded width of the widest group (multiple of 32)
     int total_items; // ngroups * units * n_mt
+    uint32_t kmagic; // floor(2^32 / K) + 1: c / K = umulhi(c, kmagic) while c K < 2^32
+    uint32_t hmagic; // floor(2^32 / Hkv) + 1: batch of unit u = umulhi(u, hmagic)
 };
 
 __device__ __forceinline__ uint64_t globaltimer()
@@ -98,9 +100,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity)
     return ok != 0;
 }
 // Bounded wait for the phase of parity `parity`; false on abort or timeout.
-__device__ __noinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int *abort_flag, int32_t *status)
+// The first test is inline; only a phase that is not yet complete takes the
+// out-of-line polling loop.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, volatile int *abort_flag, int32_t *status)
 {
-    if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (!mbar_try_wait(a, parity)) {
         if (*abort_flag) return false;
@@ -111,6 +114,11 @@ __device__ __noinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int
         }
     }
     return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int *abort_flag, int32_t *status)
+{
+    if (mbar_try_wait(a, parity)) return true;
+    return mbar_wait_slow(a, parity, abort_flag, status);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y)
@@ -171,72 +179,77 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// All ones iff the fp32 value with these bits is > 0 (so +0, -0 and NaN -> 0).
-__device__ __forceinline__ uint32_t positive_mask(uint32_t bits)
-{
-    uint32_t m;
-    asm("set.gt.u32.f32 %0, %1, 0f00000000;" : "=r"(m) : "f"(__uint_as_float(bits)));
-    return m;
-}
-
-// [x > 0] as 1.0f / 0.0f on the FMA pipe: the first saturating product sends
-// every positive normal to 1 and keeps positive subnormals above 2^-23, the
-// second sends those to 1 as well; zero, negatives and NaN give 0.
+// [x > 0] as 1.0f / 0.0f in one FMA-pipe instruction: a saturating product
+// by 2^126 sends every positive normal to 1 and zero, negatives and NaN to 0.
+// Flush-to-zero makes a subnormal projection (|x| < 2^-126) count as zero.
 __device__ __forceinline__ float positive_unit(uint32_t bits)
 {
-    return __saturatef(__saturatef(__uint_as_float(bits) * 0x1p126f) * 0x1p126f);
+    float r;
+    asm("mul.rn.ftz.sat.f32 %0, %1, 0f7E800000;" : "=f"(r) : "f"(__uint_as_float(bits)));
+    return r;
 }
 
-// Byte whose bit b is [v[b] > 0], built with FMA-pipe arithmetic: the sum
-// sum_b [v_b > 0] 2^b is exact in fp32, and adding 2^23 puts it in the low
-// byte of the float's bit pattern.
-__device__ __forceinline__ uint32_t pack_positive_byte(const uint32_t *v)
+// 16-bit integer whose bit c is [v[c] > 0], built on the FMA pipe: the sum
+// sum_c [v_c > 0] 2^c is exact in fp32, and adding 2^23 puts it in the low
+// bits of the float's bit pattern.
+__device__ __forceinline__ uint32_t pack_positive16(const uint32_t *v)
 {
-    float acc = positive_unit(v[7]);
+    float acc = positive_unit(v[15]);
 #pragma unroll
-    for (int b = 6; b >= 0; b--) acc = fmaf(acc, 2.f, positive_unit(v[b]));
+    for (int c = 14; c >= 0; c--) acc = fmaf(acc, 2.f, positive_unit(v[c]));
     return __float_as_uint(acc + 8388608.f);
 }
 
-// 32-bit word whose bit c is [v[c] > 0]: two exact 16-bit FMA-pipe sums.
-__device__ __forceinline__ uint32_t pack_positive_word(const uint32_t *v)
+// 32-bit word whose bit c is [v[c] > 0].
+__device__ __forceinline__ uint32_t pack_positive32(const uint32_t *v)
 {
-    float lo = positive_unit(v[15]), hi = positive_unit(v[31]);
-#pragma unroll
-    for (int b = 14; b >= 0; b--) {
-        lo = fmaf(lo, 2.f, positive_unit(v[b]));
-        hi = fmaf(hi, 2.f, positive_unit(v[16 + b]));
-    }
-    return __byte_perm(__float_as_uint(lo + 8388608.f), __float_as_uint(hi + 8388608.f), 0x5410);
+    return __byte_perm(pack_positive16(v), pack_positive16(v + 16), 0x5410);
 }
 
 // Within each group of 4 lanes, transposes the 4x4 byte matrix whose row r
 // (lane r of the group) is the word x: afterwards lane r holds byte r of every
-// lane of its group, in lane order.
-__device__ __forceinline__ uint32_t quad_transpose(uint32_t x, int lane)
+// lane of its group, in lane order.  sel1 / sel2 are the lane's byte
+// selectors (quad_selectors).
+__device__ __forceinline__ uint32_t quad_transpose(uint32_t x, uint32_t sel1, uint32_t sel2)
 {
     uint32_t y = __shfl_xor_sync(0xffffffffu, x, 1);
-    x = __byte_perm(x, y, (lane & 1) ? 0x3715 : 0x6240);
+    x = __byte_perm(x, y, sel1);
     y = __shfl_xor_sync(0xffffffffu, x, 2);
-    return __byte_perm(x, y, (lane & 2) ? 0x3276 : 0x5410);
+    return __byte_perm(x, y, sel2);
+}
+__device__ __forceinline__ void quad_selectors(int lane, uint32_t &sel1, uint32_t &sel2)
+{
+    sel1 = (lane & 1) ? 0x3715u : 0x6240u;
+    sel2 = (lane & 2) ? 0x3276u : 0x5410u;
 }
 
 // 32x32 bit-matrix transpose across a warp: lane t holds row t; afterwards
 // lane c holds column c (bit t of the result = bit c of lane t's input).
-__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane)
+// Stage j (16, 8, 4, 2, 1) swaps j x j blocks with the lane j apart: the lane
+// keeps the bits under keep[k] and takes the rest from the partner's word
+// rotated by rot[k] (j or 32 - j), one shuffle, one funnel shift and one
+// three-input logic op per stage.  keep / rot come from transpose_consts.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, const uint32_t (&keep)[5], const uint32_t (&rot)[5])
+{
+#pragma unroll
+    for (int k = 0; k < 5; k++) {
+        const uint32_t y = __shfl_xor_sync(0xffffffffu, x, 16 >> k);
+        const uint32_t r = __funnelshift_r(y, y, rot[k]);
+        uint32_t d;
+        asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(x), "r"(r), "r"(keep[k]));  // (x & keep) | (r & ~keep)
+        x = d;
+    }
+    return x;
+}
+__device__ __forceinline__ void transpose_consts(int lane, uint32_t (&keep)[5], uint32_t (&rot)[5])
 {
     const uint32_t masks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
 #pragma unroll
     for (int k = 0; k < 5; k++) {
         const int j = 16 >> k;
-        const uint32_t m = masks[k];
-        const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
-        if (lane & j)
-            x = (x & ~m) | ((y >> j) & m);   // take the partner's high half into our low positions
-        else
-            x = (x & m) | ((y << j) & ~m);   // take the partner's low half into our high positions
+        keep[k] = (lane & j) ? ~masks[k] : masks[k];
+        rot[k] = (lane & j) ? (uint32_t)j : (uint32_t)(32 - j);
     }
-    return x;
 }
 
 struct Item {
@@ -244,17 +257,15 @@ struct Item {
     bool skip;
 };
 
-__device__ __forceinline__ Item item_of(const Params &p, int it, const int *lens_sh)
+__device__ __forceinline__ Item make_item(const Params &p, int group, int unit, int mt, const int *lens_sh)
 {
     Item r;
-    const int units = p.s.B * p.s.Hkv;
-    r.group = it / (units * p.n_mt);
-    const int rem = it % (units * p.n_mt);
-    r.unit = rem / p.n_mt;
-    r.mt = rem % p.n_mt;
+    r.group = group;
+    r.unit = unit;
+    r.mt = mt;
     int len = p.n_tokens;
     if (p.seq_lens) {
-        const int b = r.unit / p.s.Hkv;
+        const int b = (int)__umulhi((uint32_t)unit, p.hmagic);  // unit / Hkv
         len = min(len, max(b < kLensCache ? lens_sh[b] : p.seq_lens[b], 0));
     }
     r.len = len;
@@ -262,12 +273,165 @@ __device__ __forceinline__ Item item_of(const Params &p, int it, const int *lens
     return r;
 }
 
+__device__ __forceinline__ Item item_of(const Params &p, int it, const int *lens_sh)
+{
+    const int units = p.s.B * p.s.Hkv;
+    const int rem = it % (units * p.n_mt);
+    return make_item(p, it / (units * p.n_mt), rem / p.n_mt, rem % p.n_mt, lens_sh);
+}
+
+// The items of this block, blockIdx.x + k gridDim.x for k = 0, 1, ..., in
+// (group, unit, tile) form, advanced with carries instead of divisions.
+struct ItemIter {
+    int it, group, unit, mt;
+    int dg, du, dm;  // gridDim.x in the same mixed radix
+    __device__ __forceinline__ explicit ItemIter(const Params &p)
+    {
+        const int units = p.s.B * p.s.Hkv;
+        it = blockIdx.x;
+        mt = it % p.n_mt;
+        unit = (it / p.n_mt) % units;
+        group = it / (p.n_mt * units);
+        const int g = gridDim.x;
+        dm = g % p.n_mt;
+        du = (g / p.n_mt) % units;
+        dg = g / (p.n_mt * units);
+    }
+    __device__ __forceinline__ bool live(const Params &p) const { return it < p.total_items; }
+    __device__ __forceinline__ void next(const Params &p)
+    {
+        const int units = p.s.B * p.s.Hkv;
+        it += gridDim.x;
+        mt += dm;
+        int carry = 0;
+        if (mt >= p.n_mt) {
+            mt -= p.n_mt;
+            carry = 1;
+        }
+        unit += du + carry;
+        carry = 0;
+        if (unit >= units) {
+            unit -= units;
+            carry = 1;
+        }
+        group += dg + carry;
+    }
+    __device__ __forceinline__ Item item(const Params &p, const int *lens_sh) const
+    {
+        return make_item(p, group, unit, mt, lens_sh);
+    }
+};
+
 // Columns [c0, c0 + width) of a group; width is a multiple of 32.
 __device__ __forceinline__ void group_cols(const Params &p, int g, int &c0, int &width)
 {
     c0 = g * p.gsize;
     const int real = min(p.gsize, p.s.LK - c0);
     width = (real + 31) & ~31;
+}
+
+// Where an epilogue warp writes the codes of one 128-row tile.
+struct TileDst {
+    uint8_t *bytes;    // byte codes: this lane's 4-token group, table 0
+    uint32_t *planes;  // bit planes: this warp's 32-token word, table 0, bit 0
+    int t4;            // byte codes: first token of this lane's group
+    int len;
+    bool full4, valid, warp_live;
+};
+
+// Sign-packs and stores NCH 32-column chunks of one accumulator slice.
+template <bool PLANES, int NCH>
+__device__ __forceinline__ void epilogue_slice(const Params &p, const TileDst &td, uint32_t ta, uint32_t empty_bar,
+                                               int col0, int lane, uint32_t sel1, uint32_t sel2,
+                                               const uint32_t (&keep)[5], const uint32_t (&rot)[5])
+{
+    const Shape &s = p.s;
+    uint32_t v[NCH][32];
+#pragma unroll
+    for (int q = 0; q < NCH; q++) tmem_ld32(ta + 32 * q, v[q]);
+    tmem_wait_ld();
+    tc_fence_before();
+    mbar_arrive(empty_bar);  // values are in registers: free the accumulator
+#pragma unroll
+    for (int q = 0; q < NCH; q++) {
+        const int c32 = col0 + 32 * q;  // first global column of these 32
+        if (!PLANES) {
+            // 4 table bytes of this token -> 4 tokens of one table per lane
+            const uint32_t w = quad_transpose(pack_positive32(v[q]), sel1, sel2);
+            const int l = (c32 >> 3) + (lane & 3);
+            if (l < s.L) {
+                uint8_t *dst = td.bytes + (size_t)l * s.Ncap;
+                if (td.full4) {
+                    *reinterpret_cast<uint32_t *>(dst) = w;
+                } else {
+                    for (int k = 0; k < 4 && td.t4 + k < td.len; k++) dst[k] = (uint8_t)(w >> (8 * k));
+                }
+            }
+        } else {
+            // row word (bit c = column c32 + c) -> column word (bit t = token t)
+            const uint32_t rw = td.valid ? pack_positive32(v[q]) : 0u;
+            const uint32_t mine = warp_transpose32(rw, keep, rot);
+            const uint32_t c = (uint32_t)(c32 + lane);
+            if (td.warp_live && c < (uint32_t)s.LK) {
+                const uint32_t l = __umulhi(c, p.kmagic), b = c - l * (uint32_t)s.K;
+                td.planes[(size_t)l * (s.Ncap >> 5) * s.K + b] = mine;
+            }
+        }
+    }
+}
+
+// Epilogue warps (4 .. 4 + 4 * kEpiGroups - 1).  Every epilogue warp takes
+// part in every column tile: group eg owns columns [64 eg, 64 eg + 64) of the
+// tile, warp quarter q4 owns rows [32 q4, 32 q4 + 32).  The accumulator is
+// released as soon as its values are in registers, so packing and storing
+// overlap the next MMAs.  Each slice width has its own straight-line path.
+template <bool PLANES>
+__device__ __forceinline__ void epilogue(const Params &p, const int *lens_sh, uint32_t tmem_base, uint32_t bar0,
+                                         volatile int *abort_flag, int warp, int lane)
+{
+    static_assert(kSliceCols == 64, "slices of 0, 32 or 64 columns");
+    const Shape &s = p.s;
+    const int q4 = warp & 3;         // TMEM lane quarter of this warp
+    const int eg = (warp - 4) >> 2;  // column slice of every tile
+    const int row = q4 * 32 + lane;
+    const int words = s.Ncap >> 5;
+    int seq = 0;                     // column-tile sequence number
+    uint32_t sel1, sel2, keep[5], rot[5];
+    quad_selectors(lane, sel1, sel2);
+    transpose_consts(lane, keep, rot);
+    for (ItemIter iter(p); iter.live(p) && !*abort_flag; iter.next(p)) {
+        const Item im = iter.item(p, lens_sh);
+        if (im.skip) continue;
+        int c0, width;
+        group_cols(p, im.group, c0, width);
+        TileDst td;
+        td.len = im.len;
+        td.valid = im.mt * kBM + row < im.len;
+        td.warp_live = im.mt * kBM + q4 * 32 < im.len;
+        td.t4 = im.mt * kBM + q4 * 32 + (lane & ~3);
+        td.full4 = td.t4 + 3 < im.len;
+        td.bytes = static_cast<uint8_t *>(p.codes) + (size_t)im.unit * s.L * s.Ncap + td.t4;
+        td.planes = static_cast<uint32_t *>(p.codes) + (size_t)im.unit * s.L * words * s.K +
+                    ((im.mt * kBM + q4 * 32) >> 5) * s.K;
+        for (int n0 = 0; n0 < width; n0 += kAccCols, seq++) {
+            const int acc = seq & (kAccBufs - 1);
+            const int nw = min(kAccCols, width - n0);
+            const int ch = eg * kSliceCols;                  // this group's slice of the tile
+            const int sw = max(0, min(kSliceCols, nw - ch));  // 0, 32 or 64
+            const uint32_t full = bar0 + 8u * (4 + acc), empty = bar0 + 8u * (8 + acc);
+            if (!mbar_wait(full, (seq / kAccBufs) & 1, abort_flag, p.status)) return;
+            tc_fence_after();
+            const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kAccCols + ch);
+            if (sw == 64) {
+                epilogue_slice<PLANES, 2>(p, td, ta, empty, c0 + n0 + ch, lane, sel1, sel2, keep, rot);
+            } else if (sw == 32) {
+                epilogue_slice<PLANES, 1>(p, td, ta, empty, c0 + n0 + ch, lane, sel1, sel2, keep, rot);
+            } else {
+                tc_fence_before();
+                mbar_arrive(empty);
+            }
+        }
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -330,8 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int last_issued_par[kStages] = {-1, -1};
         int cur_g = -1, w_loads = 0;
         bool first_pass = true;
-        for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
-            const Item im = item_of(p, it, lens_sh);
+        for (ItemIter iter(p); iter.live(p) && !abort_flag; iter.next(p)) {
+            const Item im = iter.item(p, lens_sh);
             if (im.skip) continue;
             if (im.group != cur_g) {
                 if (cur_g >= 0 && !mbar_wait(w_empty, (w_loads - 1) & 1, &abort_flag, p.status)) break;
@@ -350,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // later tiles of this block into L2: the first pass covers 2..kPrefetchAhead
             // items ahead, every later pass the one newly kPrefetchAhead ahead
             for (int ahead = first_pass ? 2 : kPrefetchAhead; ahead <= kPrefetchAhead; ahead++) {
-                const int it2 = it + ahead * (int)gridDim.x;
+                const int it2 = iter.it + ahead * (int)gridDim.x;
                 if (it2 < p.total_items) {
                     const Item i2 = item_of(p, it2, lens_sh);
                     if (!i2.skip) {
@@ -376,8 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0, seq = 0;  // seq: column-tile sequence number; buffer seq % 4, use seq / 4
         uint32_t full_par[kStages] = {0, 0};
         int cur_g = -1, w_uses = 0;
-        for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
-            const Item im = item_of(p, it, lens_sh);
+        for (ItemIter iter(p); iter.live(p) && !abort_flag; iter.next(p)) {
+            const Item im = iter.item(p, lens_sh);
             if (im.skip) continue;
             if (im.group != cur_g) {
                 if (cur_g >= 0) mma_commit(w_empty);  // W free once the MMAs so far complete
@@ -421,79 +585,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(final_bar);
         mbar_wait(final_bar, 0, &abort_flag, p.status);
     } else if (warp >= 4) {
-        // ------------------------------------------------------ epilogue ----
-        // Every epilogue warp takes part in every column tile: group eg owns
-        // columns [64 eg, 64 eg + 64) of the tile, warp quarter q4 owns rows
-        // [32 q4, 32 q4 + 32).  The accumulator is released as soon as its
-        // values are in registers, so packing and storing overlap the next MMAs.
-        const int q4 = warp & 3;         // TMEM lane quarter of this warp
-        const int eg = (warp - 4) >> 2;  // column slice of every tile
-        const int row = q4 * 32 + lane;
-        int seq = 0;                     // column-tile sequence number
-        const int words = s.Ncap >> 5;
-        for (int it = blockIdx.x; it < p.total_items && !abort_flag; it += gridDim.x) {
-            const Item im = item_of(p, it, lens_sh);
-            if (im.skip) continue;
-            int c0, width;
-            group_cols(p, im.group, c0, width);
-            const int tok = im.mt * kBM + row;
-            const bool valid = tok < im.len;
-            const bool warp_live = im.mt * kBM + q4 * 32 < im.len;
-            bool ok = true;
-            for (int n0 = 0; n0 < width; n0 += kAccCols, seq++) {
-                const int acc = seq & (kAccBufs - 1);
-                const int nw = min(kAccCols, width - n0);
-                const int ch = eg * kSliceCols;              // this group's slice of the tile
-                const int sw = max(0, min(kSliceCols, nw - ch));  // a multiple of 32
-                if (!mbar_wait(tmem_full(acc), (seq / kAccBufs) & 1, &abort_flag, p.status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                uint32_t v[kSliceCols];
-                const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kAccCols + ch);
-#pragma unroll
-                for (int q = 0; q < kSliceCols / 32; q++)
-                    if (32 * q < sw) tmem_ld32(ta + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * q]));
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(tmem_empty(acc));  // values are in registers: free the accumulator
-#pragma unroll
-                for (int half = 0; half < kSliceCols / 32; half++) {
-                    if (32 * half >= sw) break;
-                    const uint32_t *vv = v + 32 * half;
-                    const int col0 = c0 + n0 + ch + 32 * half;  // first global column of these 32
-                    if (!s.planes) {
-                        // 4 table bytes of this token -> 4 tokens of one table per lane
-                        const uint32_t b0 = pack_positive_byte(vv), b1 = pack_positive_byte(vv + 8);
-                        const uint32_t b2 = pack_positive_byte(vv + 16), b3 = pack_positive_byte(vv + 24);
-                        const uint32_t w = quad_transpose(
-                            __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410), lane);
-                        const int l = (col0 >> 3) + (lane & 3);
-                        const int t4 = im.mt * kBM + q4 * 32 + (lane & ~3);  // first of this lane's 4 tokens
-                        if (l < s.L) {
-                            uint8_t *dst = static_cast<uint8_t *>(p.codes) + ((size_t)im.unit * s.L + l) * s.Ncap + t4;
-                            if (t4 + 3 < im.len) {
-                                *reinterpret_cast<uint32_t *>(dst) = w;
-                            } else {
-                                for (int k = 0; k < 4 && t4 + k < im.len; k++) dst[k] = (uint8_t)(w >> (8 * k));
-                            }
-                        }
-                    } else {
-                        // row word (bit c = column col0 + c) -> column word (bit t = token t)
-                        const uint32_t rw = valid ? pack_positive_word(vv) : 0u;
-                        const uint32_t mine = warp_transpose32(rw, lane);
-                        const int c = col0 + lane;
-                        if (warp_live && c < s.LK) {
-                            const int l = c / s.K, b = c - l * s.K;
-                            static_cast<uint32_t *>(p.codes)[(((size_t)im.unit * s.L + l) * words +
-                                                              ((im.mt * kBM + q4 * 32) >> 5)) * s.K + b] = mine;
-                        }
-                    }
-                }
-            }
-            if (!ok) break;
-        }
+        if (s.planes)
+            epilogue<true>(p, lens_sh, tmem_base, bar0, &abort_flag, warp, lane);
+        else
+            epilogue<false>(p, lens_sh, tmem_base, bar0, &abort_flag, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -564,6 +659,8 @@ cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint
     p.gsize = (((s.LK + p.ngroups - 1) / p.ngroups) + 31) & ~31;
     p.gpad_max = p.gsize;
     p.total_items = p.ngroups * s.B * s.Hkv * p.n_mt;
+    p.kmagic = (uint32_t)((1ull << 32) / (uint64_t)s.K) + 1u;
+    p.hmagic = (uint32_t)((1ull << 32) / (uint64_t)s.Hkv) + 1u;
     CUtensorMap mk, mw;
     if (!make_map(&mk, keys, (uint64_t)s.B * s.Hkv * s.Ncap, kBM)) return cudaErrorInvalidValue;
     if (!make_map(&mw, W, (uint64_t)s.LK, kWBox)) return cudaErrorInvalidValue;
