@@ -12,9 +12,9 @@ constexpr int kHeadDim = 128;
 constexpr int kMaxGroup = 8;
 constexpr int kScanThreads = 256;  // scan block: token groups x table splits
 constexpr int kSplitsK8 = 8;       // byte codes: tables l = ts, ts + 8, ... per split
-constexpr int kSplitsK10 = 4;      // bit planes: tables l = ts, ts + 4, ...
+constexpr int kSplitsPlanes = 8;   // bit planes: tables l = ts, ts + 8, ... per split (a warp each)
 constexpr int kChunkBytes = 512;   // scan chunk (tokens) for byte codes: 32 groups x 16 tokens
-constexpr int kChunkPlanes = 8192; // scan chunk (tokens) for bit planes: 64 groups x 128 tokens
+constexpr int kChunkPlanes = 1024; // scan chunk (tokens) for bit planes: 32 words of 32 tokens
 
 struct Shape {
     int B, Hq, Hkv, G, d, Ncap, K, L, LK, sink, window;

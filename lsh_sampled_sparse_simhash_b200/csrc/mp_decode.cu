@@ -384,15 +384,38 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
 }
 
 // ------------------------------------------------------ scan, bit planes ----
-// Bit-plane codes [unit][L][Ncap/32][K] (uint32).  An 8192-token chunk per
-// block of 256 threads: 64 token groups of 128 tokens (4 words x K planes,
-// 16 K contiguous bytes per table, so a warp streams 512 K contiguous bytes)
-// x 4 table splits.  A token mismatches table l for head h iff some
+// Bit-plane codes [unit][L][Ncap/32][K] (uint32).  A 1024-token chunk per
+// block of 256 threads: 32 token words (thread = one 32-token word, its K
+// planes of a table are 4K contiguous bytes, so a warp streams 128 K
+// contiguous bytes per table) x 8 table splits (split = warp, so the query
+// masks it reads are warp-uniform broadcasts).  Each thread keeps kPlaneTables
+// tables of loads in flight.  A token mismatches table l for head h iff some
 // plane differs from the query bit: mis = OR_b (plane_b ^ qmask_b), with
-// qmask_b = 0 or ~0 from shared memory (KB + 2 logic operations per 32
-// tokens per table and head).
+// qmask_b = 0 or ~0 from shared memory.  Small chunks keep the last, partly
+// filled wave of blocks short.
+constexpr int kPlaneTables = 4;  // tables of plane loads in flight per thread
+
+template <int KB>
+__device__ __forceinline__ void load_planes(const uint32_t *src, uint32_t (&w)[KB])
+{
+    if constexpr (KB == 8) {
+        asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+                       "=r"(w[7])
+                     : "l"(src));
+    } else {
+        static_assert(KB % 2 == 0, "plane records of whole 8-byte pairs");
+#pragma unroll
+        for (int q = 0; q < KB / 2; q++) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src) + q);
+            w[2 * q] = v.x;
+            w[2 * q + 1] = v.y;
+        }
+    }
+}
+
 template <int G, int KB>
-__global__ void __launch_bounds__(kScanThreads) scan_planes_kernel(
+__global__ void __launch_bounds__(kScanThreads, 4) scan_planes_kernel(
     Shape s, const uint32_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
     const int32_t *__restrict__ seq_lens, int max_len, int nchunk, ScanOut o)
 {
@@ -401,7 +424,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_planes_kernel(
     uint32_t *qm = dyn;
     uint32_t *part = dyn + s.L * G * QW;
     __shared__ int scratch[64];
-    constexpr int TS = kSplitsK10, TG = kScanThreads / TS;
+    constexpr int TS = kSplitsPlanes, TG = kScanThreads / TS, U = kPlaneTables;
+    static_assert(TG == 32 && TG * 32 == kChunkPlanes, "a warp per table split, a word per thread");
     const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
     const int unit = blockIdx.y, chunk = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
@@ -409,70 +433,73 @@ __global__ void __launch_bounds__(kScanThreads) scan_planes_kernel(
     const int N = clamp_len(seq_lens, b, max_len, o.status, chunk == 0 && kvh == 0 && threadIdx.x == 0);
     const int c0 = chunk * kChunkPlanes;
     if (c0 >= N) return;
-    for (int i = threadIdx.x; i < s.L * G * QW; i += blockDim.x) {
-        const int l = i / (G * QW), g = (i / QW) % G, bb = i % QW;
+    for (int i = threadIdx.x; i < s.L * G; i += blockDim.x) {
+        const int l = i / G, g = i % G;
         const unsigned code = qcodes[((size_t)b * s.Hq + kvh * G + g) * s.L + l];
-        qm[i] = bb < KB ? 0u - ((code >> bb) & 1u) : 0u;
+        uint4 *dst = reinterpret_cast<uint4 *>(qm + (size_t)i * QW);
+#pragma unroll
+        for (int q = 0; q < QW / 4; q++) {
+            uint32_t m[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++) m[e] = 4 * q + e < KB ? 0u - ((code >> (4 * q + e)) & 1u) : 0u;
+            dst[q] = make_uint4(m[0], m[1], m[2], m[3]);
+        }
     }
     __syncthreads();
 
-    const int t0 = c0 + tg * 128;
+    const int t0 = c0 + tg * 32;
     const int words = s.Ncap >> 5;
-    uint32_t s1[G][4], s2[G][4];
+    uint32_t s1[G][1], s2[G][1];
 #pragma unroll
-    for (int g = 0; g < G; g++)
-#pragma unroll
-        for (int j = 0; j < 4; j++) s1[g][j] = s2[g][j] = 0u;
+    for (int g = 0; g < G; g++) s1[g][0] = s2[g][0] = 0u;
 
     if (t0 < N) {
-        // this thread's 4 words x KB planes of one table: 16 * KB contiguous bytes
         const uint32_t *base = codes + ((size_t)unit * s.L * words + (t0 >> 5)) * KB;
+        const size_t lstride = (size_t)words * KB;
 #pragma unroll 1
-        for (int l = ts; l < s.L; l += TS) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(base + (size_t)l * words * KB);
-            uint32_t pw[4 * KB];  // pw[j * KB + b] = plane b of token word j
+        for (int l0 = ts; l0 < s.L; l0 += TS * U) {
+            uint32_t pw[U][KB];
 #pragma unroll
-            for (int q = 0; q < KB; q++) {
-                const uint4 v = ld_cached_16(src + q);
-                pw[4 * q] = v.x;
-                pw[4 * q + 1] = v.y;
-                pw[4 * q + 2] = v.z;
-                pw[4 * q + 3] = v.w;
+            for (int u = 0; u < U; u++) {
+                const int l = l0 + u * TS;
+                if (l < s.L) {
+                    load_planes<KB>(base + (size_t)l * lstride, pw[u]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < KB; q++) pw[u][q] = 0u;
+                }
             }
 #pragma unroll
-            for (int g = 0; g < G; g++) {
-                const uint4 *m4 = reinterpret_cast<const uint4 *>(qm + (l * G + g) * QW);
-                uint32_t msk[QW];
+            for (int u = 0; u < U; u++) {
+                const int l = l0 + u * TS;
+                if (l >= s.L) break;
 #pragma unroll
-                for (int q = 0; q < QW / 4; q++) {
-                    const uint4 mq = m4[q];
-                    msk[4 * q] = mq.x;
-                    msk[4 * q + 1] = mq.y;
-                    msk[4 * q + 2] = mq.z;
-                    msk[4 * q + 3] = mq.w;
-                }
-                uint32_t mis[4] = {0u, 0u, 0u, 0u};
+                for (int g = 0; g < G; g++) {
+                    const uint4 *m4 = reinterpret_cast<const uint4 *>(qm + (l * G + g) * QW);
+                    uint32_t msk[QW];
 #pragma unroll
-                for (int bb = 0; bb < KB; bb++) {
+                    for (int q = 0; q < QW / 4; q++) {
+                        const uint4 mq = m4[q];
+                        msk[4 * q] = mq.x;
+                        msk[4 * q + 1] = mq.y;
+                        msk[4 * q + 2] = mq.z;
+                        msk[4 * q + 3] = mq.w;
+                    }
+                    uint32_t mis = 0u;
 #pragma unroll
-                    for (int j = 0; j < 4; j++) mis[j] |= pw[j * KB + bb] ^ msk[bb];
-                }
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    s2[g][j] |= s1[g][j] & ~mis[j];
-                    s1[g][j] |= ~mis[j];
+                    for (int bb = 0; bb < KB; bb++) mis |= pw[u][bb] ^ msk[bb];
+                    s2[g][0] |= s1[g][0] & ~mis;
+                    s1[g][0] |= ~mis;
                 }
             }
         }
     }
-    combine_splits<G, 4, TS>(s1, s2, part, ts, tg);
+    combine_splits<G, 1, TS>(s1, s2, part, ts, tg);
     if (ts != 0) {
 #pragma unroll
-        for (int g = 0; g < G; g++)
-#pragma unroll
-            for (int j = 0; j < 4; j++) s2[g][j] = 0u;
+        for (int g = 0; g < G; g++) s2[g][0] = 0u;
     }
-    compact_and_store<G, 4, 32>(s, unit, chunk, nchunk, kChunkPlanes, t0, N, s.sink, min(N - s.window, N), s2,
+    compact_and_store<G, 1, 32>(s, unit, chunk, nchunk, kChunkPlanes, t0, N, s.sink, min(N - s.window, N), s2,
                                 ts == 0, o, scratch);
 }
 
@@ -647,37 +674,34 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     const uint16_t *vbase = a.vc + (size_t)unit * s.Ncap * kHeadDim;
     const int ntiles = (nrows + kAttRows - 1) / kAttRows;
 
-    // Candidate entries of a tile for this thread's rows (tid/16 + 8 i); the
-    // list is read one tile ahead of the copies so its latency is hidden.
+    // Candidate entries: threads 0..63 each read the entry of one row of a tile
+    // two tiles ahead (its load overlaps the current tile's arithmetic) and
+    // leave it in a 2-slot shared ring; the copy issue reads its 8 rows there.
+    static_assert(kAttStages == 2, "entry ring sized for one tile of copies in flight");
+    __shared__ uint32_t ents[2][kAttRows];
     int jc = 0;  // chunk of this thread's next candidate (rows are visited in increasing order)
-    auto fetch = [&](int tile, uint32_t (&ent)[8]) {
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const int e = tile * kAttRows + (tid >> 4) + 8 * i;
-            if (e >= nrows) {
-                ent[i] = 0xFFFFFFFFu;
-            } else if (dsplit) {
-                ent[i] = (uint32_t)(e < n_sink ? e : win0 + (e - n_sink));
-            } else {
-                const int r = e0 + e;
-                while (cpre[jc + 1] <= r) jc++;
-                ent[i] = lists[(size_t)jc * a.chunk_tokens + (r - cpre[jc])];
-            }
-        }
+    auto fetch1 = [&](int tile) -> uint32_t {
+        const int e = tile * kAttRows + tid;
+        if (e >= nrows) return 0xFFFFFFFFu;
+        if (dsplit) return (uint32_t)(e < n_sink ? e : win0 + (e - n_sink));
+        const int r = e0 + e;
+        while (cpre[jc + 1] <= r) jc++;
+        return lists[(size_t)jc * a.chunk_tokens + (r - cpre[jc])];
     };
-    auto issue = [&](const uint32_t (&ent)[8], int stage) {
+    auto issue = [&](int tile, int stage) {
         uint8_t *ks_ = smem + stage * kStageBytes;
         uint8_t *vs_ = ks_ + kAttRows * kRowStride;
         const int col = tid & 15;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
             const int r = (tid >> 4) + 8 * i;
-            const bool ok = ent[i] != 0xFFFFFFFFu;
-            const int tok = ok ? (int)(ent[i] & 0xFFFFFFu) : 0;
+            const uint32_t ent = ents[tile & 1][r];
+            const bool ok = ent != 0xFFFFFFFFu;
+            const int tok = ok ? (int)(ent & 0xFFFFFFu) : 0;
             const size_t off = (size_t)tok * kHeadDim + col * 8;
             cp_async_16(ks_ + r * kRowStride + col * 16, kbase + off, ok ? 16 : 0);
             cp_async_16(vs_ + r * kRowStride + col * 16, vbase + off, ok ? 16 : 0);
-            if (col == 0) meta[stage][r] = ok ? (dsplit ? dmeta : (ent[i] >> 24)) : 0u;
+            if (col == 0) meta[stage][r] = ok ? (dsplit ? dmeta : (ent >> 24)) : 0u;
         }
     };
 
@@ -688,30 +712,22 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
 #pragma unroll
         for (int e = 0; e < 4; e++) acc[mt][e] = 0.f;
 
-    uint32_t nxt[8];
-#pragma unroll
-    for (int st = 0; st < kAttStages - 1; st++) {
-        if (st < ntiles) {
-            fetch(st, nxt);
-            issue(nxt, st);
-        }
-        cp_async_commit();
+    if (tid < kAttRows) {
+        if (ntiles > 0) ents[0][tid] = fetch1(0);
+        if (ntiles > 1) ents[1][tid] = fetch1(1);
     }
-    if (kAttStages - 1 < ntiles) fetch(kAttStages - 1, nxt);
-    __syncthreads();  // qinv
+    __syncthreads();  // entries of tiles 0 and 1, qinv
+    if (ntiles > 0) issue(0, 0);
+    cp_async_commit();
     const int h0 = 2 * tq, h1 = 2 * tq + 1;
     const float qi0 = h0 < G ? qinv[h0] : 0.f, qi1 = h1 < G ? qinv[h1] : 0.f;
     const float inv_scale = 1.f / a.scale;
 
     for (int tile = 0; tile < ntiles; tile++) {
-        {
-            const int nt = tile + kAttStages - 1;
-            if (nt < ntiles) {
-                issue(nxt, nt % kAttStages);
-                if (nt + 1 < ntiles) fetch(nt + 1, nxt);
-            }
-            cp_async_commit();
-        }
+        if (tile + 1 < ntiles) issue(tile + 1, (tile + 1) % kAttStages);
+        cp_async_commit();
+        const bool fetcher = tid < kAttRows && tile + 2 < ntiles;
+        const uint32_t pend = fetcher ? fetch1(tile + 2) : 0u;
         cp_async_wait<kAttStages - 1>();
         __syncthreads();
         const int stage = tile % kAttStages;
@@ -819,6 +835,7 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
                 mma_bf16_16816(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3], a0, a1, a2, a3, bl0, bl1);
             }
         }
+        if (fetcher) ents[tile & 1][tid] = pend;  // slot of tile + 2, read after the barrier
         __syncthreads();  // stage may be refilled next iteration
     }
     cp_async_wait<0>();
@@ -985,8 +1002,9 @@ struct Workspace {
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // How attention blocks cover the scan chunks.  Many chunks: each block takes
-// `span` consecutive chunks (about 600 blocks in all, so that the per-block
-// set-up is amortised and the merge sees few partials).  Few, large chunks:
+// `span` consecutive chunks (about 1200 blocks in all: a few waves of 3 blocks
+// per SM, so that uneven candidate counts even out, while the per-block set-up
+// stays amortised and the merge sees few partials).  Few, large chunks:
 // each chunk's list is shared by `subs` blocks.  Fixed counts, so the
 // workspace size does not depend on the device.
 struct SplitPlan {
@@ -999,8 +1017,8 @@ static SplitPlan split_plan(const Shape &s, int max_len)
     const int C = chunk_tokens(s);
     p.nchunk = (max_len + C - 1) / C;
     const int blocks = p.nchunk * s.B * s.Hkv;
-    if (blocks >= 600) {
-        p.span = std::min(kMaxSpan, blocks / 600);
+    if (blocks >= 1200) {
+        p.span = std::min(kMaxSpan, blocks / 1200);
         p.subs = 1;
     } else {
         // few chunks: split each chunk's list so that about 1200 blocks run,
@@ -1076,7 +1094,8 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     ScanOut so{ws.cand, ws.cnt, dbg ? dbg->member_out : nullptr, ws.status, 1u};
     if (nchunk > 0) {
         dim3 grid(nchunk, units);
-        const size_t part = (size_t)2 * G * 4 * kScanThreads * sizeof(uint32_t);
+        const size_t part = (size_t)2 * G * 4 * kScanThreads * sizeof(uint32_t);       // byte scan: 4 words
+        const size_t part1 = (size_t)2 * G * 1 * kScanThreads * sizeof(uint32_t);      // plane scan: 1 word
         if (!s.planes) {
             const size_t sm = (size_t)((s.L * G + 3) & ~3) * sizeof(uint32_t) + part;
             if ((e = ensure_smem(reinterpret_cast<const void *>(scan_k8_kernel<G>), (int)sm)) != cudaSuccess) return e;
@@ -1084,14 +1103,14 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
                            static_cast<const uint8_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
                            nchunk, so);
         } else if (s.K == 8) {
-            const size_t sm = (size_t)s.L * G * 8 * sizeof(uint32_t) + part;
+            const size_t sm = (size_t)s.L * G * 8 * sizeof(uint32_t) + part1;
             if ((e = ensure_smem(reinterpret_cast<const void *>(scan_planes_kernel<G, 8>), (int)sm)) != cudaSuccess)
                 return e;
             e = launch_pdl(scan_planes_kernel<G, 8>, grid, dim3(kScanThreads), sm, st, s,
                            static_cast<const uint32_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
                            nchunk, so);
         } else {
-            const size_t sm = (size_t)s.L * G * 12 * sizeof(uint32_t) + part;
+            const size_t sm = (size_t)s.L * G * 12 * sizeof(uint32_t) + part1;
             if ((e = ensure_smem(reinterpret_cast<const void *>(scan_planes_kernel<G, 10>), (int)sm)) != cudaSuccess)
                 return e;
             e = launch_pdl(scan_planes_kernel<G, 10>, grid, dim3(kScanThreads), sm, st, s,
