@@ -78,4 +78,67 @@ __device__ __forceinline__ void mma_bf16_16816(float &d0, float &d1, float &d2, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// ------------------------------------------------ mbarriers, bulk copies ----
+// Every spin on an mbarrier in this library gives up after kWaitLimitNs of
+// %globaltimer, records MP_ERR_CUDA in the status word and lets the kernel
+// wind down instead of hanging.
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t a)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for phase `parity` of mbarrier `a`: false once kWaitLimitNs
+// has passed.  The first test is inline, the polling loop out of line.
+static __device__ __noinline__ bool mbar_wait_bounded_slow(uint32_t a, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(a, parity))
+        if (globaltimer() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t a, uint32_t parity)
+{
+    return mbar_try_wait(a, parity) || mbar_wait_bounded_slow(a, parity);
+}
+
+// One contiguous global -> shared copy on the async (TMA) engine, completing
+// `bytes` of the transaction count of mbarrier `bar`.  dst, src and bytes are
+// multiples of 16.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before its
+// later async-proxy ones (a buffer that was read is about to be refilled).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 }  // namespace mp

@@ -384,123 +384,330 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
 }
 
 // ------------------------------------------------------ scan, bit planes ----
-// Bit-plane codes [unit][L][Ncap/32][K] (uint32).  A 1024-token chunk per
-// block of 256 threads: 32 token words (thread = one 32-token word, its K
-// planes of a table are 4K contiguous bytes, so a warp streams 128 K
-// contiguous bytes per table) x 8 table splits (split = warp, so the query
-// masks it reads are warp-uniform broadcasts).  Each thread keeps kPlaneTables
-// tables of loads in flight.  A token mismatches table l for head h iff some
-// plane differs from the query bit: mis = OR_b (plane_b ^ qmask_b), with
-// qmask_b = 0 or ~0 from shared memory.  Small chunks keep the last, partly
-// filled wave of blocks short.
-constexpr int kPlaneTables = 4;  // tables of plane loads in flight per thread
+// Bit-plane codes [unit][L][Ncap/32][K] (uint32).  Work item = one 1024-token
+// chunk of one (sequence, kv head) unit; a persistent block walks a
+// contiguous share of the live items.  Warp 8 is the producer: one 3-D TMA
+// copy (two for K = 10) brings a stage of 8 consecutive tables x the chunk's
+// 32 words x K planes into a ring of kScanStages(K) stages, tables past L
+// zero-filled.  Warps 0..7 consume: warp ts takes table 8 j + ts of stage j,
+// lane t the 32-token word t.  A token mismatches table l for head h iff some
+// plane differs from the query bit: mis = OR_b (plane_b ^ qmask_b), qmask_b =
+// 0 or ~0 from shared memory; two bit-sliced counters (seen >= 1, >= 2) per
+// head.  After an item's stages the consumers leave their counters in a
+// partial buffer (double-buffered by item parity) and go straight on; the
+// producer warp, once it has issued the next item's stages, folds the eight
+// splits and compacts the candidates, one item behind the consumers.
+constexpr int kScanConsumers = 8;  // consumer warps = table splits = tables per stage
 
 template <int KB>
-__device__ __forceinline__ void load_planes(const uint32_t *src, uint32_t (&w)[KB])
+struct PlaneStage {
+    static constexpr int kBoxWords = KB == 8 ? 256 : 160;  // inner TMA box (<= 256 elements)
+    static constexpr int kBoxes = 32 * KB / kBoxWords;      // 1 or 2 copies per stage
+    static constexpr int kBytes = kScanConsumers * 32 * KB * 4;
+    static constexpr int kStages = KB == 8 ? 5 : 4;         // ring depth (stages of 8 tables)
+};
+
+// Live items of the plane scan: (sequence b, kv head, chunk) with chunk below
+// ceil(N_b / chunk), in unit-major order.  Advanced with carries.
+struct LiveCursor {
+    int b, kvh, chunk, nch, N;
+    __device__ __forceinline__ void load_seq(const int32_t *seq_lens, int max_len)
+    {
+        N = min(max(seq_lens[b], 0), max_len);
+        nch = (N + kChunkPlanes - 1) / kChunkPlanes;
+    }
+    __device__ __forceinline__ void next(const Shape &s, const int32_t *seq_lens, int max_len)
+    {
+        if (++chunk < nch) return;
+        chunk = 0;
+        if (++kvh < s.Hkv) return;
+        kvh = 0;
+        do {
+            if (++b >= s.B) return;
+            load_seq(seq_lens, max_len);
+        } while (nch == 0);
+    }
+    __device__ __forceinline__ int unit(const Shape &s) const { return b * s.Hkv + kvh; }
+};
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y, int z)
 {
-    if constexpr (KB == 8) {
-        asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
-                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
-                       "=r"(w[7])
-                     : "l"(src));
-    } else {
-        static_assert(KB % 2 == 0, "plane records of whole 8-byte pairs");
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// Named barriers of the plane scan (0 is __syncthreads):
+//   1  the 8 consumer warps (query-mask rewrite)
+//   2  consumers arrive, producer waits: an item's split partials are written
+//   3  producer arrives, consumers wait: the previous item's partials are read
+__device__ __forceinline__ void consumer_barrier() { asm volatile("bar.sync 1, %0;" ::"n"(kScanThreads) : "memory"); }
+__device__ __forceinline__ void bar_sync_all(int id) { asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kScanThreads + 32) : "memory"); }
+__device__ __forceinline__ void bar_arrive_all(int id) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kScanThreads + 32) : "memory"); }
+
+// Candidate list of one item by one warp (lane = 32-token word at t0):
+// hm[g] bit i = token t0 + i is in S_g.  Entries keep token order.
+template <int G>
+__device__ __forceinline__ void compact_warp(const Shape &s, int unit, int chunk, int nchunk, int t0, int N, int lo,
+                                             int hi, uint32_t (&hm)[G], const ScanOut &o, int lane)
+{
+    const uint32_t v = range_mask(t0, lo, hi, 32);
+    uint32_t any = 0u;
 #pragma unroll
-        for (int q = 0; q < KB / 2; q++) {
-            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src) + q);
-            w[2 * q] = v.x;
-            w[2 * q + 1] = v.y;
-        }
+    for (int g = 0; g < G; g++) {
+        hm[g] &= v;
+        any |= hm[g];
+    }
+    const int mine = __popc(any);
+    int incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += t;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int off = incl - mine;
+    uint32_t *dst = o.cand + ((size_t)unit * nchunk + chunk) * kChunkPlanes;
+    while (any) {
+        const int bit = __ffs(any) - 1;
+        any &= any - 1u;
+        uint32_t heads = 0u;
+#pragma unroll
+        for (int g = 0; g < G; g++) heads |= ((hm[g] >> bit) & 1u) << g;
+        dst[off++] = (uint32_t)(t0 + bit) | (heads << 24);
+    }
+    int32_t *cnt = o.cnt + ((size_t)unit * nchunk + chunk) * 16;
+    if (lane == 0) cnt[0] = total;
+#pragma unroll
+    for (int g = 0; g < G; g++) {
+        int c = __popc(hm[g]);
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) c += __shfl_xor_sync(0xffffffffu, c, d);
+        if (lane == 0) cnt[1 + g] = c;
+    }
+    if (o.member_out) {
+        const int b = unit / s.Hkv, kvh = unit % s.Hkv;
+        for (int i = 0; i < 32 && t0 + i < N; i++)
+#pragma unroll
+            for (int g = 0; g < G; g++)
+                o.member_out[((size_t)b * s.Hq + kvh * G + g) * s.Ncap + t0 + i] = (hm[g] >> i) & 1u;
     }
 }
 
 template <int G, int KB>
-__global__ void __launch_bounds__(kScanThreads, 4) scan_planes_kernel(
-    Shape s, const uint32_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
+__global__ void __launch_bounds__(kScanThreads + 32) scan_planes_kernel(
+    const __grid_constant__ CUtensorMap tmap, Shape s, const uint16_t *__restrict__ qcodes,
     const int32_t *__restrict__ seq_lens, int max_len, int nchunk, ScanOut o)
 {
+    using St = PlaneStage<KB>;
     constexpr int QW = (KB + 3) & ~3;  // query masks per (table, head), padded to whole uint4s
-    extern __shared__ uint32_t dyn[];  // qm [L][G][QW] (qmask of the KB planes), then split partials
-    uint32_t *qm = dyn;
-    uint32_t *part = dyn + s.L * G * QW;
-    __shared__ int scratch[64];
-    constexpr int TS = kSplitsPlanes, TG = kScanThreads / TS, U = kPlaneTables;
-    static_assert(TG == 32 && TG * 32 == kChunkPlanes, "a warp per table split, a word per thread");
-    const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
-    const int unit = blockIdx.y, chunk = blockIdx.x;
-    const int b = unit / s.Hkv, kvh = unit % s.Hkv;
+    constexpr int S = St::kStages, NC = kScanConsumers;
+    static_assert(NC * 32 == kScanThreads && 32 * 32 == kChunkPlanes, "8 consumer warps, a word per lane");
+    extern __shared__ __align__(1024) uint8_t dyn_raw[];
+    uint32_t *ring = reinterpret_cast<uint32_t *>(dyn_raw);  // [S][box][8 tables][kBoxWords]
+    uint32_t *qm = ring + S * St::kBytes / 4;                // [L][G][QW]
+    uint32_t *part = qm + s.L * G * QW;                      // [2 parities][G][2][kScanThreads]
+    __shared__ __align__(8) uint64_t full[S], empty[S];
+    __shared__ int range_sh[4];  // first item (b, kvh, chunk), item count
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     grid_dependency_wait();
-    const int N = clamp_len(seq_lens, b, max_len, o.status, chunk == 0 && kvh == 0 && threadIdx.x == 0);
-    const int c0 = chunk * kChunkPlanes;
-    if (c0 >= N) return;
-    for (int i = threadIdx.x; i < s.L * G; i += blockDim.x) {
-        const int l = i / G, g = i % G;
-        const unsigned code = qcodes[((size_t)b * s.Hq + kvh * G + g) * s.L + l];
-        uint4 *dst = reinterpret_cast<uint4 *>(qm + (size_t)i * QW);
-#pragma unroll
-        for (int q = 0; q < QW / 4; q++) {
-            uint32_t m[4];
-#pragma unroll
-            for (int e = 0; e < 4; e++) m[e] = 4 * q + e < KB ? 0u - ((code >> (4 * q + e)) & 1u) : 0u;
-            dst[q] = make_uint4(m[0], m[1], m[2], m[3]);
+
+    if (threadIdx.x == 0) {
+        // this block's contiguous share of the live items
+        long long total = 0;
+        for (int b = 0; b < s.B; b++) {
+            const int n = clamp_len(seq_lens, b, max_len, o.status, blockIdx.x == 0);
+            total += (long long)s.Hkv * ((n + kChunkPlanes - 1) / kChunkPlanes);
         }
+        long long x = total * blockIdx.x / gridDim.x;
+        const long long x1 = total * (blockIdx.x + 1) / gridDim.x;
+        range_sh[3] = (int)(x1 - x);
+        range_sh[0] = range_sh[1] = range_sh[2] = 0;
+        for (int b = 0; b < s.B && x1 > x; b++) {
+            const int n = min(max(seq_lens[b], 0), max_len);
+            const long long nch = (n + kChunkPlanes - 1) / kChunkPlanes, items = nch * s.Hkv;
+            if (x < items) {
+                range_sh[0] = b;
+                range_sh[1] = (int)(x / nch);
+                range_sh[2] = (int)(x % nch);
+                break;
+            }
+            x -= items;
+        }
+        for (int i = 0; i < S; i++) {
+            mbar_init(smem_u32(&full[i]), 1);
+            mbar_init(smem_u32(&empty[i]), NC);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+    const int count = range_sh[3];
+    if (count <= 0) return;
+    LiveCursor cur;
+    cur.b = range_sh[0];
+    cur.kvh = range_sh[1];
+    cur.chunk = range_sh[2];
+    cur.load_seq(seq_lens, max_len);
+    const int nst = (s.L + NC - 1) / NC;  // stages per item
 
-    const int t0 = c0 + tg * 32;
-    const int words = s.Ncap >> 5;
-    uint32_t s1[G][1], s2[G][1];
+    if (warp == NC) {
+        // ------------------------------------------- producer + compactor ----
+        // Issue item it's stages, then fold and compact item it - 1 (whose
+        // stages were all issued earlier, so the consumers can finish it).
+        int e = 0;
+        bool ok = true;
+        LiveCursor pc = cur;
+        for (int it = 0; it <= count; it++) {
+            if (it < count) {
+                if (lane == 0 && ok) {
+                    const int x0 = pc.chunk * 32 * KB, z = pc.unit(s);
+                    for (int j = 0; j < nst; j++, e++) {
+                        const int st = e % S;
+                        if (e >= S && !mbar_wait_bounded(smem_u32(&empty[st]), (uint32_t)(e / S - 1) & 1u)) {
+                            set_status(o.status, MP_ERR_CUDA);
+                            ok = false;
+                            break;
+                        }
+                        mbar_expect_tx(smem_u32(&full[st]), St::kBytes);
 #pragma unroll
-    for (int g = 0; g < G; g++) s1[g][0] = s2[g][0] = 0u;
-
-    if (t0 < N) {
-        const uint32_t *base = codes + ((size_t)unit * s.L * words + (t0 >> 5)) * KB;
-        const size_t lstride = (size_t)words * KB;
+                        for (int bx = 0; bx < St::kBoxes; bx++)
+                            tma_load_3d(smem_u32(ring) + (uint32_t)(st * St::kBytes + bx * NC * St::kBoxWords * 4),
+                                        &tmap, smem_u32(&full[st]), x0 + bx * St::kBoxWords, NC * j, z);
+                    }
+                }
+                __syncwarp();
+                pc.next(s, seq_lens, max_len);
+            }
+            if (it >= 1) {
+                const int ci = it - 1;
+                bar_sync_all(2);  // the consumers' partials of item ci are in buffer ci & 1
+                const uint32_t *pp = part + (ci & 1) * (G * 2 * kScanThreads);
+                uint32_t s1[G], s2[G];
+#pragma unroll
+                for (int g = 0; g < G; g++) s1[g] = s2[g] = 0u;
 #pragma unroll 1
-        for (int l0 = ts; l0 < s.L; l0 += TS * U) {
-            uint32_t pw[U][KB];
+                for (int t = 0; t < NC; t++) {
 #pragma unroll
-            for (int u = 0; u < U; u++) {
-                const int l = l0 + u * TS;
-                if (l < s.L) {
-                    load_planes<KB>(base + (size_t)l * lstride, pw[u]);
-                } else {
+                    for (int g = 0; g < G; g++) {
+                        const uint32_t a1 = pp[(g * 2 + 0) * kScanThreads + t * 32 + lane];
+                        const uint32_t a2 = pp[(g * 2 + 1) * kScanThreads + t * 32 + lane];
+                        s2[g] |= a2 | (s1[g] & a1);
+                        s1[g] |= a1;
+                    }
+                }
+                if (ci + 1 < count) bar_arrive_all(3);  // item ci is read: the consumers may post item ci + 1
+                // tokens eligible for S: [sink, N - window) and below N
+                compact_warp<G>(s, cur.unit(s), cur.chunk, nchunk, cur.chunk * kChunkPlanes + lane * 32, cur.N,
+                                s.sink, min(cur.N - s.window, cur.N), s2, o, lane);
+                cur.next(s, seq_lens, max_len);
+            }
+        }
+        // every copy issued lands before the block exits (the last use of each stage)
+        if (lane == 0)
+            for (int st = 0; st < S && st < e; st++) {
+                const int last = st + ((e - 1 - st) / S) * S;
+                mbar_wait_bounded(smem_u32(&full[st]), (uint32_t)(last / S) & 1u);
+            }
+        return;
+    }
+
+    // ------------------------------------------------------- consumers ----
+    const int ts = warp;
+    const int box = (lane * KB) / St::kBoxWords, in_box = lane * KB - box * St::kBoxWords;
+    const int lane_off = box * NC * St::kBoxWords + ts * St::kBoxWords + in_box;  // words into a stage
+    int e = 0, qm_unit = -1;
+    bool dead = false;  // a copy never landed: stop waiting, keep the barriers in step
+    for (int it = 0; it < count; it++, cur.next(s, seq_lens, max_len)) {
+        const int unit = cur.unit(s);
+        if (unit != qm_unit) {  // uniform over the consumers
+            if (qm_unit >= 0) consumer_barrier();  // every consumer is done with the old masks
+            for (int i = threadIdx.x; i < s.L * G; i += kScanThreads) {
+                const int l = i / G, g = i % G;
+                const unsigned code = qcodes[((size_t)cur.b * s.Hq + cur.kvh * G + g) * s.L + l];
+                uint4 *dst = reinterpret_cast<uint4 *>(qm + (size_t)i * QW);
 #pragma unroll
-                    for (int q = 0; q < KB; q++) pw[u][q] = 0u;
+                for (int q = 0; q < QW / 4; q++) {
+                    uint32_t m[4];
+#pragma unroll
+                    for (int x = 0; x < 4; x++) m[x] = 4 * q + x < KB ? 0u - ((code >> (4 * q + x)) & 1u) : 0u;
+                    dst[q] = make_uint4(m[0], m[1], m[2], m[3]);
                 }
             }
+            consumer_barrier();
+            qm_unit = unit;
+        }
+        uint32_t s1[G], s2[G];
 #pragma unroll
-            for (int u = 0; u < U; u++) {
-                const int l = l0 + u * TS;
-                if (l >= s.L) break;
+        for (int g = 0; g < G; g++) s1[g] = s2[g] = 0u;
+        for (int j = 0; j < nst; j++, e++) {
+            const int st = e % S;
+            if (!dead) {
+                // every lane waits (bounded); the warp goes on only if all saw the stage land
+                const bool landed = mbar_wait_bounded(smem_u32(&full[st]), (uint32_t)(e / S) & 1u);
+                if (!__all_sync(0xffffffffu, landed)) {
+                    if (lane == 0) set_status(o.status, MP_ERR_CUDA);
+                    dead = true;
+                }
+            }
+            const int l = ts + NC * j;
+            const bool live = !dead && l < s.L;
+            uint32_t pw[KB];
+            if (live) {
+                const uint32_t *src = ring + st * (St::kBytes / 4) + lane_off;
+                if constexpr (KB % 4 == 0) {
+#pragma unroll
+                    for (int q = 0; q < KB / 4; q++) {
+                        const uint4 v = reinterpret_cast<const uint4 *>(src)[q];
+                        pw[4 * q] = v.x;
+                        pw[4 * q + 1] = v.y;
+                        pw[4 * q + 2] = v.z;
+                        pw[4 * q + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < KB / 2; q++) {
+                        const uint2 v = reinterpret_cast<const uint2 *>(src)[q];
+                        pw[2 * q] = v.x;
+                        pw[2 * q + 1] = v.y;
+                    }
+                }
 #pragma unroll
                 for (int g = 0; g < G; g++) {
                     const uint4 *m4 = reinterpret_cast<const uint4 *>(qm + (l * G + g) * QW);
-                    uint32_t msk[QW];
+                    uint32_t mis = 0u;
 #pragma unroll
                     for (int q = 0; q < QW / 4; q++) {
                         const uint4 mq = m4[q];
-                        msk[4 * q] = mq.x;
-                        msk[4 * q + 1] = mq.y;
-                        msk[4 * q + 2] = mq.z;
-                        msk[4 * q + 3] = mq.w;
-                    }
-                    uint32_t mis = 0u;
+                        const uint32_t mm[4] = {mq.x, mq.y, mq.z, mq.w};
 #pragma unroll
-                    for (int bb = 0; bb < KB; bb++) mis |= pw[u][bb] ^ msk[bb];
-                    s2[g][0] |= s1[g][0] & ~mis;
-                    s1[g][0] |= ~mis;
+                        for (int x = 0; x < 4; x++)
+                            if (4 * q + x < KB) mis |= pw[4 * q + x] ^ mm[x];
+                    }
+                    s2[g] |= s1[g] & ~mis;
+                    s1[g] |= ~mis;
                 }
             }
+            // Release the stage only once every lane has used (so received) its
+            // words; the proxy fence orders those reads before the TMA refill.
+            __syncwarp();
+            if (lane == 0 && !dead) {
+                fence_proxy_async_smem();
+                mbar_arrive(smem_u32(&empty[st]));
+            }
         }
-    }
-    combine_splits<G, 1, TS>(s1, s2, part, ts, tg);
-    if (ts != 0) {
+        // this item's split partials -> buffer it & 1, once the producer has read
+        // item it - 1 (so each barrier generation sees exactly one item)
+        if (it >= 1) bar_sync_all(3);
+        uint32_t *pp = part + (it & 1) * (G * 2 * kScanThreads);
 #pragma unroll
-        for (int g = 0; g < G; g++) s2[g][0] = 0u;
+        for (int g = 0; g < G; g++) {
+            pp[(g * 2 + 0) * kScanThreads + threadIdx.x] = s1[g];
+            pp[(g * 2 + 1) * kScanThreads + threadIdx.x] = s2[g];
+        }
+        bar_arrive_all(2);
     }
-    compact_and_store<G, 1, 32>(s, unit, chunk, nchunk, kChunkPlanes, t0, N, s.sink, min(N - s.window, N), s2,
-                                ts == 0, o, scratch);
 }
 
 // ---------------------------------------------------------------- attend ----
@@ -1073,6 +1280,43 @@ static LogU make_logu(const Shape &s)
     return u;
 }
 
+// Persistent plane scan: as many blocks as fit on the device at once (at
+// most one per possible item); each walks its share of the live items.
+template <int G, int KB>
+static cudaError_t launch_scan_planes(const Shape &s, const uint32_t *codes, const Workspace &ws,
+                                      const int32_t *seq_lens, int max_len, int nchunk, const ScanOut &so,
+                                      cudaStream_t st)
+{
+    using Stg = PlaneStage<KB>;
+    const size_t sm = (size_t)Stg::kStages * Stg::kBytes + (size_t)s.L * G * ((KB + 3) & ~3) * sizeof(uint32_t) +
+                      (size_t)2 * G * 2 * kScanThreads * sizeof(uint32_t);
+    const void *fn = reinterpret_cast<const void *>(scan_planes_kernel<G, KB>);
+    cudaError_t e = ensure_smem(fn, (int)sm);
+    if (e != cudaSuccess) return e;
+    // codes as a 3-D uint32 tensor: (word x plane) within a table, table, unit
+    const int words = s.Ncap >> 5;
+    const uint64_t dims[3] = {(uint64_t)words * KB, (uint64_t)s.L, (uint64_t)s.B * s.Hkv};
+    const uint64_t strides[2] = {(uint64_t)words * KB * 4, (uint64_t)s.L * words * KB * 4};
+    const uint32_t box[3] = {(uint32_t)Stg::kBoxWords, (uint32_t)kScanConsumers, 1};
+    CUtensorMap tmap;
+    if (!encode_tensor_map(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, codes, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    }
+    int per_sm = 1;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kScanThreads + 32, sm)) != cudaSuccess)
+        return e;
+    const long long items = (long long)nchunk * s.B * s.Hkv;
+    const int grid = (int)std::max(1LL, std::min(items, (long long)std::max(per_sm, 1) * sms));
+    return launch_pdl(scan_planes_kernel<G, KB>, dim3(grid), dim3(kScanThreads + 32), sm, st, tmap, s,
+                      (const uint16_t *)ws.qcodes, seq_lens, max_len, nchunk, so);
+}
+
 template <int G>
 static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint16_t *W, const void *codes,
                                    const uint16_t *kc, const uint16_t *vc, const int32_t *seq_lens,
@@ -1095,7 +1339,6 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     if (nchunk > 0) {
         dim3 grid(nchunk, units);
         const size_t part = (size_t)2 * G * 4 * kScanThreads * sizeof(uint32_t);       // byte scan: 4 words
-        const size_t part1 = (size_t)2 * G * 1 * kScanThreads * sizeof(uint32_t);      // plane scan: 1 word
         if (!s.planes) {
             const size_t sm = (size_t)((s.L * G + 3) & ~3) * sizeof(uint32_t) + part;
             if ((e = ensure_smem(reinterpret_cast<const void *>(scan_k8_kernel<G>), (int)sm)) != cudaSuccess) return e;
@@ -1103,19 +1346,11 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
                            static_cast<const uint8_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
                            nchunk, so);
         } else if (s.K == 8) {
-            const size_t sm = (size_t)s.L * G * 8 * sizeof(uint32_t) + part1;
-            if ((e = ensure_smem(reinterpret_cast<const void *>(scan_planes_kernel<G, 8>), (int)sm)) != cudaSuccess)
-                return e;
-            e = launch_pdl(scan_planes_kernel<G, 8>, grid, dim3(kScanThreads), sm, st, s,
-                           static_cast<const uint32_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
-                           nchunk, so);
+            e = launch_scan_planes<G, 8>(s, static_cast<const uint32_t *>(codes), ws, seq_lens, max_len, nchunk,
+                                         so, st);
         } else {
-            const size_t sm = (size_t)s.L * G * 12 * sizeof(uint32_t) + part1;
-            if ((e = ensure_smem(reinterpret_cast<const void *>(scan_planes_kernel<G, 10>), (int)sm)) != cudaSuccess)
-                return e;
-            e = launch_pdl(scan_planes_kernel<G, 10>, grid, dim3(kScanThreads), sm, st, s,
-                           static_cast<const uint32_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
-                           nchunk, so);
+            e = launch_scan_planes<G, 10>(s, static_cast<const uint32_t *>(codes), ws, seq_lens, max_len, nchunk,
+                                          so, st);
         }
         if (e != cudaSuccess) return e;
     }

@@ -53,7 +53,6 @@ constexpr int kHalfBytes = kBM * 128;        // one 64-element (128 B) K half of
 constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KB
 constexpr int kMaxGroupCols = 640;
 constexpr int kWBox = 32;                    // W rows per TMA box
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 struct Params {
     Shape s;
@@ -70,35 +69,6 @@ struct Params {
     uint32_t hmagic; // floor(2^32 / Hkv) + 1: batch of unit u = umulhi(u, hmagic)
 };
 
-__device__ __forceinline__ uint64_t globaltimer()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t a)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t a, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
 // Bounded wait for the phase of parity `parity`; false on abort or timeout.
 // The first test is inline; only a phase that is not yet complete takes the
 // out-of-line polling loop.
@@ -600,6 +570,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host ----
+// 2-D bf16 row-major [rows][128] view, box = 64 elements x box_rows, 128B swizzle.
+static bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows)
+{
+    const uint64_t dims[2] = {128, rows};
+    const uint64_t strides[1] = {256};
+    const uint32_t box[2] = {64, box_rows};
+    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+static int num_sms()
+{
+    int dev = 0, n = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+}  // namespace tc
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -619,29 +609,22 @@ static EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 2-D bf16 row-major [rows][128] view, box = 64 elements x box_rows, 128B swizzle.
-static bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint32_t box_rows)
+bool encode_tensor_map(CUtensorMap *m, CUtensorMapDataType type, int rank, const void *ptr, const uint64_t *dims,
+                       const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swizzle)
 {
     EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {128, rows};
-    cuuint64_t strides[1] = {256};
-    cuuint32_t box[2] = {64, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (!fn || rank < 1 || rank > 5) return false;
+    cuuint64_t d[5], st[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; i++) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) st[i] = strides[i];
+    }
+    return fn(m, type, (cuuint32_t)rank, const_cast<void *>(ptr), d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-static int num_sms()
-{
-    int dev = 0, n = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
-}
-
-}  // namespace tc
 
 cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint16_t *W, const int32_t *seq_lens,
                                 int n_tokens, void *codes, int32_t *status, cudaStream_t st)

@@ -2,6 +2,8 @@
 // argument validation).  All launch asynchronously on `st`.
 #pragma once
 
+#include <cuda.h>
+
 #include <initializer_list>
 
 #include "mp_common.cuh"
@@ -26,6 +28,12 @@ cudaError_t launch_decode(const Shape &s, const uint16_t *q, const uint16_t *W, 
                           float *out, float *lse, int32_t *n_sampled, void *workspace,
                           const mp_decode_debug *dbg, cudaStream_t st);
 size_t decode_workspace_bytes(const Shape &s, int max_len);
+
+// A tiled TMA descriptor for a rank-`rank` tensor (dims and box innermost
+// first, byte strides of dims 1..rank-1), no interleave, zero fill out of
+// bounds.  False if the driver rejects it.
+bool encode_tensor_map(CUtensorMap *m, CUtensorMapDataType type, int rank, const void *ptr, const uint64_t *dims,
+                       const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swizzle);
 
 // Raises the dynamic shared-memory limit of `func` on the current device once.
 cudaError_t ensure_smem(const void *func, int bytes);
