@@ -275,8 +275,9 @@ class Bench:
         return statistics.mean(times), h2d, d2h
 
 
-def traffic_record(kernel, workload):
-    """dram bytes per launch from a committed ncu summary, if its kernel source is unchanged."""
+def traffic_record(kernel, workload, layout):
+    """DRAM bytes (read + write) per call from a committed ncu capture, keyed
+    kernel@workload:layout, if the kernel source it was taken on is unchanged."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -284,7 +285,7 @@ def traffic_record(kernel, workload):
         recs = json.load(open(path))
     except ValueError:
         return None
-    rec = recs.get(f"{kernel}@{workload}")
+    rec = recs.get(f"{kernel}@{workload}:{layout}")
     if not rec:
         return None
     import hashlib
@@ -455,12 +456,12 @@ def main():
             hash_bound, hash_peak, hash_unit = "alu", 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12, "TFLOP/s"
         hash_roof = dict(kernel="mp_hash_keys", bound=hash_bound, achieved=hash_flops / (hash_ms / 1e3) / 1e12,
                          peak=hash_peak, unit=hash_unit, algorithmic=hash_flops, units=f"{hash_rows} key rows",
-                         traffic=traffic_record("hash_keys", w.name))
+                         traffic=traffic_record("hash_keys", w.name, config_of(w)["code_layout"]))
         hash_roof["frac"] = hash_roof["achieved"] / hash_roof["peak"]
         dec_roof = dict(kernel="mp_decode_attend", bound="hbm", achieved=dec_bytes / (decode_ms / 1e3) / 1e9,
                         peak=peaks["hbm"], unit="GB/s", algorithmic=dec_bytes,
                         units=f"{int(lens_after.sum())} tokens x {w.n_kv_heads} kv heads; {union} union rows",
-                        traffic=traffic_record("decode", w.name))
+                        traffic=traffic_record("decode", w.name, config_of(w)["code_layout"]))
         dec_roof["frac"] = dec_roof["achieved"] / dec_roof["peak"]
         dominant = hash_roof if hash_ms >= decode_ms else dec_roof
         roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
