@@ -48,6 +48,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--code-layout", default=None, choices=["auto", "bytes", "planes"],
                    help="key-code layout (default: the workload's, i.e. bytes for K=8, planes for K=10)")
+    p.add_argument("--decode-path", default="auto", choices=["auto", "split", "fused"],
+                   help="decode kernels: auto, split (scan then attention) or fused (one kernel; bit planes)")
     return p.parse_args()
 
 
@@ -135,7 +137,7 @@ class ClockSampler:
 # --------------------------------------------------------- our arm ----
 
 class Bench:
-    def __init__(self, w, device):
+    def __init__(self, w, device, path="auto"):
         import torch
         import lsh_sampled_sparse_simhash_b200 as mp
         from workloads import make_inputs
@@ -165,7 +167,10 @@ class Bench:
         self.ns = torch.empty((B, Hq), dtype=torch.int32, device=device)
         self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
         self.tokens = step_tokens(inp["seq_lens"] + 1)
-        self.launches_per_step = 7  # hash 1, append 2, decode 4 (qhash, scan, attend, merge)
+        self.path = {"auto": mp.MP_PATH_AUTO, "split": mp.MP_PATH_SPLIT, "fused": mp.MP_PATH_FUSED}[path]
+        fused = self.path == mp.MP_PATH_FUSED
+        # hash 1, append 2, decode: qhash + (scan, attention | fused) + merge
+        self.launches_per_step = 3 + (3 if fused else 4)
 
     def hash(self):
         self.mp.hash_keys(self.shape, self.K, self.W, self.prefill, self.codes, seq_lens=self.lens0)
@@ -175,7 +180,7 @@ class Bench:
 
     def decode(self):
         self.mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
-                              self.out, self.lse, self.ns, self.ws)
+                              self.out, self.lse, self.ns, self.ws, path=self.path)
 
     def step(self):
         self.lens.copy_(self.lens0, non_blocking=True)
@@ -190,7 +195,7 @@ class Bench:
         self.step()
         mem = torch.zeros((w.batch, w.n_q_heads, w.capacity), dtype=torch.uint8, device=self.q.device)
         self.mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
-                              self.out, self.lse, self.ns, self.ws, member_out=mem)
+                              self.out, self.lse, self.ns, self.ws, member_out=mem, path=self.path)
         torch.cuda.synchronize()
         m = mem.view(w.batch, w.n_kv_heads, w.group, w.capacity).amax(dim=2)
         return int(m.sum().item()), float(self.ns.float().mean().item())
@@ -404,7 +409,7 @@ def main():
     import __graft_entry__
     __graft_entry__.build()
     w = workload_for_rank(args.workload, rank, args.code_layout)
-    bench = Bench(w, device)
+    bench = Bench(w, device, args.decode_path)
     union, mean_ns = bench.union_rows()
 
     def barrier():
@@ -470,7 +475,7 @@ def main():
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype="bf16-in/fp32-acc", data="synthetic",
-                    config=config_of(w), roofline=roofline,
+                    config=dict(config_of(w), decode_path=args.decode_path), roofline=roofline,
                     breakdown=dict(hash_ms=hash_ms, append_ms=append_ms, decode_ms=decode_ms,
                                    hash_roofline=hash_roof, decode_roofline=dec_roof,
                                    decode_only_tokens_per_s=bench.tokens / (decode_ms / 1e3),

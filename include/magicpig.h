@@ -128,11 +128,18 @@ int mp_append_token(const mp_shape *shape, const void *k_new, const void *v_new,
                     void *k_cache, void *v_cache, void *codes, int32_t *seq_lens,
                     int32_t *status, void *stream);
 
-/* Test hooks of mp_decode_attend (all nullable). */
+/* Kernel paths of mp_decode_attend (mp_decode_debug.path). */
+#define MP_PATH_AUTO 0     /* the faster path for the shape: currently always MP_PATH_SPLIT */
+#define MP_PATH_SPLIT 1    /* collision scan, then sampled attention (two kernels) */
+#define MP_PATH_FUSED 2    /* one kernel scans and attends (bit-plane codes, G <= 4);
+                              MP_ERR_SHAPE where it does not apply */
+
+/* Test hooks of mp_decode_attend (all nullable / zero). */
 typedef struct mp_decode_debug {
     const uint16_t *qcodes_in; /* [B][Hq][L]: use these query codes instead of hashing q */
     uint16_t *qcodes_out;      /* [B][Hq][L]: copy of the query codes used */
     uint8_t *member_out;       /* [B][Hq][Ncap]: 1 iff token i is in S_h (i < N_b) */
+    int32_t path;              /* MP_PATH_*: which kernel path to take */
 } mp_decode_debug;
 
 /* Workspace bytes that mp_decode_attend needs for sequences up to max_len. */

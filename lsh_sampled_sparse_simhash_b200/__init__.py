@@ -32,6 +32,9 @@ from ._binding import (  # noqa: F401
     MP_CODES_AUTO,
     MP_CODES_BYTES,
     MP_CODES_PLANES,
+    MP_PATH_AUTO,
+    MP_PATH_SPLIT,
+    MP_PATH_FUSED,
 )
 
 __all__ = [

@@ -20,6 +20,9 @@ MP_ERR_TOO_LARGE = -7
 MP_CODES_AUTO = 0
 MP_CODES_BYTES = 1
 MP_CODES_PLANES = 2
+MP_PATH_AUTO = 0
+MP_PATH_SPLIT = 1
+MP_PATH_FUSED = 2
 
 
 class MagicPIGError(RuntimeError):
@@ -36,7 +39,7 @@ class _CShape(ctypes.Structure):
 
 class _CDebug(ctypes.Structure):
     _fields_ = [("qcodes_in", ctypes.c_void_p), ("qcodes_out", ctypes.c_void_p),
-                ("member_out", ctypes.c_void_p)]
+                ("member_out", ctypes.c_void_p), ("path", ctypes.c_int32)]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -160,10 +163,10 @@ def append_token(shape: Shape, k_new, v_new, W, k_cache, v_cache, codes, seq_len
 
 
 def decode_attend(shape: Shape, q, W, codes, k_cache, v_cache, seq_lens, max_len: int, out, lse, n_sampled,
-                  workspace, qcodes_in=None, qcodes_out=None, member_out=None, stream=None):
+                  workspace, qcodes_in=None, qcodes_out=None, member_out=None, path: int = 0, stream=None):
     dbg = None
-    if qcodes_in is not None or qcodes_out is not None or member_out is not None:
-        dbg = ctypes.byref(_CDebug(_ptr(qcodes_in), _ptr(qcodes_out), _ptr(member_out)))
+    if qcodes_in is not None or qcodes_out is not None or member_out is not None or path:
+        dbg = ctypes.byref(_CDebug(_ptr(qcodes_in), _ptr(qcodes_out), _ptr(member_out), int(path)))
     nbytes = workspace.numel() * workspace.element_size()
     _check(library().mp_decode_attend(ctypes.byref(shape.c()), _ptr(q), _ptr(W), _ptr(codes), _ptr(k_cache),
                                       _ptr(v_cache), _ptr(seq_lens), int(max_len), _ptr(out), _ptr(lse),

@@ -137,6 +137,13 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uin
                  : "memory");
 }
 
+// Pulls `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
+// without waiting for it: the later real load then finds it there.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Orders this thread's earlier generic-proxy shared-memory accesses before its
 // later async-proxy ones (a buffer that was read is about to be refilled).
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }

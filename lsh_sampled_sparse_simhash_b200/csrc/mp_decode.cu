@@ -443,6 +443,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
 //   1  the 8 consumer warps (query-mask rewrite)
 //   2  consumers arrive, producer waits: an item's split partials are written
 //   3  producer arrives, consumers wait: the previous item's partials are read
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
 __device__ __forceinline__ void consumer_barrier() { asm volatile("bar.sync 1, %0;" ::"n"(kScanThreads) : "memory"); }
 __device__ __forceinline__ void bar_sync_all(int id) { asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kScanThreads + 32) : "memory"); }
 __device__ __forceinline__ void bar_arrive_all(int id) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kScanThreads + 32) : "memory"); }
@@ -797,6 +804,240 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 //   P.V     O^T (128 dims x 8 heads) += V^T . P^T on the tensor cores: P is
 //           split into bf16 hi + lo parts (error ~2^-17 relative), transposed
 //           into B fragments with movmatrix, V^T comes from ldmatrix.trans.
+// Attention state of one warp of a 4-warp (128-thread) group: the warp owns
+// 16 rows of every 64-row tile.  Lane (g, t) holds rows g, g + 8 for heads
+// 2t, 2t + 1, the B fragments of Q^T, those heads' online-softmax state (m, l)
+// and O^T fragments acc[mt] (dims 16 mt + g and 16 mt + g + 8).
+template <int G>
+struct AttnWarp {
+    uint32_t qb[8][2];
+    float qi0, qi1;  // 1/|q| of heads 2t, 2t + 1
+    float m0, m1, l0, l1;
+    float acc[8][4];
+};
+
+// Loads the Q^T fragments of the G heads starting at query vector vec0 and
+// clears the state (the 1/|q| values come later, from attn_qinv's shared array).
+template <int G>
+__device__ __forceinline__ void attn_begin(AttnWarp<G> &w, const uint16_t *q, size_t vec0, int lane)
+{
+    const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < 8; ks++) {
+        if (gq < G) {
+            const uint32_t *qp = reinterpret_cast<const uint32_t *>(q + (vec0 + gq) * kHeadDim);
+            w.qb[ks][0] = qp[(ks * 16 + 2 * tq) >> 1];
+            w.qb[ks][1] = qp[(ks * 16 + 2 * tq + 8) >> 1];
+        } else {
+            w.qb[ks][0] = w.qb[ks][1] = 0u;
+        }
+    }
+    w.m0 = w.m1 = -INFINITY;
+    w.l0 = w.l1 = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < 8; mt++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) w.acc[mt][e] = 0.f;
+}
+
+// 1/|q_h| of the G heads into qinv[G] (warp `warp` of a 4-warp group).
+template <int G>
+__device__ __forceinline__ void attn_qinv(const uint16_t *q, size_t vec0, int warp, int lane, float *qinv)
+{
+    for (int h = warp; h < G; h += 4) {
+        const uint2 qv = reinterpret_cast<const uint2 *>(q + (vec0 + h) * kHeadDim)[lane];
+        float x0 = bf16_lo(qv.x), x1 = bf16_hi(qv.x), x2 = bf16_lo(qv.y), x3 = bf16_hi(qv.y);
+        float qq = x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) qq += __shfl_xor_sync(0xffffffffu, qq, o);
+        if (lane == 0) qinv[h] = qq > 0.f ? rsqrtf(qq) : 0.f;
+    }
+}
+
+template <int G>
+__device__ __forceinline__ void attn_set_qinv(AttnWarp<G> &w, const float *qinv, int lane)
+{
+    const int h0 = 2 * (lane & 3), h1 = h0 + 1;
+    w.qi0 = h0 < G ? qinv[h0] : 0.f;
+    w.qi1 = h1 < G ? qinv[h1] : 0.f;
+}
+
+// One 64-row tile for this warp: its 16 K rows at ks_ and V rows at vs_
+// (kRowStride apart, the tile's rows 16 warp ..), meta[64] = the rows' head
+// masks (| 0x100 for the exact set); ucos / uval are this warp's [16 G] scratch.
+template <int G>
+__device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, const uint8_t *vs_,
+                                          const uint32_t *meta, int warp, int lane, float scale, const LogU &lu,
+                                          float *ucos, float *uval)
+{
+    const int gq = lane >> 2, tq = lane & 3;
+    const int h0 = 2 * tq, h1 = 2 * tq + 1;
+    // ---- S^T = K rows . Q^T and |k|^2 ----
+    // The A fragments of K double as B fragments of K^T, so two more MMAs
+    // per k-step give the 16x16 Gram matrix K K^T, whose diagonal is |k|^2.
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    float na, nb;
+    {
+        float g0[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStride + (lane >> 4) * 16;
+#pragma unroll
+        for (int kst = 0; kst < 8; kst++) {
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(a0, a1, a2, a3, arow + kst * 32);
+            mma_bf16_16816(c[0], c[1], c[2], c[3], a0, a1, a2, a3, w.qb[kst][0], w.qb[kst][1]);
+            mma_bf16_16816(g0[0], g0[1], g0[2], g0[3], a0, a1, a2, a3, a0, a2);  // columns: rows 0-7
+            mma_bf16_16816(g1[0], g1[1], g1[2], g1[3], a0, a1, a2, a3, a1, a3);  // columns: rows 8-15
+        }
+        // |k_r|^2 = Gram[r][r]: row gq sits in lane 4 gq + gq/2 (g0, element gq & 1),
+        // row gq + 8 in the same lane (g1, element 2 + (gq & 1)).
+        const int src = 4 * gq + (gq >> 1);
+        const float d0 = (gq & 1) ? g0[1] : g0[0];
+        const float d1 = (gq & 1) ? g1[3] : g1[2];
+        na = __shfl_sync(0xffffffffu, d0, src);
+        nb = __shfl_sync(0xffffffffu, d1, src);
+    }
+
+    // ---- log-weights: s (exact) or s - log u (sampled), -inf if absent ----
+    const uint32_t mg = meta[warp * 16 + gq], mg8 = meta[warp * 16 + gq + 8];
+    float tv[4];
+    bool need[4];
+    int pos[4];
+    {
+        const uint32_t mrow[4] = {mg, mg, mg8, mg8};
+        const int hh[4] = {h0, h1, h0, h1};
+        const float kinv_g = na > 0.f ? rsqrtf(na) : 0.f, kinv_g8 = nb > 0.f ? rsqrtf(nb) : 0.f;
+        const float kin[4] = {kinv_g, kinv_g, kinv_g8, kinv_g8};
+        const float qin[4] = {w.qi0, w.qi1, w.qi0, w.qi1};
+        int base = 0;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const bool mem = hh[j] < G && ((mrow[j] >> hh[j]) & 1u);
+            need[j] = mem && !(mrow[j] & 0x100u);
+            tv[j] = mem ? c[j] * scale : -INFINITY;
+            const uint32_t bal = __ballot_sync(0xffffffffu, need[j]);
+            pos[j] = base + __popc(bal & ((1u << lane) - 1u));
+            if (need[j]) ucos[pos[j]] = c[j] * qin[j] * kin[j];
+            base += __popc(bal);
+        }
+        __syncwarp();
+        for (int i = lane; i < base; i += 32) uval[i] = log_sampling_prob(ucos[i], lu);
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+            if (need[j]) tv[j] -= uval[pos[j]];
+    }
+
+    // ---- online softmax over this warp's rows (lanes with equal t share heads) ----
+    float mt0 = fmaxf(tv[0], tv[2]), mt1 = fmaxf(tv[1], tv[3]);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, o));
+        mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, o));
+    }
+    const float mn0 = fmaxf(w.m0, mt0), mn1 = fmaxf(w.m1, mt1);
+    const float al0 = mn0 == -INFINITY ? 1.f : expf(w.m0 - mn0);
+    const float al1 = mn1 == -INFINITY ? 1.f : expf(w.m1 - mn1);
+    float p[4];
+    p[0] = tv[0] == -INFINITY ? 0.f : expf(tv[0] - mn0);
+    p[1] = tv[1] == -INFINITY ? 0.f : expf(tv[1] - mn1);
+    p[2] = tv[2] == -INFINITY ? 0.f : expf(tv[2] - mn0);
+    p[3] = tv[3] == -INFINITY ? 0.f : expf(tv[3] - mn1);
+    w.l0 = w.l0 * al0 + p[0] + p[2];
+    w.l1 = w.l1 * al1 + p[1] + p[3];
+    w.m0 = mn0;
+    w.m1 = mn1;
+#pragma unroll
+    for (int mt = 0; mt < 8; mt++) {
+        w.acc[mt][0] *= al0;
+        w.acc[mt][1] *= al1;
+        w.acc[mt][2] *= al0;
+        w.acc[mt][3] *= al1;
+    }
+
+    // ---- O^T += V^T . P^T (P split into bf16 hi + lo) ----
+    const uint32_t hi_g = pack_bf16x2(p[0], p[1]), hi_g8 = pack_bf16x2(p[2], p[3]);
+    const uint32_t lo_g = pack_bf16x2(p[0] - bf16_lo(hi_g), p[1] - bf16_hi(hi_g));
+    const uint32_t lo_g8 = pack_bf16x2(p[2] - bf16_lo(hi_g8), p[3] - bf16_hi(hi_g8));
+    const uint32_t bh0 = movmatrix_trans(hi_g), bh1 = movmatrix_trans(hi_g8);
+    const uint32_t bl0 = movmatrix_trans(lo_g), bl1 = movmatrix_trans(lo_g8);
+    {
+        const int mrow = lane >> 3;
+        const uint8_t *vrow =
+            vs_ + (warp * 16 + (mrow >> 1) * 8 + (lane & 7)) * kRowStride + (mrow & 1) * 16;
+#pragma unroll
+        for (int mt = 0; mt < 8; mt++) {
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(a0, a1, a2, a3, vrow + mt * 32);
+            mma_bf16_16816(w.acc[mt][0], w.acc[mt][1], w.acc[mt][2], w.acc[mt][3], a0, a1, a2, a3, bh0, bh1);
+            mma_bf16_16816(w.acc[mt][0], w.acc[mt][1], w.acc[mt][2], w.acc[mt][3], a0, a1, a2, a3, bl0, bl1);
+        }
+    }
+}
+
+// Folds the 4 warps' states of a group (red: shared [4 G 128 + 8 G] floats,
+// free for the group; bar(): the group's barrier) and writes one partial per
+// head: m, l at pm/pl[(vec0 + g) nsplit + split], acc at pacc[..][128].  The
+// caller keeps `red` untouched by other warps until bar() is passed again.
+template <int G, typename Bar>
+__device__ __forceinline__ void attn_store_partial(AttnWarp<G> &w, float *red, int warp, int lane, int tid, Bar bar,
+                                                   size_t vec0, size_t nsplit, int split, float *pm, float *pl,
+                                                   float *pacc)
+{
+    const int gq = lane >> 2, tq = lane & 3;
+    const int h0 = 2 * tq, h1 = 2 * tq + 1;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        w.l0 += __shfl_xor_sync(0xffffffffu, w.l0, o);
+        w.l1 += __shfl_xor_sync(0xffffffffu, w.l1, o);
+    }
+    float *redm = red + 4 * G * kHeadDim;
+    float *redl = redm + 4 * G;
+#pragma unroll
+    for (int mt = 0; mt < 8; mt++) {
+        if (h0 < G) {
+            red[(warp * G + h0) * kHeadDim + mt * 16 + gq] = w.acc[mt][0];
+            red[(warp * G + h0) * kHeadDim + mt * 16 + gq + 8] = w.acc[mt][2];
+        }
+        if (h1 < G) {
+            red[(warp * G + h1) * kHeadDim + mt * 16 + gq] = w.acc[mt][1];
+            red[(warp * G + h1) * kHeadDim + mt * 16 + gq + 8] = w.acc[mt][3];
+        }
+    }
+    if (gq == 0) {
+        if (h0 < G) {
+            redm[warp * G + h0] = w.m0;
+            redl[warp * G + h0] = w.l0;
+        }
+        if (h1 < G) {
+            redm[warp * G + h1] = w.m1;
+            redl[warp * G + h1] = w.l1;
+        }
+    }
+    bar();
+    const int dim = tid;  // 128 threads = head_dim
+    for (int g = 0; g < G; g++) {
+        float M = -INFINITY;
+        for (int w = 0; w < 4; w++) M = fmaxf(M, redm[w * G + g]);
+        float Ls = 0.f, A = 0.f;
+        if (M != -INFINITY) {
+            for (int w = 0; w < 4; w++) {
+                const float mw = redm[w * G + g];
+                if (mw == -INFINITY) continue;
+                const float f = expf(mw - M);
+                Ls += redl[w * G + g] * f;
+                A += red[(w * G + g) * kHeadDim + dim] * f;
+            }
+        }
+        const size_t bh = vec0 + g;
+        const size_t pidx = bh * nsplit + split;
+        pacc[pidx * kHeadDim + dim] = A;
+        if (dim == 0) {
+            pm[pidx] = M;
+            pl[pidx] = Ls;
+        }
+    }
+}
+
 template <int G>
 __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
 {
@@ -855,27 +1096,9 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     const uint32_t dmeta = ((1u << G) - 1u) | 0x100u;
 
     const size_t vec0 = (size_t)b * s.Hq + (size_t)kvh * G;
-    const int gq = lane >> 2, tq = lane & 3;
-    // B fragments of Q^T (k = head_dim, n = head), 8 k-steps x 2 registers.
-    uint32_t qb[8][2];
-#pragma unroll
-    for (int ks = 0; ks < 8; ks++) {
-        if (gq < G) {
-            const uint32_t *qp = reinterpret_cast<const uint32_t *>(a.q + (vec0 + gq) * kHeadDim);
-            qb[ks][0] = qp[(ks * 16 + 2 * tq) >> 1];
-            qb[ks][1] = qp[(ks * 16 + 2 * tq + 8) >> 1];
-        } else {
-            qb[ks][0] = qb[ks][1] = 0u;
-        }
-    }
-    for (int h = warp; h < G; h += 4) {
-        const uint2 qv = reinterpret_cast<const uint2 *>(a.q + (vec0 + h) * kHeadDim)[lane];
-        float x0 = bf16_lo(qv.x), x1 = bf16_hi(qv.x), x2 = bf16_lo(qv.y), x3 = bf16_hi(qv.y);
-        float qq = x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) qq += __shfl_xor_sync(0xffffffffu, qq, o);
-        if (lane == 0) qinv[h] = qq > 0.f ? rsqrtf(qq) : 0.f;
-    }
+    AttnWarp<G> w;
+    attn_begin<G>(w, a.q, vec0, lane);
+    attn_qinv<G>(a.q, vec0, warp, lane, qinv);
 
     const uint16_t *kbase = a.kc + (size_t)unit * s.Ncap * kHeadDim;
     const uint16_t *vbase = a.vc + (size_t)unit * s.Ncap * kHeadDim;
@@ -895,6 +1118,7 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
         while (cpre[jc + 1] <= r) jc++;
         return lists[(size_t)jc * a.chunk_tokens + (r - cpre[jc])];
     };
+
     auto issue = [&](int tile, int stage) {
         uint8_t *ks_ = smem + stage * kStageBytes;
         uint8_t *vs_ = ks_ + kAttRows * kRowStride;
@@ -912,13 +1136,6 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
         }
     };
 
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2t, 2t+1 of this lane
-    float acc[8][4];
-#pragma unroll
-    for (int mt = 0; mt < 8; mt++)
-#pragma unroll
-        for (int e = 0; e < 4; e++) acc[mt][e] = 0.f;
-
     if (tid < kAttRows) {
         if (ntiles > 0) ents[0][tid] = fetch1(0);
         if (ntiles > 1) ents[1][tid] = fetch1(1);
@@ -926,9 +1143,7 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     __syncthreads();  // entries of tiles 0 and 1, qinv
     if (ntiles > 0) issue(0, 0);
     cp_async_commit();
-    const int h0 = 2 * tq, h1 = 2 * tq + 1;
-    const float qi0 = h0 < G ? qinv[h0] : 0.f, qi1 = h1 < G ? qinv[h1] : 0.f;
-    const float inv_scale = 1.f / a.scale;
+    attn_set_qinv<G>(w, qinv, lane);
 
     for (int tile = 0; tile < ntiles; tile++) {
         if (tile + 1 < ntiles) issue(tile + 1, (tile + 1) % kAttStages);
@@ -941,107 +1156,7 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
         const uint8_t *ks_ = smem + stage * kStageBytes;
         const uint8_t *vs_ = ks_ + kAttRows * kRowStride;
 
-        // ---- S^T = K rows . Q^T and |k|^2 ----
-        // The A fragments of K double as B fragments of K^T, so two more MMAs
-        // per k-step give the 16x16 Gram matrix K K^T, whose diagonal is |k|^2.
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        float na, nb;
-        {
-            float g0[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f};
-            const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStride + (lane >> 4) * 16;
-#pragma unroll
-            for (int kst = 0; kst < 8; kst++) {
-                uint32_t a0, a1, a2, a3;
-                ldmatrix_x4(a0, a1, a2, a3, arow + kst * 32);
-                mma_bf16_16816(c[0], c[1], c[2], c[3], a0, a1, a2, a3, qb[kst][0], qb[kst][1]);
-                mma_bf16_16816(g0[0], g0[1], g0[2], g0[3], a0, a1, a2, a3, a0, a2);  // columns: rows 0-7
-                mma_bf16_16816(g1[0], g1[1], g1[2], g1[3], a0, a1, a2, a3, a1, a3);  // columns: rows 8-15
-            }
-            // |k_r|^2 = Gram[r][r]: row gq sits in lane 4 gq + gq/2 (g0, element gq & 1),
-            // row gq + 8 in the same lane (g1, element 2 + (gq & 1)).
-            const int src = 4 * gq + (gq >> 1);
-            const float d0 = (gq & 1) ? g0[1] : g0[0];
-            const float d1 = (gq & 1) ? g1[3] : g1[2];
-            na = __shfl_sync(0xffffffffu, d0, src);
-            nb = __shfl_sync(0xffffffffu, d1, src);
-        }
-
-        // ---- log-weights: s (exact) or s - log u (sampled), -inf if absent ----
-        const uint32_t mg = meta[stage][warp * 16 + gq], mg8 = meta[stage][warp * 16 + gq + 8];
-        float tv[4];
-        bool need[4];
-        int pos[4];
-        {
-            const uint32_t mrow[4] = {mg, mg, mg8, mg8};
-            const int hh[4] = {h0, h1, h0, h1};
-            const float kinv_g = na > 0.f ? rsqrtf(na) : 0.f, kinv_g8 = nb > 0.f ? rsqrtf(nb) : 0.f;
-            const float kin[4] = {kinv_g, kinv_g, kinv_g8, kinv_g8};
-            const float qin[4] = {qi0, qi1, qi0, qi1};
-            int base = 0;
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const bool mem = hh[j] < G && ((mrow[j] >> hh[j]) & 1u);
-                need[j] = mem && !(mrow[j] & 0x100u);
-                tv[j] = mem ? c[j] * a.scale : -INFINITY;
-                const uint32_t bal = __ballot_sync(0xffffffffu, need[j]);
-                pos[j] = base + __popc(bal & ((1u << lane) - 1u));
-                if (need[j]) ucos[warp][pos[j]] = c[j] * qin[j] * kin[j];
-                base += __popc(bal);
-            }
-            __syncwarp();
-            for (int i = lane; i < base; i += 32) uval[warp][i] = log_sampling_prob(ucos[warp][i], a.lu);
-            __syncwarp();
-#pragma unroll
-            for (int j = 0; j < 4; j++)
-                if (need[j]) tv[j] -= uval[warp][pos[j]];
-        }
-        (void)inv_scale;
-
-        // ---- online softmax over this warp's rows (lanes with equal t share heads) ----
-        float mt0 = fmaxf(tv[0], tv[2]), mt1 = fmaxf(tv[1], tv[3]);
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-            mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, o));
-            mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, o));
-        }
-        const float mn0 = fmaxf(m0, mt0), mn1 = fmaxf(m1, mt1);
-        const float al0 = mn0 == -INFINITY ? 1.f : expf(m0 - mn0);
-        const float al1 = mn1 == -INFINITY ? 1.f : expf(m1 - mn1);
-        float p[4];
-        p[0] = tv[0] == -INFINITY ? 0.f : expf(tv[0] - mn0);
-        p[1] = tv[1] == -INFINITY ? 0.f : expf(tv[1] - mn1);
-        p[2] = tv[2] == -INFINITY ? 0.f : expf(tv[2] - mn0);
-        p[3] = tv[3] == -INFINITY ? 0.f : expf(tv[3] - mn1);
-        l0 = l0 * al0 + p[0] + p[2];
-        l1 = l1 * al1 + p[1] + p[3];
-        m0 = mn0;
-        m1 = mn1;
-#pragma unroll
-        for (int mt = 0; mt < 8; mt++) {
-            acc[mt][0] *= al0;
-            acc[mt][1] *= al1;
-            acc[mt][2] *= al0;
-            acc[mt][3] *= al1;
-        }
-
-        // ---- O^T += V^T . P^T (P split into bf16 hi + lo) ----
-        const uint32_t hi_g = pack_bf16x2(p[0], p[1]), hi_g8 = pack_bf16x2(p[2], p[3]);
-        const uint32_t lo_g = pack_bf16x2(p[0] - bf16_lo(hi_g), p[1] - bf16_hi(hi_g));
-        const uint32_t lo_g8 = pack_bf16x2(p[2] - bf16_lo(hi_g8), p[3] - bf16_hi(hi_g8));
-        const uint32_t bh0 = movmatrix_trans(hi_g), bh1 = movmatrix_trans(hi_g8);
-        const uint32_t bl0 = movmatrix_trans(lo_g), bl1 = movmatrix_trans(lo_g8);
-        {
-            const int mrow = lane >> 3;
-            const uint8_t *vrow =
-                vs_ + (warp * 16 + (mrow >> 1) * 8 + (lane & 7)) * kRowStride + (mrow & 1) * 16;
-#pragma unroll
-            for (int mt = 0; mt < 8; mt++) {
-                uint32_t a0, a1, a2, a3;
-                ldmatrix_x4_trans(a0, a1, a2, a3, vrow + mt * 32);
-                mma_bf16_16816(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3], a0, a1, a2, a3, bh0, bh1);
-                mma_bf16_16816(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3], a0, a1, a2, a3, bl0, bl1);
-            }
-        }
+        attn_tile<G>(w, ks_, vs_, meta[stage], warp, lane, a.scale, a.lu, ucos[warp], uval[warp]);
         if (fetcher) ents[tile & 1][tid] = pend;  // slot of tile + 2, read after the barrier
         __syncthreads();  // stage may be refilled next iteration
     }
@@ -1049,57 +1164,418 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     __syncthreads();
 
     // ---- merge the 4 warps' states, write this split's partial ----
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    }
-    float *red = reinterpret_cast<float *>(smem);  // [4][G][128] acc, then m, l
-    float *redm = red + 4 * G * kHeadDim;
-    float *redl = redm + 4 * G;
-#pragma unroll
-    for (int mt = 0; mt < 8; mt++) {
-        if (h0 < G) {
-            red[(warp * G + h0) * kHeadDim + mt * 16 + gq] = acc[mt][0];
-            red[(warp * G + h0) * kHeadDim + mt * 16 + gq + 8] = acc[mt][2];
+    attn_store_partial<G>(w, reinterpret_cast<float *>(smem), warp, lane, tid, [] { __syncthreads(); }, vec0,
+                          (size_t)a.ngroups * a.subs + 1, split, a.pm, a.pl, a.pacc);
+}
+
+// ------------------------------------------------ fused scan + attend ----
+// Bit-plane codes only.  One persistent block of 14 warps per SM walks a
+// contiguous share of the live (sequence, kv head, 1024-token chunk) items,
+// like scan_planes_kernel, and attends each item's candidates itself, so the
+// candidate lists never leave shared memory and the code stream and the K/V
+// row gathers of different items overlap on the same SM:
+//   warp 0      TMA producer of the code stages (8 tables per 3-D copy);
+//   warp 1      fold of the scan partials and compaction of each item's
+//               candidates into a shared queue (sampled rows with their head
+//               masks, then the exact-set rows of the chunk with an empty mask);
+//   warps 2-5   scan: two tables of every stage each, bit-sliced counters;
+//   warps 6-13  two attention groups of 4 warps, taking alternate items:
+//               K/V rows of 64 queue entries per tile through a 2-stage
+//               cp.async ring, the same per-warp tile math as attend_kernel,
+//               one (m, l, acc) partial per item and head.
+// Hand-offs: code stages by full/empty mbarriers, scan partials by named
+// barriers 2/3 (double-buffered by item parity), queue buffers (2 per group)
+// by full/empty mbarriers; each group syncs on its own named barrier.
+constexpr int kFusedScanWarps = 4;
+constexpr int kFusedGroups = 2;
+constexpr int kFusedThreads = 32 * (2 + kFusedScanWarps + 4 * kFusedGroups);  // 448
+constexpr int kFusedQueues = 2 * kFusedGroups;                                // candidate queue buffers
+constexpr int kFusedPrefetch = 16;  // code stages pulled into L2 ahead of the ring
+
+template <int KB>
+struct FusedCfg {
+    static constexpr int kStages = KB == 8 ? 5 : 3;  // code ring depth
+};
+
+struct FusedArgs {
+    Shape s;
+    const uint16_t *q, *kc, *vc, *qcodes;
+    const int32_t *seq_lens;
+    int max_len, nchunk;
+    int32_t *cnt;         // [B*Hkv][nchunk][16]: [0] sampled union, [1+g] per head
+    uint8_t *member_out;  // nullable [B][Hq][Ncap]
+    int32_t *status;
+    float *pm, *pl, *pacc;  // [B*Hq][nchunk + 1], [..][..][128]; split = chunk
+    LogU lu;
+    float scale;
+};
+
+template <int G, int KB>
+constexpr size_t fused_smem_bytes(int L)
+{
+    return (size_t)FusedCfg<KB>::kStages * PlaneStage<KB>::kBytes + (size_t)L * G * ((KB + 3) & ~3) * 4 +
+           (size_t)2 * G * 2 * (kFusedScanWarps * 32) * 4 + (size_t)kFusedQueues * kChunkPlanes * 4 +
+           (size_t)kFusedGroups * kAttStages * kStageBytes;
+}
+
+__device__ __forceinline__ void bar_sync_n(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+__device__ __forceinline__ void bar_arrive_n(int id, int n) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+template <int G, int KB>
+__global__ void __launch_bounds__(kFusedThreads, 1) fused_planes_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                        FusedArgs a)
+{
+    using St = PlaneStage<KB>;
+    constexpr int S = FusedCfg<KB>::kStages, QW = (KB + 3) & ~3, NSW = kFusedScanWarps, NQ = kFusedQueues;
+    constexpr int SCAN_T = NSW * 32, HAND_T = SCAN_T + 32;  // scan warps; scan warps + the compaction warp
+    const Shape &s = a.s;
+    extern __shared__ __align__(1024) uint8_t dyn_raw[];
+    uint32_t *ring = reinterpret_cast<uint32_t *>(dyn_raw);  // [S][box][8 tables][kBoxWords]
+    uint32_t *qm = ring + S * St::kBytes / 4;                // [L][G][QW]
+    uint32_t *part = qm + s.L * G * QW;                      // [2][G][2][SCAN_T]
+    uint32_t *cq = part + 2 * G * 2 * SCAN_T;                // [NQ][1024] queue entries
+    uint8_t *att = reinterpret_cast<uint8_t *>(cq + NQ * kChunkPlanes);  // [groups][stages][K rows, V rows]
+    __shared__ __align__(8) uint64_t full[S], empty[S], cqf[NQ], cqe[NQ];
+    __shared__ int cq_meta[NQ][4];  // unit, chunk, rows
+    __shared__ int range_sh[4];
+    __shared__ int gflag[kFusedGroups];
+    __shared__ uint32_t meta[kFusedGroups][kAttStages][kAttRows];
+    __shared__ float ucos[4 * kFusedGroups][16 * G], uval[4 * kFusedGroups][16 * G];
+    __shared__ float qinv[kFusedGroups][G];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    grid_dependency_wait();
+
+    if (threadIdx.x == 0) {
+        // this block's contiguous share of the live items (as scan_planes_kernel)
+        long long total = 0;
+        for (int b = 0; b < s.B; b++) {
+            const int n = clamp_len(a.seq_lens, b, a.max_len, a.status, blockIdx.x == 0);
+            total += (long long)s.Hkv * ((n + kChunkPlanes - 1) / kChunkPlanes);
         }
-        if (h1 < G) {
-            red[(warp * G + h1) * kHeadDim + mt * 16 + gq] = acc[mt][1];
-            red[(warp * G + h1) * kHeadDim + mt * 16 + gq + 8] = acc[mt][3];
+        long long x = total * blockIdx.x / gridDim.x;
+        const long long x1 = total * (blockIdx.x + 1) / gridDim.x;
+        range_sh[3] = (int)(x1 - x);
+        range_sh[0] = range_sh[1] = range_sh[2] = 0;
+        for (int b = 0; b < s.B && x1 > x; b++) {
+            const int n = min(max(a.seq_lens[b], 0), a.max_len);
+            const long long nch = (n + kChunkPlanes - 1) / kChunkPlanes, items = nch * s.Hkv;
+            if (x < items) {
+                range_sh[0] = b;
+                range_sh[1] = (int)(x / nch);
+                range_sh[2] = (int)(x % nch);
+                break;
+            }
+            x -= items;
         }
-    }
-    if (gq == 0) {
-        if (h0 < G) {
-            redm[warp * G + h0] = m0;
-            redl[warp * G + h0] = l0;
+        for (int i = 0; i < S; i++) {
+            mbar_init(smem_u32(&full[i]), 1);
+            mbar_init(smem_u32(&empty[i]), NSW);
         }
-        if (h1 < G) {
-            redm[warp * G + h1] = m1;
-            redl[warp * G + h1] = l1;
+        for (int i = 0; i < NQ; i++) {
+            mbar_init(smem_u32(&cqf[i]), 1);
+            mbar_init(smem_u32(&cqe[i]), 1);
         }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    const int dim = tid;  // 128 threads = head_dim
-    for (int g = 0; g < G; g++) {
-        float M = -INFINITY;
-        for (int w = 0; w < 4; w++) M = fmaxf(M, redm[w * G + g]);
-        float Ls = 0.f, A = 0.f;
-        if (M != -INFINITY) {
-            for (int w = 0; w < 4; w++) {
-                const float mw = redm[w * G + g];
-                if (mw == -INFINITY) continue;
-                const float f = expf(mw - M);
-                Ls += redl[w * G + g] * f;
-                A += red[(w * G + g) * kHeadDim + dim] * f;
+    const int count = range_sh[3];
+    if (count <= 0) return;
+    LiveCursor cur;
+    cur.b = range_sh[0];
+    cur.kvh = range_sh[1];
+    cur.chunk = range_sh[2];
+    cur.load_seq(a.seq_lens, a.max_len);
+    const int nst = (s.L + 7) / 8;  // stages per item
+
+    if (warp == 0) {
+        // -------------------------------------------------- code producer ----
+        if (lane == 0) {
+            int e = 0;
+            LiveCursor pc = cur;
+            // a second cursor kFusedPrefetch stages ahead pulls stages into L2,
+            // so that far more code bytes are in flight than the ring holds
+            LiveCursor fc = cur;
+            int fj = 0, fit = 0;
+            auto prefetch_next = [&] {
+                if (fit >= count) return;
+#pragma unroll
+                for (int bx = 0; bx < St::kBoxes; bx++)
+                    tma_prefetch_3d(&tmap, fc.chunk * 32 * KB + bx * St::kBoxWords, 8 * fj, fc.unit(s));
+                if (++fj == nst) {
+                    fj = 0;
+                    fit++;
+                    fc.next(s, a.seq_lens, a.max_len);
+                }
+            };
+            for (int i = 0; i < kFusedPrefetch; i++) prefetch_next();
+            for (int it = 0; it < count; it++, pc.next(s, a.seq_lens, a.max_len)) {
+                const int x0 = pc.chunk * 32 * KB, z = pc.unit(s);
+                bool ok = true;
+                for (int j = 0; j < nst; j++, e++) {
+                    const int st = e % S;
+                    prefetch_next();
+                    if (e >= S && !mbar_wait_bounded(smem_u32(&empty[st]), (uint32_t)(e / S - 1) & 1u)) {
+                        set_status(a.status, MP_ERR_CUDA);
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(smem_u32(&full[st]), St::kBytes);
+#pragma unroll
+                    for (int bx = 0; bx < St::kBoxes; bx++)
+                        tma_load_3d(smem_u32(ring) + (uint32_t)(st * St::kBytes + bx * 8 * St::kBoxWords * 4), &tmap,
+                                    smem_u32(&full[st]), x0 + bx * St::kBoxWords, 8 * j, z);
+                }
+                if (!ok) break;
+            }
+            // every code copy issued lands before the block exits (the last use of each stage)
+            for (int st = 0; st < S && st < e; st++) {
+                const int last = st + ((e - 1 - st) / S) * S;
+                mbar_wait_bounded(smem_u32(&full[st]), (uint32_t)(last / S) & 1u);
             }
         }
-        const size_t bh = vec0 + g;
-        const size_t pidx = bh * ((size_t)a.ngroups * a.subs + 1) + split;
-        a.pacc[pidx * kHeadDim + dim] = A;
-        if (dim == 0) {
-            a.pm[pidx] = M;
-            a.pl[pidx] = Ls;
+        return;
+    }
+
+    if (warp == 1) {
+        // --------------------------------------------- fold and compaction ----
+        for (int ci = 0; ci < count; ci++, cur.next(s, a.seq_lens, a.max_len)) {
+            const int qb = ci % NQ;
+            bar_sync_n(2, HAND_T);  // the scan partials of item ci are in buffer ci & 1
+            const uint32_t *pp = part + (ci & 1) * (G * 2 * SCAN_T);
+            uint32_t s1[G], s2[G];
+#pragma unroll
+            for (int g = 0; g < G; g++) s1[g] = s2[g] = 0u;
+#pragma unroll 1
+            for (int t = 0; t < NSW; t++) {
+#pragma unroll
+                for (int g = 0; g < G; g++) {
+                    const uint32_t a1 = pp[(g * 2 + 0) * SCAN_T + t * 32 + lane];
+                    const uint32_t a2 = pp[(g * 2 + 1) * SCAN_T + t * 32 + lane];
+                    s2[g] |= a2 | (s1[g] & a1);
+                    s1[g] |= a1;
+                }
+            }
+            if (ci + 1 < count) bar_arrive_n(3, HAND_T);  // item ci read: the scan may post item ci + 1
+            // the queue buffer's previous item (ci - NQ) must have been attended
+            bool free_ok = true;
+            if (ci >= NQ && lane == 0)
+                free_ok = mbar_wait_bounded(smem_u32(&cqe[qb]), (uint32_t)(ci / NQ - 1) & 1u);
+            if (!__shfl_sync(0xffffffffu, (int)free_ok, 0) && lane == 0) set_status(a.status, MP_ERR_CUDA);
+            const int unit = cur.unit(s), N = cur.N, c0 = cur.chunk * kChunkPlanes, t0 = c0 + lane * 32;
+            uint32_t *q_ent = cq + qb * kChunkPlanes;
+            // sampled rows: tokens in [sink, N - window) and below N, in token order
+            const uint32_t v = range_mask(t0, s.sink, min(N - s.window, N), 32);
+            uint32_t any = 0u;
+#pragma unroll
+            for (int g = 0; g < G; g++) {
+                s2[g] &= v;
+                any |= s2[g];
+            }
+            const int mine = __popc(any);
+            int incl = mine;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += t;
+            }
+            const int nsamp = __shfl_sync(0xffffffffu, incl, 31);
+            int off = incl - mine;
+            while (any) {
+                const int bit = __ffs(any) - 1;
+                any &= any - 1u;
+                uint32_t heads = 0u;
+#pragma unroll
+                for (int g = 0; g < G; g++) heads |= ((s2[g] >> bit) & 1u) << g;
+                q_ent[off++] = (uint32_t)(t0 + bit) | (heads << 24);
+            }
+            // then the chunk's exact-set rows (empty head mask)
+            const int n_sink = min(s.sink, N), win0 = max(n_sink, N - s.window);
+            const int sink_hi = min(c0 + kChunkPlanes, n_sink);
+            const int win_lo = max(c0, win0), win_hi = min(c0 + kChunkPlanes, N);
+            const int na = max(0, sink_hi - c0), nb = max(0, win_hi - win_lo);
+            for (int i = lane; i < na + nb; i += 32)
+                q_ent[nsamp + i] = (uint32_t)(i < na ? c0 + i : win_lo + (i - na));
+            int32_t *cnt = a.cnt + ((size_t)unit * a.nchunk + cur.chunk) * 16;
+            if (lane == 0) cnt[0] = nsamp;
+#pragma unroll
+            for (int g = 0; g < G; g++) {
+                int c = __popc(s2[g]);
+#pragma unroll
+                for (int d = 16; d > 0; d >>= 1) c += __shfl_xor_sync(0xffffffffu, c, d);
+                if (lane == 0) cnt[1 + g] = c;
+            }
+            if (a.member_out)
+                for (int i = 0; i < 32 && t0 + i < N; i++)
+#pragma unroll
+                    for (int g = 0; g < G; g++)
+                        a.member_out[((size_t)cur.b * s.Hq + cur.kvh * G + g) * s.Ncap + t0 + i] =
+                            (s2[g] >> i) & 1u;
+            if (lane == 0) {
+                cq_meta[qb][0] = unit;
+                cq_meta[qb][1] = cur.chunk;
+                cq_meta[qb][2] = nsamp + na + nb;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&cqf[qb]));  // the queue buffer is ready for its group
         }
+        return;
+    }
+
+    if (warp < 2 + NSW) {
+        // ------------------------------------------------------------ scan ----
+        const int ts = warp - 2;  // tables 8 j + ts and 8 j + ts + 4 of stage j
+        int e = 0, qm_unit = -1;
+        bool dead = false;
+        for (int it = 0; it < count; it++, cur.next(s, a.seq_lens, a.max_len)) {
+            const int unit = cur.unit(s);
+            if (unit != qm_unit) {  // uniform over the scan warps
+                if (qm_unit >= 0) bar_sync_n(1, SCAN_T);  // every scan warp is done with the old masks
+                for (int i = threadIdx.x - 64; i < s.L * G; i += SCAN_T) {
+                    const int l = i / G, g = i % G;
+                    const unsigned code = a.qcodes[((size_t)cur.b * s.Hq + cur.kvh * G + g) * s.L + l];
+                    uint4 *dst = reinterpret_cast<uint4 *>(qm + (size_t)i * QW);
+#pragma unroll
+                    for (int q = 0; q < QW / 4; q++) {
+                        uint32_t m[4];
+#pragma unroll
+                        for (int x = 0; x < 4; x++) m[x] = 4 * q + x < KB ? 0u - ((code >> (4 * q + x)) & 1u) : 0u;
+                        dst[q] = make_uint4(m[0], m[1], m[2], m[3]);
+                    }
+                }
+                bar_sync_n(1, SCAN_T);
+                qm_unit = unit;
+            }
+            uint32_t s1[G], s2[G];
+#pragma unroll
+            for (int g = 0; g < G; g++) s1[g] = s2[g] = 0u;
+            for (int j = 0; j < nst; j++, e++) {
+                const int st = e % S;
+                if (!dead) {
+                    const bool landed = mbar_wait_bounded(smem_u32(&full[st]), (uint32_t)(e / S) & 1u);
+                    if (!__all_sync(0xffffffffu, landed)) {
+                        if (lane == 0) set_status(a.status, MP_ERR_CUDA);
+                        dead = true;
+                    }
+                }
+#pragma unroll
+                for (int half = 0; half < 2; half++) {
+                    const int r = ts + 4 * half, l = 8 * j + r;  // row of the stage, table
+                    if (dead || l >= s.L) continue;
+                    const int box = (lane * KB) / St::kBoxWords, in_box = lane * KB - box * St::kBoxWords;
+                    const uint32_t *src = ring + st * (St::kBytes / 4) + box * 8 * St::kBoxWords + r * St::kBoxWords + in_box;
+                    uint32_t pw[KB];
+                    if constexpr (KB % 4 == 0) {
+#pragma unroll
+                        for (int q = 0; q < KB / 4; q++) {
+                            const uint4 v = reinterpret_cast<const uint4 *>(src)[q];
+                            pw[4 * q] = v.x;
+                            pw[4 * q + 1] = v.y;
+                            pw[4 * q + 2] = v.z;
+                            pw[4 * q + 3] = v.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < KB / 2; q++) {
+                            const uint2 v = reinterpret_cast<const uint2 *>(src)[q];
+                            pw[2 * q] = v.x;
+                            pw[2 * q + 1] = v.y;
+                        }
+                    }
+#pragma unroll
+                    for (int g = 0; g < G; g++) {
+                        const uint4 *m4 = reinterpret_cast<const uint4 *>(qm + (l * G + g) * QW);
+                        uint32_t mis = 0u;
+#pragma unroll
+                        for (int q = 0; q < QW / 4; q++) {
+                            const uint4 mq = m4[q];
+                            const uint32_t mm[4] = {mq.x, mq.y, mq.z, mq.w};
+#pragma unroll
+                            for (int x = 0; x < 4; x++)
+                                if (4 * q + x < KB) mis |= pw[4 * q + x] ^ mm[x];
+                        }
+                        s2[g] |= s1[g] & ~mis;
+                        s1[g] |= ~mis;
+                    }
+                }
+                // release the stage once every lane has used its words
+                __syncwarp();
+                if (lane == 0 && !dead) {
+                    fence_proxy_async_smem();
+                    mbar_arrive(smem_u32(&empty[st]));
+                }
+            }
+            if (it >= 1) bar_sync_n(3, HAND_T);  // warp 0 has read item it - 1's partials
+            uint32_t *pp = part + (it & 1) * (G * 2 * SCAN_T);
+#pragma unroll
+            for (int g = 0; g < G; g++) {
+                pp[(g * 2 + 0) * SCAN_T + ts * 32 + lane] = s1[g];
+                pp[(g * 2 + 1) * SCAN_T + ts * 32 + lane] = s2[g];
+            }
+            bar_arrive_n(2, HAND_T);
+        }
+        return;
+    }
+
+    // ------------------------------------------------------- attention ----
+    const int grp = (warp - 2 - NSW) >> 2, gw = (warp - 2 - NSW) & 3, gtid = gw * 32 + lane;
+    const int gbar_id = 4 + grp;
+    auto gbar = [&] { bar_sync_n(gbar_id, 128); };
+    uint8_t *gring = att + grp * kAttStages * kStageBytes;
+    const uint32_t dmeta = ((1u << G) - 1u) | 0x100u;
+    for (int k = grp; k < count; k += kFusedGroups) {
+        const int qb = k % NQ;
+        if (gtid == 0) gflag[grp] = mbar_wait_bounded(smem_u32(&cqf[qb]), (uint32_t)(k / NQ) & 1u) ? 1 : 0;
+        gbar();  // the queue buffer (and, from the item before, the ring and qinv) is ours
+        if (!gflag[grp]) {
+            if (gtid == 0) set_status(a.status, MP_ERR_CUDA);
+            break;
+        }
+        const int unit = cq_meta[qb][0], chunk = cq_meta[qb][1], rows = cq_meta[qb][2];
+        const int b = unit / s.Hkv, kvh = unit % s.Hkv;
+        const size_t vec0 = (size_t)b * s.Hq + (size_t)kvh * G;
+        const uint16_t *kbase = a.kc + (size_t)unit * s.Ncap * kHeadDim;
+        const uint16_t *vbase = a.vc + (size_t)unit * s.Ncap * kHeadDim;
+        const uint32_t *ents = cq + qb * kChunkPlanes;
+        AttnWarp<G> w;
+        attn_begin<G>(w, a.q, vec0, lane);
+        attn_qinv<G>(a.q, vec0, gw, lane, qinv[grp]);
+        auto issue = [&](int tile, int stage) {
+            uint8_t *ks_ = gring + stage * kStageBytes;
+            uint8_t *vs_ = ks_ + kAttRows * kRowStride;
+            const int col = gtid & 15;
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const int r = (gtid >> 4) + 8 * i, idx = tile * kAttRows + r;
+                const uint32_t ent = idx < rows ? ents[idx] : 0xFFFFFFFFu;
+                const bool ok = ent != 0xFFFFFFFFu;
+                const int tok = ok ? (int)(ent & 0xFFFFFFu) : 0;
+                const size_t off = (size_t)tok * kHeadDim + col * 8;
+                cp_async_16(ks_ + r * kRowStride + col * 16, kbase + off, ok ? 16 : 0);
+                cp_async_16(vs_ + r * kRowStride + col * 16, vbase + off, ok ? 16 : 0);
+                if (col == 0) meta[grp][stage][r] = ok ? ((ent >> 24) ? (ent >> 24) : dmeta) : 0u;
+            }
+        };
+        const int ntiles = (rows + kAttRows - 1) / kAttRows;
+        if (ntiles > 0) issue(0, 0);
+        cp_async_commit();
+        gbar();  // qinv
+        attn_set_qinv<G>(w, qinv[grp], lane);
+        for (int tile = 0; tile < ntiles; tile++) {
+            if (tile + 1 < ntiles) issue(tile + 1, (tile + 1) % kAttStages);
+            cp_async_commit();
+            cp_async_wait<kAttStages - 1>();
+            gbar();
+            const int stage = tile % kAttStages;
+            const uint8_t *ks_ = gring + stage * kStageBytes;
+            attn_tile<G>(w, ks_, ks_ + kAttRows * kRowStride, meta[grp][stage], gw, lane, a.scale, a.lu,
+                         ucos[grp * 4 + gw], uval[grp * 4 + gw]);
+            gbar();  // the stage may be refilled
+        }
+        cp_async_wait<0>();
+        gbar();  // every entry of the queue buffer has been read, the ring is idle
+        if (gtid == 0) mbar_arrive(smem_u32(&cqe[qb]));
+        attn_store_partial<G>(w, reinterpret_cast<float *>(gring), gw, lane, gtid, gbar, vec0,
+                              (size_t)a.nchunk + 1, chunk, a.pm, a.pl, a.pacc);
     }
 }
 
@@ -1116,7 +1592,7 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
                                                          const float *__restrict__ pl,
                                                          const float *__restrict__ pacc,
                                                          const int32_t *__restrict__ cnt, float *out,
-                                                         float *lse, int32_t *n_sampled)
+                                                         float *lse, int32_t *n_sampled, int has_d)
 {
     __shared__ float red_m[4], red_l[4];
     __shared__ int red_n[4];
@@ -1130,14 +1606,15 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
     N = N < 0 ? 0 : (N > max_len ? max_len : N);
     const int nch = (N + chunk_tokens - 1) / chunk_tokens;
     const int nsp = ((nch + span - 1) / span) * subs;  // live chunk splits
-    const int dsp = ngroups * subs;                     // the exact-set split
+    const int dsp = ngroups * subs;                     // the exact-set split (if has_d)
     const size_t base = (size_t)bh * (dsp + 1);
     auto split_index = [&](int j) { return j < nsp ? j : dsp; };  // j in [0, nsp]
+    const int last = has_d ? nsp : nsp - 1;                       // splits 0..last are read
 
     // pass 1: M = max over live splits and D; sampled count
     float m = -INFINITY;
     int ns = 0;
-    for (int j = tid; j <= nsp; j += blockDim.x) m = fmaxf(m, pm[base + split_index(j)]);
+    for (int j = tid; j <= last; j += blockDim.x) m = fmaxf(m, pm[base + split_index(j)]);
     for (int j = tid; j < nch; j += blockDim.x) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -1156,7 +1633,7 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
     float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
     if (M != -INFINITY) {
 #pragma unroll 4
-        for (int j = warp; j <= nsp; j += 4) {
+        for (int j = warp; j <= last; j += 4) {
             const size_t sp = base + split_index(j);
             const float mj = pm[sp];
             const float f = mj == -INFINITY ? 0.f : expf(mj - M);
@@ -1208,7 +1685,8 @@ struct Workspace {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// How attention blocks cover the scan chunks.  Many chunks: each block takes
+// How attention blocks cover the scan chunks (the fused kernel instead writes
+// one partial per 1024-token chunk).  Many chunks: each block takes
 // `span` consecutive chunks (about 1200 blocks in all: a few waves of 3 blocks
 // per SM, so that uneven candidate counts even out, while the per-block set-up
 // stays amortised and the merge sees few partials).  Few, large chunks:
@@ -1244,7 +1722,8 @@ Workspace workspace_layout(const Shape &s, int max_len, void *base)
     const int C = chunk_tokens(s);
     const SplitPlan sp = split_plan(s, max_len);
     const int nchunk = sp.nchunk;
-    const size_t nsplit = (size_t)sp.nsplit;
+    // bit planes may take the fused kernel, which writes one partial per chunk
+    const size_t nsplit = s.planes ? std::max((size_t)sp.nsplit, (size_t)nchunk + 1) : (size_t)sp.nsplit;
     const size_t units = (size_t)s.B * s.Hkv, bh = (size_t)s.B * s.Hq;
     size_t off = 0;
     Workspace w{};
@@ -1317,6 +1796,39 @@ static cudaError_t launch_scan_planes(const Shape &s, const uint32_t *codes, con
                       (const uint16_t *)ws.qcodes, seq_lens, max_len, nchunk, so);
 }
 
+// The fused scan + attend kernel, if its shared memory fits on the device
+// (`used` tells the caller whether it ran).  One block per SM.
+template <int G, int KB>
+static cudaError_t launch_fused(const Shape &s, const uint32_t *codes, const Workspace &ws, const FusedArgs &fa,
+                                cudaStream_t st, bool &used)
+{
+    used = false;
+    const void *fn = reinterpret_cast<const void *>(fused_planes_kernel<G, KB>);
+    const size_t sm = fused_smem_bytes<G, KB>(s.L);
+    int dev = 0, optin = 0, sms = 0;
+    cudaError_t e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cudaFuncAttributes attr;
+    if ((e = cudaFuncGetAttributes(&attr, fn)) != cudaSuccess) return e;
+    if (sm + attr.sharedSizeBytes > (size_t)optin) return cudaSuccess;  // does not fit: two-kernel path
+    if ((e = ensure_smem(fn, (int)sm)) != cudaSuccess) return e;
+    const int words = s.Ncap >> 5;
+    const uint64_t dims[3] = {(uint64_t)words * KB, (uint64_t)s.L, (uint64_t)s.B * s.Hkv};
+    const uint64_t strides[2] = {(uint64_t)words * KB * 4, (uint64_t)s.L * words * KB * 4};
+    const uint32_t box[3] = {(uint32_t)PlaneStage<KB>::kBoxWords, 8, 1};
+    CUtensorMap tmap;
+    if (!encode_tensor_map(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, codes, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const long long items = (long long)fa.nchunk * s.B * s.Hkv;
+    const int grid = (int)std::max(1LL, std::min(items, (long long)sms));
+    e = launch_pdl(fused_planes_kernel<G, KB>, dim3(grid), dim3(kFusedThreads), sm, st, tmap, fa);
+    used = e == cudaSuccess;
+    return e;
+}
+
 template <int G>
 static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint16_t *W, const void *codes,
                                    const uint16_t *kc, const uint16_t *vc, const int32_t *seq_lens,
@@ -1336,7 +1848,37 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
         if (e != cudaSuccess) return e;
     }
     ScanOut so{ws.cand, ws.cnt, dbg ? dbg->member_out : nullptr, ws.status, 1u};
-    if (nchunk > 0) {
+    const LogU lu = make_logu(s);
+    const float scale = 1.0f / sqrtf((float)s.d);
+    const int path = dbg ? dbg->path : MP_PATH_AUTO;
+    bool fused = false;
+    // The fused kernel is opt-in: it shares each SM's warps and shared memory
+    // between the code stream and the row gathers, and measured slower than
+    // giving each phase the whole device in turn.
+    if (nchunk > 0 && s.planes && path == MP_PATH_FUSED) {
+        FusedArgs fa;
+        fa.s = s;
+        fa.q = q;
+        fa.kc = kc;
+        fa.vc = vc;
+        fa.qcodes = ws.qcodes;
+        fa.seq_lens = seq_lens;
+        fa.max_len = max_len;
+        fa.nchunk = nchunk;
+        fa.cnt = ws.cnt;
+        fa.member_out = dbg ? dbg->member_out : nullptr;
+        fa.status = ws.status;
+        fa.pm = ws.pm;
+        fa.pl = ws.pl;
+        fa.pacc = ws.pacc;
+        fa.lu = lu;
+        fa.scale = scale;
+        e = s.K == 8 ? launch_fused<G, 8>(s, static_cast<const uint32_t *>(codes), ws, fa, st, fused)
+                     : launch_fused<G, 10>(s, static_cast<const uint32_t *>(codes), ws, fa, st, fused);
+        if (e != cudaSuccess) return e;
+        if (!fused && path == MP_PATH_FUSED) return cudaErrorNotSupported;
+    }
+    if (nchunk > 0 && !fused) {
         dim3 grid(nchunk, units);
         const size_t part = (size_t)2 * G * 4 * kScanThreads * sizeof(uint32_t);       // byte scan: 4 words
         if (!s.planes) {
@@ -1372,17 +1914,19 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     aa.pl = ws.pl;
     aa.pacc = ws.pacc;
 
-    aa.lu = make_logu(s);
-    aa.scale = 1.0f / sqrtf((float)s.d);
-    {
+    aa.lu = lu;
+    aa.scale = scale;
+    if (!fused) {
         const int sm = kAttStages * kStageBytes;
         if ((e = ensure_smem(reinterpret_cast<const void *>(attend_kernel<G>), sm)) != cudaSuccess) return e;
         dim3 grid(sp.nsplit, units);
         if ((e = launch_pdl(attend_kernel<G>, grid, dim3(kAttThreads), sm, st, aa)) != cudaSuccess) return e;
     }
-    e = launch_pdl(merge_kernel<G>, dim3(s.B * s.Hq), dim3(kHeadDim), 0, st, s, seq_lens, max_len, nchunk, sp.span,
-                   sp.subs, sp.ngroups, C, (const float *)ws.pm, (const float *)ws.pl, (const float *)ws.pacc,
-                   (const int32_t *)ws.cnt, out, lse, n_sampled);
+    // partials: per chunk (fused) or per split of the plan, then the exact set
+    const int m_span = fused ? 1 : sp.span, m_subs = fused ? 1 : sp.subs, m_groups = fused ? nchunk : sp.ngroups;
+    e = launch_pdl(merge_kernel<G>, dim3(s.B * s.Hq), dim3(kHeadDim), 0, st, s, seq_lens, max_len, nchunk, m_span,
+                   m_subs, m_groups, C, (const float *)ws.pm, (const float *)ws.pl, (const float *)ws.pacc,
+                   (const int32_t *)ws.cnt, out, lse, n_sampled, fused ? 0 : 1);
     if (e != cudaSuccess) return e;
     if (dbg && dbg->qcodes_out)
         e = cudaMemcpyAsync(dbg->qcodes_out, ws.qcodes, (size_t)s.B * s.Hq * s.L * sizeof(uint16_t),

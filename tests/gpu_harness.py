@@ -102,13 +102,14 @@ class Run:
             a = a.view(np.uint32)
         return unpack_codes(a, self.w.k_bits, self.w.n_tables, n, self.shape.planes)
 
-    def decode(self, qcodes_in: Optional[np.ndarray] = None, member: bool = True):
+    def decode(self, qcodes_in: Optional[np.ndarray] = None, member: bool = True, path: int = 0):
         w = self.w
         mem = torch.zeros((w.batch, w.n_q_heads, w.capacity), dtype=torch.uint8, device="cuda") if member else None
         qco = torch.zeros((w.batch, w.n_q_heads, w.n_tables), dtype=torch.int16, device="cuda")
         qci = dev(qcodes_in) if qcodes_in is not None else None
         mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
-                         self.out, self.lse, self.ns, self.ws, qcodes_in=qci, qcodes_out=qco, member_out=mem)
+                         self.out, self.lse, self.ns, self.ws, qcodes_in=qci, qcodes_out=qco, member_out=mem,
+                         path=path)
         torch.cuda.synchronize()
         res = dict(out=host(self.out), lse=host(self.lse), ns=host(self.ns), qcodes=host(qco, np.uint16))
         if member:

@@ -106,3 +106,19 @@ def test_workspace_grows_with_max_len(lib):
         assert lib.mp_decode_workspace_bytes(ctypes.byref(s), m, ctypes.byref(n)) == 0
         sizes.append(n.value)
     assert sizes == sorted(sizes) and sizes[1] < sizes[3]
+
+
+def test_decode_path_selector_checked(lib):
+    """mp_decode_debug.path: out-of-range values are MP_ERR_ARG; the fused path
+    needs bit-plane codes and at most 4 query heads per kv head (MP_ERR_SHAPE).
+    Rejected on the host, so nothing launches."""
+    A = 1 << 12  # aligned fake device pointers (never dereferenced)
+    for lay, G, path, want in [(1, 4, 2, mp.MP_ERR_SHAPE), (2, 8, 2, mp.MP_ERR_SHAPE), (2, 4, 7, mp.MP_ERR_ARG),
+                               (2, 4, -1, mp.MP_ERR_ARG)]:
+        s = good_shape(code_layout=lay, n_q_heads=2 * G)
+        need = ctypes.c_size_t()
+        assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 1024, ctypes.byref(need)) == 0
+        dbg = B._CDebug(None, None, None, path)
+        rc = lib.mp_decode_attend(ctypes.byref(s), A, A, A, A, A, A, 1024, A, A, A, A, need.value, ctypes.byref(dbg),
+                                  None)
+        assert rc == want, (lay, G, path, rc)

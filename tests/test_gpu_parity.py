@@ -94,6 +94,50 @@ def test_decode_same_codes_matches_oracle(case):
     assert gpu["ns"].sum() > 0 or w.context <= w.sink + w.window
 
 
+PLANE_CASES = ["g4_k10", "g2_k10_short", "g4_k8_planes", "g1_k8_planes_short"]
+
+
+@pytest.mark.parametrize("path", [mp.MP_PATH_SPLIT, mp.MP_PATH_FUSED])
+@pytest.mark.parametrize("case", PLANE_CASES)
+def test_plane_decode_paths_match_oracle(case, path):
+    """Bit-plane codes have two decode paths (collision scan then attention,
+    or one fused kernel); each must give the oracle's S_h exactly and its
+    outputs within tolerance on the oracle's codes."""
+    w = SMALL_CASES[case]
+    run = Run(w)
+    units, codes, _ = oracle_codes_all(run)
+    run.set_codes(codes, units)
+    qref, _ = oracle_query_codes(run.inp, w)
+    gpu = run.decode(qcodes_in=qref, path=path)
+    assert gpu["status"] == 0
+    ref = oracle_decode_units(run.inp, w, units, codes, qref)
+    check_outputs(gpu, ref, w)
+
+
+def test_fused_decode_ragged_lengths_and_boundaries():
+    """Fused path over lengths that hit its item boundaries: empty, all-exact
+    (N <= sink + window), one token past a 1024-token chunk, a chunk's last
+    token, and a long sequence; the exact set spans two chunks in one."""
+    w = SMALL_CASES["g4_k10"].with_(name="fz", batch=6, context=5000, seed=2013)
+    inp = make_inputs(w)
+    inp["seq_lens"] = np.array([0, 50, 1025, 2048, 5000, 1060], np.int32)
+    for b, n in enumerate(inp["seq_lens"]):
+        inp["K"][b, :, n:] = 0
+        inp["V"][b, :, n:] = 0
+    run = Run(w, inp)
+    units = [(b, kh) for b in range(w.batch) for kh in range(w.n_kv_heads)]
+    codes = [oracle_unit_codes(inp, w, b, kh, int(inp["seq_lens"][b]))[0] for b, kh in units]
+    run.set_codes(codes, units)
+    qref, _ = oracle_query_codes(inp, w)
+    for path in (mp.MP_PATH_FUSED, mp.MP_PATH_SPLIT):
+        gpu = run.decode(qcodes_in=qref, path=path)
+        assert gpu["status"] == 0
+        ref = oracle_decode_units(inp, w, units, codes, qref)
+        check_outputs(gpu, ref, w)
+        assert np.isneginf(gpu["lse"][0]).all() and not gpu["out"][0].any()
+        assert (gpu["ns"][1] == 0).all()
+
+
 @pytest.mark.parametrize("case", ["tiny_g1_k8", "g4_k10", "g8_k8", "g4_k8_planes"])
 def test_end_to_end_gpu_codes(case):
     """GPU hashing feeds the GPU scan.  Where a GPU code equals the oracle's,
