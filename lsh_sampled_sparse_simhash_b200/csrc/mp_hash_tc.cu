@@ -159,15 +159,30 @@ __device__ __forceinline__ float positive_unit(uint32_t bits)
     return r;
 }
 
+__device__ __forceinline__ uint64_t pair2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
 // 16-bit integer whose bit c is [v[c] > 0], built on the FMA pipe: the sum
-// sum_c [v_c > 0] 2^c is exact in fp32, and adding 2^23 puts it in the low
-// bits of the float's bit pattern.
+// sum_c [v_c > 0] 2^c is exact in fp32.  The even and the odd bits are the two
+// lanes of one paired (f32x2) FMA chain, E = sum_i u_2i 4^i and
+// O = sum_i u_2i+1 4^i, which halves the chain's length; then 2 O + E, and
+// adding 2^23 puts the integer in the low bits of the float's bit pattern.
 __device__ __forceinline__ uint32_t pack_positive16(const uint32_t *v)
 {
-    float acc = positive_unit(v[15]);
+    uint64_t acc = pair2(positive_unit(v[14]), positive_unit(v[15]));
+    const uint64_t four = 0x4080000040800000ull;  // {4.0f, 4.0f}
 #pragma unroll
-    for (int c = 14; c >= 0; c--) acc = fmaf(acc, 2.f, positive_unit(v[c]));
-    return __float_as_uint(acc + 8388608.f);
+    for (int i = 6; i >= 0; i--) {
+        const uint64_t u = pair2(positive_unit(v[2 * i]), positive_unit(v[2 * i + 1]));
+        asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(acc) : "l"(four), "l"(u));
+    }
+    float e, o;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(e), "=f"(o) : "l"(acc));
+    return __float_as_uint(fmaf(o, 2.f, e) + 8388608.f);
 }
 
 // 32-bit word whose bit c is [v[c] > 0].
