@@ -804,6 +804,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 //   P.V     O^T (128 dims x 8 heads) += V^T . P^T on the tensor cores: P is
 //           split into bf16 hi + lo parts (error ~2^-17 relative), transposed
 //           into B fragments with movmatrix, V^T comes from ldmatrix.trans.
+// 2^x with the MUFU approximation (relative error about 2^-22; flushes
+// subnormal results to zero).  The attention's log-weights are kept in base 2:
+// s log2(e) and log2 u, so each weight is a single ex2.
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
 // Attention state of one warp of a 4-warp (128-thread) group: the warp owns
 // 16 rows of every 64-row tile.  Lane (g, t) holds rows g, g + 8 for heads
 // 2t, 2t + 1, the B fragments of Q^T, those heads' online-softmax state (m, l)
@@ -870,6 +882,7 @@ __device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, co
                                           const uint32_t *meta, int warp, int lane, float scale, const LogU &lu,
                                           float *ucos, float *uval)
 {
+    const float scale2 = scale * kLog2e;  // scores in log2 units
     const int gq = lane >> 2, tq = lane & 3;
     const int h0 = 2 * tq, h1 = 2 * tq + 1;
     // ---- S^T = K rows . Q^T and |k|^2 ----
@@ -913,7 +926,7 @@ __device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, co
         for (int j = 0; j < 4; j++) {
             const bool mem = hh[j] < G && ((mrow[j] >> hh[j]) & 1u);
             need[j] = mem && !(mrow[j] & 0x100u);
-            tv[j] = mem ? c[j] * scale : -INFINITY;
+            tv[j] = mem ? c[j] * scale2 : -INFINITY;
             const uint32_t bal = __ballot_sync(0xffffffffu, need[j]);
             pos[j] = base + __popc(bal & ((1u << lane) - 1u));
             if (need[j]) ucos[pos[j]] = c[j] * qin[j] * kin[j];
@@ -924,7 +937,7 @@ __device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, co
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < 4; j++)
-            if (need[j]) tv[j] -= uval[pos[j]];
+            if (need[j]) tv[j] = fmaf(-kLog2e, uval[pos[j]], tv[j]);  // - log2 u
     }
 
     // ---- online softmax over this warp's rows (lanes with equal t share heads) ----
@@ -934,25 +947,31 @@ __device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, co
         mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, o));
         mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, o));
     }
+    // (log2 units; a running max that stays -inf keeps weights and scale at 0 / 1)
     const float mn0 = fmaxf(w.m0, mt0), mn1 = fmaxf(w.m1, mt1);
-    const float al0 = mn0 == -INFINITY ? 1.f : expf(w.m0 - mn0);
-    const float al1 = mn1 == -INFINITY ? 1.f : expf(w.m1 - mn1);
+    const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
     float p[4];
-    p[0] = tv[0] == -INFINITY ? 0.f : expf(tv[0] - mn0);
-    p[1] = tv[1] == -INFINITY ? 0.f : expf(tv[1] - mn1);
-    p[2] = tv[2] == -INFINITY ? 0.f : expf(tv[2] - mn0);
-    p[3] = tv[3] == -INFINITY ? 0.f : expf(tv[3] - mn1);
-    w.l0 = w.l0 * al0 + p[0] + p[2];
-    w.l1 = w.l1 * al1 + p[1] + p[3];
+    p[0] = fast_exp2(tv[0] - b0);  // tv = -inf -> 0
+    p[1] = fast_exp2(tv[1] - b1);
+    p[2] = fast_exp2(tv[2] - b0);
+    p[3] = fast_exp2(tv[3] - b1);
+    if (__any_sync(0xffffffffu, mn0 != w.m0 || mn1 != w.m1)) {
+        // some head's maximum moved: rescale its running sum and accumulators
+        const float al0 = fast_exp2(w.m0 - b0), al1 = fast_exp2(w.m1 - b1);
+        w.l0 *= al0;
+        w.l1 *= al1;
+#pragma unroll
+        for (int mt = 0; mt < 8; mt++) {
+            w.acc[mt][0] *= al0;
+            w.acc[mt][1] *= al1;
+            w.acc[mt][2] *= al0;
+            w.acc[mt][3] *= al1;
+        }
+    }
+    w.l0 += p[0] + p[2];
+    w.l1 += p[1] + p[3];
     w.m0 = mn0;
     w.m1 = mn1;
-#pragma unroll
-    for (int mt = 0; mt < 8; mt++) {
-        w.acc[mt][0] *= al0;
-        w.acc[mt][1] *= al1;
-        w.acc[mt][2] *= al0;
-        w.acc[mt][3] *= al1;
-    }
 
     // ---- O^T += V^T . P^T (P split into bf16 hi + lo) ----
     const uint32_t hi_g = pack_bf16x2(p[0], p[1]), hi_g8 = pack_bf16x2(p[2], p[3]);
@@ -1023,7 +1042,7 @@ __device__ __forceinline__ void attn_store_partial(AttnWarp<G> &w, float *red, i
             for (int w = 0; w < 4; w++) {
                 const float mw = redm[w * G + g];
                 if (mw == -INFINITY) continue;
-                const float f = expf(mw - M);
+                const float f = fast_exp2(mw - M);
                 Ls += redl[w * G + g] * f;
                 A += red[(w * G + g) * kHeadDim + dim] * f;
             }
@@ -1636,7 +1655,7 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
         for (int j = warp; j <= last; j += 4) {
             const size_t sp = base + split_index(j);
             const float mj = pm[sp];
-            const float f = mj == -INFINITY ? 0.f : expf(mj - M);
+            const float f = mj == -INFINITY ? 0.f : fast_exp2(mj - M);
             const float lj = pl[sp];
             const float4 aj = reinterpret_cast<const float4 *>(pacc + sp * kHeadDim)[lane];
             Ls = fmaf(lj, f, Ls);
@@ -1667,7 +1686,7 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
         o.w *= inv;
         reinterpret_cast<float4 *>(out + (size_t)bh * kHeadDim)[lane] = o;
         if (lane == 0) {
-            lse[bh] = Lt > 0.f ? M + logf(Lt) : -INFINITY;
+            lse[bh] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;  // partials keep log2 units
             n_sampled[bh] = red_n[0] + red_n[1] + red_n[2] + red_n[3];
         }
     }
