@@ -108,6 +108,24 @@ int mp_hash_keys(const mp_shape *shape, const void *keys, const void *W, const i
                  int32_t n_tokens, void *codes, int32_t *status, void *stream);
 
 /*
+ * Streamed key hashing: SimHash of the token range [first_token, first_token +
+ * n_tokens) of every (b, kv head) unit, for a prefill that fills the cache
+ * block by block (the pages' "optimized hash table construction", done while
+ * the cache grows).  Same kernel and arithmetic as mp_hash_keys; nothing
+ * outside the range is read, and for the byte layout nothing outside it is
+ * written.  It can run on a second stream next to mp_decode_attend calls that
+ * read only tokens below first_token.
+ *   first_token  multiple of 128 (the kernel's row tile); else MP_ERR_ALIGN
+ *   n_tokens     >= 0, first_token + n_tokens <= Ncap (else MP_ERR_CAPACITY)
+ *   keys, W, codes, status, stream as for mp_hash_keys.  With bit-plane codes
+ *   the 32-token word holding the range's last token is written whole: its
+ *   bits for tokens past the range are cleared (they are hashed with a later
+ *   block).
+ */
+int mp_hash_keys_range(const mp_shape *shape, const void *keys, const void *W, int32_t first_token,
+                       int32_t n_tokens, void *codes, int32_t *status, void *stream);
+
+/*
  * Query hashing: qcodes[b][h][l] (uint16) = table-l SimHash code of q[b][h].
  *   q bf16 [B][Hq][d]; W as above; qcodes out uint16 [B][Hq][L].
  */

@@ -16,6 +16,7 @@ from ._binding import (  # noqa: F401
     decode_attend_noalloc,
     decode_workspace_bytes,
     hash_keys,
+    hash_keys_range,
     hash_queries,
     library,
     library_path,
@@ -40,6 +41,6 @@ from ._binding import (  # noqa: F401
 __all__ = [
     "MagicPIGError", "Shape", "append_token", "codes_bytes", "codes_shape", "decode_attend",
     "decode_attend_noalloc",
-    "decode_workspace_bytes", "hash_keys", "hash_queries", "library", "library_path", "read_status",
+    "decode_workspace_bytes", "hash_keys", "hash_keys_range", "hash_queries", "library", "library_path", "read_status",
     "status_string",
 ]

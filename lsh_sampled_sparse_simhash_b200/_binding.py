@@ -78,6 +78,7 @@ def library() -> ctypes.CDLL:
         SP = ctypes.POINTER(_CShape)
         lib.mp_codes_bytes.argtypes = [SP, ctypes.POINTER(SZ)]
         lib.mp_hash_keys.argtypes = [SP, P, P, P, I32, P, P, P]
+        lib.mp_hash_keys_range.argtypes = [SP, P, P, I32, I32, P, P, P]
         lib.mp_hash_queries.argtypes = [SP, P, P, P, P]
         lib.mp_append_token.argtypes = [SP, P, P, P, P, P, P, P, P, P]
         lib.mp_decode_workspace_bytes.argtypes = [SP, I32, ctypes.POINTER(SZ)]
@@ -87,7 +88,7 @@ def library() -> ctypes.CDLL:
         lib.mp_read_status.argtypes = [P, ctypes.POINTER(I32), P]
         lib.mp_status_string.argtypes = [ctypes.c_int]
         lib.mp_status_string.restype = ctypes.c_char_p
-        for f in ("mp_codes_bytes", "mp_hash_keys", "mp_hash_queries", "mp_append_token",
+        for f in ("mp_codes_bytes", "mp_hash_keys", "mp_hash_keys_range", "mp_hash_queries", "mp_append_token",
                   "mp_decode_workspace_bytes", "mp_decode_attend", "mp_decode_attend_noalloc",
                   "mp_read_status"):
             getattr(lib, f).restype = ctypes.c_int
@@ -149,6 +150,14 @@ def decode_workspace_bytes(shape: Shape, max_len: int) -> int:
 def hash_keys(shape: Shape, keys, W, n_tokens: int, codes, seq_lens=None, status=None, stream=None):
     _check(library().mp_hash_keys(ctypes.byref(shape.c()), _ptr(keys), _ptr(W), _ptr(seq_lens), int(n_tokens),
                                   _ptr(codes), _ptr(status), _stream(stream)), "mp_hash_keys")
+
+
+def hash_keys_range(shape: Shape, keys, W, first_token: int, n_tokens: int, codes, status=None, stream=None):
+    """Hashes tokens [first_token, first_token + n_tokens) of every unit (a
+    streamed prefill block; first_token a multiple of 128)."""
+    _check(library().mp_hash_keys_range(ctypes.byref(shape.c()), _ptr(keys), _ptr(W), int(first_token),
+                                        int(n_tokens), _ptr(codes), _ptr(status), _stream(stream)),
+           "mp_hash_keys_range")
 
 
 def hash_queries(shape: Shape, q, W, qcodes, stream=None):

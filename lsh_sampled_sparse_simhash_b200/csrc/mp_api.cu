@@ -108,7 +108,22 @@ int mp_hash_keys(const mp_shape *shape, const void *keys, const void *W, const i
     if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return MP_ERR_ALIGN;
     if (n_tokens < 0 || n_tokens > s.Ncap) return MP_ERR_CAPACITY;
     return cuda_status(launch_hash_keys_tc(s, static_cast<const uint16_t *>(keys), static_cast<const uint16_t *>(W),
-                                           seq_lens, n_tokens, codes, status, static_cast<cudaStream_t>(stream)));
+                                           seq_lens, 0, n_tokens, codes, status, static_cast<cudaStream_t>(stream)));
+}
+
+int mp_hash_keys_range(const mp_shape *shape, const void *keys, const void *W, int32_t first_token,
+                       int32_t n_tokens, void *codes, int32_t *status, void *stream)
+{
+    Shape s;
+    int r = validate_shape(shape, s);
+    if (r) return r;
+    if ((r = check_ptrs({keys, W, codes}))) return r;
+    if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return MP_ERR_ALIGN;
+    if (first_token < 0 || n_tokens < 0 || (int64_t)first_token + n_tokens > s.Ncap) return MP_ERR_CAPACITY;
+    if (first_token % 128 != 0) return MP_ERR_ALIGN;
+    return cuda_status(launch_hash_keys_tc(s, static_cast<const uint16_t *>(keys), static_cast<const uint16_t *>(W),
+                                           nullptr, first_token, n_tokens, codes, status,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int mp_hash_queries(const mp_shape *shape, const void *q, const void *W, uint16_t *qcodes, void *stream)

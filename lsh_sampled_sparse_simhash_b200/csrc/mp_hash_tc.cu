@@ -59,7 +59,8 @@ struct Params {
     const int32_t *seq_lens;
     void *codes;
     int32_t *status;
-    int n_tokens;
+    int tok0;        // first token of the hashed range (multiple of kBM)
+    int n_tokens;    // tokens of the range
     int n_mt;        // 128-row tiles per unit
     int ngroups;
     int gsize;       // columns per group (multiple of 32)
@@ -248,13 +249,13 @@ __device__ __forceinline__ Item make_item(const Params &p, int group, int unit, 
     r.group = group;
     r.unit = unit;
     r.mt = mt;
-    int len = p.n_tokens;
+    int len = p.tok0 + p.n_tokens;  // end of the range (absolute token index)
     if (p.seq_lens) {
         const int b = (int)__umulhi((uint32_t)unit, p.hmagic);  // unit / Hkv
         len = min(len, max(b < kLensCache ? lens_sh[b] : p.seq_lens[b], 0));
     }
     r.len = len;
-    r.skip = r.mt * kBM >= len;
+    r.skip = p.tok0 + r.mt * kBM >= len;
     return r;
 }
 
@@ -391,13 +392,14 @@ __device__ __forceinline__ void epilogue(const Params &p, const int *lens_sh, ui
         group_cols(p, im.group, c0, width);
         TileDst td;
         td.len = im.len;
-        td.valid = im.mt * kBM + row < im.len;
-        td.warp_live = im.mt * kBM + q4 * 32 < im.len;
-        td.t4 = im.mt * kBM + q4 * 32 + (lane & ~3);
+        const int tile0 = p.tok0 + im.mt * kBM;  // first token of this row tile
+        td.valid = tile0 + row < im.len;
+        td.warp_live = tile0 + q4 * 32 < im.len;
+        td.t4 = tile0 + q4 * 32 + (lane & ~3);
         td.full4 = td.t4 + 3 < im.len;
         td.bytes = static_cast<uint8_t *>(p.codes) + (size_t)im.unit * s.L * s.Ncap + td.t4;
         td.planes = static_cast<uint32_t *>(p.codes) + (size_t)im.unit * s.L * words * s.K +
-                    ((im.mt * kBM + q4 * 32) >> 5) * s.K;
+                    ((tile0 + q4 * 32) >> 5) * s.K;
         for (int n0 = 0; n0 < width; n0 += kAccCols, seq++) {
             const int acc = seq & (kAccBufs - 1);
             const int nw = min(kAccCols, width - n0);
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!mbar_wait(empty_a(stage), empty_par[stage] ^ 1u, &abort_flag, p.status)) break;
             empty_par[stage] ^= 1u;
-            const int row0 = im.unit * s.Ncap + im.mt * kBM;
+            const int row0 = im.unit * s.Ncap + p.tok0 + im.mt * kBM;
             // later tiles of this block into L2: the first pass covers 2..kPrefetchAhead
             // items ahead, every later pass the one newly kPrefetchAhead ahead
             for (int ahead = first_pass ? 2 : kPrefetchAhead; ahead <= kPrefetchAhead; ahead++) {
@@ -503,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (it2 < p.total_items) {
                     const Item i2 = item_of(p, it2, lens_sh);
                     if (!i2.skip) {
-                        const int r2 = i2.unit * s.Ncap + i2.mt * kBM;
+                        const int r2 = i2.unit * s.Ncap + p.tok0 + i2.mt * kBM;
                         tma_prefetch_l2_2d(&tmap_keys, 0, r2);
                         tma_prefetch_l2_2d(&tmap_keys, 64, r2);
                     }
@@ -642,7 +644,7 @@ bool encode_tensor_map(CUtensorMap *m, CUtensorMapDataType type, int rank, const
 }
 
 cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint16_t *W, const int32_t *seq_lens,
-                                int n_tokens, void *codes, int32_t *status, cudaStream_t st)
+                                int tok0, int n_tokens, void *codes, int32_t *status, cudaStream_t st)
 {
     using namespace tc;
     if (n_tokens == 0) return cudaSuccess;
@@ -651,6 +653,7 @@ cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint
     p.seq_lens = seq_lens;
     p.codes = codes;
     p.status = status;
+    p.tok0 = tok0;
     p.n_tokens = n_tokens;
     p.n_mt = (n_tokens + kBM - 1) / kBM;
     p.ngroups = (s.LK + kMaxGroupCols - 1) / kMaxGroupCols;

@@ -16,8 +16,10 @@ bool aligned16(const void *p);
 int check_ptrs(std::initializer_list<const void *> ptrs);
 int cuda_status(cudaError_t e);
 
+// Hashes tokens [tok0, tok0 + n_tokens) of every unit (tok0 a multiple of 128;
+// with seq_lens, unit (b, .) stops at seq_lens[b]).
 cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint16_t *W, const int32_t *seq_lens,
-                                int n_tokens, void *codes, int32_t *status, cudaStream_t st);
+                                int tok0, int n_tokens, void *codes, int32_t *status, cudaStream_t st);
 cudaError_t launch_hash_queries(const Shape &s, const uint16_t *q, const uint16_t *W, uint16_t *qcodes,
                                 cudaStream_t st);
 cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t *v_new, const uint16_t *W,

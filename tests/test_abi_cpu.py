@@ -122,3 +122,23 @@ def test_decode_path_selector_checked(lib):
         rc = lib.mp_decode_attend(ctypes.byref(s), A, A, A, A, A, A, 1024, A, A, A, A, need.value, ctypes.byref(dbg),
                                   None)
         assert rc == want, (lay, G, path, rc)
+
+
+def test_hash_range_checked(lib):
+    """mp_hash_keys_range: the range starts on a 128-token tile and ends within
+    the capacity; rejected on the host, so nothing launches."""
+    s = good_shape()
+    A = 1 << 12
+    f = lib.mp_hash_keys_range
+    assert f(ctypes.byref(s), A, A, 64, 10, A, None, None) == mp.MP_ERR_ALIGN
+    assert f(ctypes.byref(s), A, A, 896, 129, A, None, None) == mp.MP_ERR_CAPACITY
+    assert f(ctypes.byref(s), A, A, -128, 10, A, None, None) == mp.MP_ERR_CAPACITY
+    assert f(ctypes.byref(s), A, A, 0, -1, A, None, None) == mp.MP_ERR_CAPACITY
+
+
+def test_binding_declares_argument_types_for_every_entry_point(lib):
+    """Every C entry point has ctypes argument types, so no 64-bit pointer or
+    stream handle is ever passed as a C int."""
+    decl = re.findall(r"^\s*(?:int|const char \*)\s*(mp_\w+)\s*\(", open(HEADER).read(), re.M)
+    for name in decl:
+        assert getattr(lib, name).argtypes is not None, name
