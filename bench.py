@@ -152,19 +152,25 @@ class Bench:
         def dev(a):
             return torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a)).to(device)
 
-        self.W, self.q, self.K, self.V = dev(inp["W"]), dev(inp["q"]), dev(inp["K"]), dev(inp["V"])
-        self.k_new, self.v_new = dev(inp["k_new"]), dev(inp["v_new"])
-        self.lens0 = dev(inp["seq_lens"].astype(np.int32))
-        self.lens = self.lens0.clone()
+        self.W, self.K, self.V = dev(inp["W"]), dev(inp["K"]), dev(inp["V"])
+        # The per-step inputs (q, k_new, v_new, lengths) live in one device
+        # buffer and the outputs (out, lse, n_sampled) in another, so that the
+        # end-to-end measurement moves each direction with a single copy.
+        step_in = [inp["q"].view(np.int16), inp["k_new"].view(np.int16), inp["v_new"].view(np.int16),
+                   inp["seq_lens"].astype(np.int32)]
+        self.in_host = _pack_host(step_in)
+        self.in_dev = torch.from_numpy(self.in_host).to(device)
+        self.q, self.k_new, self.v_new, self.lens = _views(self.in_dev, step_in)
+        self.lens0 = self.lens.clone()
         self.prefill = int(inp["seq_lens"].max())
         self.max_len = self.prefill + 1
         kind, cshape = mp.codes_shape(self.shape)
         self.codes = torch.zeros(cshape, dtype=torch.uint8 if kind == "uint8" else torch.int32, device=device)
         self.ws = torch.empty(mp.decode_workspace_bytes(self.shape, self.max_len), dtype=torch.uint8, device=device)
         B, Hq, d = w.batch, w.n_q_heads, w.head_dim
-        self.out = torch.empty((B, Hq, d), dtype=torch.float32, device=device)
-        self.lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
-        self.ns = torch.empty((B, Hq), dtype=torch.int32, device=device)
+        step_out = [np.zeros((B, Hq, d), np.float32), np.zeros((B, Hq), np.float32), np.zeros((B, Hq), np.int32)]
+        self.out_dev = torch.from_numpy(_pack_host(step_out)).to(device)
+        self.out, self.lse, self.ns = _views(self.out_dev, step_out)
         self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
         self.tokens = step_tokens(inp["seq_lens"] + 1)
         self.path = {"auto": mp.MP_PATH_AUTO, "split": mp.MP_PATH_SPLIT, "fused": mp.MP_PATH_FUSED}[path]
@@ -289,39 +295,53 @@ class Bench:
                     hash_rows_per_s_concurrent=rows / (t_both / 1e3))
 
     def run_e2e(self, steps, warmup):
-        """Public API with host buffers: per step, H2D of the step's inputs
-        (q, k_new, v_new, lengths) from pinned memory, the three calls, and
-        D2H of out / lse / n_sampled into pinned memory; device-timed."""
+        """Public API with host buffers: per step, one H2D copy of the step's
+        inputs (q, k_new, v_new, lengths, packed) from pinned memory, the
+        three calls, and one D2H copy of out / lse / n_sampled (packed) into
+        pinned memory; device-timed."""
         torch = self.torch
-        hq = torch.from_numpy(self.inp["q"].view(np.int16)).pin_memory()
-        hk = torch.from_numpy(self.inp["k_new"].view(np.int16)).pin_memory()
-        hv = torch.from_numpy(self.inp["v_new"].view(np.int16)).pin_memory()
-        hl = torch.from_numpy(self.inp["seq_lens"].astype(np.int32)).pin_memory()
-        ho = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
-        hlse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
-        hns = torch.empty(self.ns.shape, dtype=torch.int32).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hl))
-        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hns))
+        hin = torch.from_numpy(self.in_host).pin_memory()
+        hout = torch.empty(self.out_dev.shape, dtype=torch.uint8).pin_memory()
+        h2d = hin.numel()
+        d2h = hout.numel()
         times = []
         for i in range(warmup + steps):
             self.flush.zero_()
             s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s.record()
-            self.q.copy_(hq, non_blocking=True)
-            self.k_new.copy_(hk, non_blocking=True)
-            self.v_new.copy_(hv, non_blocking=True)
-            self.lens.copy_(hl, non_blocking=True)
+            self.in_dev.copy_(hin, non_blocking=True)
             self.hash()
             self.append()
             self.decode()
-            ho.copy_(self.out, non_blocking=True)
-            hlse.copy_(self.lse, non_blocking=True)
-            hns.copy_(self.ns, non_blocking=True)
+            hout.copy_(self.out_dev, non_blocking=True)
             e.record()
             e.synchronize()
             if i >= warmup:
                 times.append(s.elapsed_time(e))
         return statistics.mean(times), h2d, d2h
+
+
+def _pack_host(arrays):
+    """Concatenates arrays into one uint8 buffer, each starting on 256 bytes."""
+    off, spans = 0, []
+    for a in arrays:
+        spans.append(off)
+        off += (a.nbytes + 255) // 256 * 256
+    buf = np.zeros(off, np.uint8)
+    for a, o in zip(arrays, spans):
+        buf[o:o + a.nbytes] = np.ascontiguousarray(a).view(np.uint8).ravel()
+    return buf
+
+
+def _views(buf, arrays):
+    """Typed views of a packed device buffer (layout of _pack_host)."""
+    import torch
+    tmap = {np.dtype(np.int16): torch.int16, np.dtype(np.int32): torch.int32, np.dtype(np.float32): torch.float32}
+    out, off = [], 0
+    for a in arrays:
+        out.append(buf[off:off + a.nbytes].view(tmap[a.dtype]).view(a.shape))
+        off += (a.nbytes + 255) // 256 * 256
+    return out
 
 
 def traffic_record(kernel, workload, layout):

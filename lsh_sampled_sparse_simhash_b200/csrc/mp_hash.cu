@@ -11,11 +11,14 @@
 
 namespace mp {
 
+constexpr int kAppendCols = 64;  // hyperplane columns per append block (4 lanes each)
+
 // --------------------------------------------------------------- append ----
-// grid (ceil(L / TB), B * Hkv), 256 threads: thread = one hyperplane column of a
-// block of TB = 256 / K whole tables, projection = fp32 sum of exact bf16
-// products in ascending j (bits can differ from the tensor-core hash only where
-// the projection is within fp32 rounding of zero).
+// grid (ceil(L / TB), B * Hkv), 256 threads: 4 lanes per hyperplane column
+// of a block of TB = 64 / K whole tables; each lane sums 32 exact bf16
+// products in fp32 and two shuffles add the quarters (bits can differ from
+// the tensor-core hash only where the projection is within fp32 rounding of
+// zero).
 __global__ void __launch_bounds__(256) append_kernel(Shape s, const uint16_t *__restrict__ k_new,
                                                      const uint16_t *__restrict__ v_new,
                                                      const uint16_t *__restrict__ W, uint16_t *kc, uint16_t *vc,
@@ -23,7 +26,7 @@ __global__ void __launch_bounds__(256) append_kernel(Shape s, const uint16_t *__
                                                      int32_t *status)
 {
     __shared__ float xs[kHeadDim];
-    __shared__ uint8_t bits[256];
+    __shared__ uint8_t bits[kAppendCols];
     const int tid = threadIdx.x;
     const int unit = blockIdx.y;
     const int b = unit / s.Hkv;
@@ -42,37 +45,40 @@ __global__ void __launch_bounds__(256) append_kernel(Shape s, const uint16_t *__
     }
     if (tid < kHeadDim) xs[tid] = bf16_to_f32(kn[tid]);
     __syncthreads();
-    const int TB = 256 / s.K;
+    const int TB = kAppendCols / s.K;
     const int l0 = blockIdx.x * TB;
-    const int c = l0 * s.K + tid;
-    const bool valid = tid < TB * s.K && c < s.LK;
-    bool bit = false;
+    const int col = tid >> 2, part = tid & 3;  // column of the block, quarter of the dims
+    const int c = l0 * s.K + col;
+    const bool valid = col < TB * s.K && c < s.LK;
+    float dot = 0.f;
     if (valid) {
-        const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)c * kHeadDim);
-        float dot = 0.f;
+        const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)c * kHeadDim + part * 32);
+        const float *xp = xs + part * 32;
 #pragma unroll
-        for (int j8 = 0; j8 < kHeadDim / 8; j8++) {
+        for (int j8 = 0; j8 < 4; j8++) {
             const uint4 w = __ldg(wr + j8);
-            dot = fmaf(xs[j8 * 8 + 0], bf16_lo(w.x), dot);
-            dot = fmaf(xs[j8 * 8 + 1], bf16_hi(w.x), dot);
-            dot = fmaf(xs[j8 * 8 + 2], bf16_lo(w.y), dot);
-            dot = fmaf(xs[j8 * 8 + 3], bf16_hi(w.y), dot);
-            dot = fmaf(xs[j8 * 8 + 4], bf16_lo(w.z), dot);
-            dot = fmaf(xs[j8 * 8 + 5], bf16_hi(w.z), dot);
-            dot = fmaf(xs[j8 * 8 + 6], bf16_lo(w.w), dot);
-            dot = fmaf(xs[j8 * 8 + 7], bf16_hi(w.w), dot);
+            dot = fmaf(xp[j8 * 8 + 0], bf16_lo(w.x), dot);
+            dot = fmaf(xp[j8 * 8 + 1], bf16_hi(w.x), dot);
+            dot = fmaf(xp[j8 * 8 + 2], bf16_lo(w.y), dot);
+            dot = fmaf(xp[j8 * 8 + 3], bf16_hi(w.y), dot);
+            dot = fmaf(xp[j8 * 8 + 4], bf16_lo(w.z), dot);
+            dot = fmaf(xp[j8 * 8 + 5], bf16_hi(w.z), dot);
+            dot = fmaf(xp[j8 * 8 + 6], bf16_lo(w.w), dot);
+            dot = fmaf(xp[j8 * 8 + 7], bf16_hi(w.w), dot);
         }
-        bit = dot > 0.f;
     }
+    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+    const bool bit = valid && dot > 0.f;
     if (!s.planes) {
-        bits[tid] = bit;
+        if (part == 0) bits[col] = bit;
         __syncthreads();
         if (tid < TB && l0 + tid < s.L) {
             unsigned code = 0;
             for (int bb = 0; bb < 8; bb++) code |= (unsigned)bits[tid * 8 + bb] << bb;
             static_cast<uint8_t *>(codes)[((size_t)unit * s.L + l0 + tid) * s.Ncap + pos] = (uint8_t)code;
         }
-    } else if (valid) {
+    } else if (valid && part == 0) {
         const int l = c / s.K, bb = c - l * s.K;
         unsigned int *word =
             static_cast<unsigned int *>(codes) + (((size_t)unit * s.L + l) * (s.Ncap >> 5) + (pos >> 5)) * s.K + bb;
@@ -97,7 +103,7 @@ cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t 
                           uint16_t *kc, uint16_t *vc, void *codes, int32_t *seq_lens, int32_t *status,
                           cudaStream_t st)
 {
-    const int TB = 256 / s.K;
+    const int TB = kAppendCols / s.K;
     dim3 grid((s.L + TB - 1) / TB, s.B * s.Hkv);
     cudaError_t e = launch_pdl(append_kernel, grid, dim3(256), 0, st, s, k_new, v_new, W, kc, vc, codes,
                                (const int32_t *)seq_lens, status);
