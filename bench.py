@@ -48,6 +48,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--code-layout", default=None, choices=["auto", "bytes", "planes"],
                    help="key-code layout (default: the workload's, i.e. bytes for K=8, planes for K=10)")
+    p.add_argument("--no-graph", action="store_true",
+                   help="launch every timed step eagerly instead of replaying a captured CUDA graph")
     p.add_argument("--decode-path", default="auto", choices=["auto", "split", "fused"],
                    help="decode kernels: auto, split (scan then attention) or fused (one kernel; bit planes)")
     return p.parse_args()
@@ -174,6 +176,7 @@ class Bench:
         self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
         self.tokens = step_tokens(inp["seq_lens"] + 1)
         self.path = {"auto": mp.MP_PATH_AUTO, "split": mp.MP_PATH_SPLIT, "fused": mp.MP_PATH_FUSED}[path]
+        self.graph_error = None
         fused = self.path == mp.MP_PATH_FUSED
         # hash 1, append 2, decode: qhash + (scan, attention | fused) + merge
         self.launches_per_step = 3 + (3 if fused else 4)
@@ -224,16 +227,39 @@ class Bench:
                 self.step()
             torch.cuda.synchronize()
 
-    def run_timed(self, ev):
+    def capture(self):
+        """Captures one step (hash, append, decode: every kernel of the step,
+        programmatic launch edges included) in a CUDA graph; None if capture
+        is not possible here."""
+        torch = self.torch
+        try:
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.hash()
+                self.append()
+                self.decode()
+            torch.cuda.synchronize()
+            return g
+        except Exception as exc:  # report the eager fallback in the JSON line
+            self.graph_error = f"{type(exc).__name__}: {exc}"
+            torch.cuda.synchronize()
+            return None
+
+    def run_timed(self, ev, graph=None):
         """K steps, one event pair per step (no events between the calls, which
-        would serialise the programmatic launch chain)."""
+        would serialise the programmatic launch chain); with a graph, each step
+        is one replay of the captured hash + append + decode."""
         for e in ev:
             self.flush.zero_()
             self.lens.copy_(self.lens0, non_blocking=True)
             e[0].record()
-            self.hash()
-            self.append()
-            self.decode()
+            if graph is not None:
+                graph.replay()
+            else:
+                self.hash()
+                self.append()
+                self.decode()
             e[1].record()
 
     def run_breakdown(self, ev):
@@ -294,7 +320,7 @@ class Bench:
                     overlap=(t_dec + t_hash) / t_both,
                     hash_rows_per_s_concurrent=rows / (t_both / 1e3))
 
-    def run_e2e(self, steps, warmup):
+    def run_e2e(self, steps, warmup, use_graph=True):
         """Public API with host buffers: per step, one H2D copy of the step's
         inputs (q, k_new, v_new, lengths, packed) from pinned memory, the
         three calls, and one D2H copy of out / lse / n_sampled (packed) into
@@ -304,21 +330,39 @@ class Bench:
         hout = torch.empty(self.out_dev.shape, dtype=torch.uint8).pin_memory()
         h2d = hin.numel()
         d2h = hout.numel()
-        times = []
-        for i in range(warmup + steps):
-            self.flush.zero_()
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s.record()
+
+        def one_step():
             self.in_dev.copy_(hin, non_blocking=True)
             self.hash()
             self.append()
             self.decode()
             hout.copy_(self.out_dev, non_blocking=True)
+
+        graph = None
+        if use_graph:  # the copies are captured too: every replay moves the step's bytes
+            try:
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    one_step()
+                torch.cuda.synchronize()
+            except Exception:
+                graph = None
+                torch.cuda.synchronize()
+        times = []
+        for i in range(warmup + steps):
+            self.flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            if graph is not None:
+                graph.replay()
+            else:
+                one_step()
             e.record()
             e.synchronize()
             if i >= warmup:
                 times.append(s.elapsed_time(e))
-        return statistics.mean(times), h2d, d2h
+        return statistics.mean(times), h2d, d2h, graph is not None
 
 
 def _pack_host(arrays):
@@ -481,12 +525,17 @@ def main():
             dist.barrier()
 
     ev = bench.timed(args.steps, args.warmup)
+    graph = None if args.no_graph else bench.capture()
+    for _ in range(3 if graph is not None else 0):  # warm replays
+        bench.flush.zero_()
+        bench.lens.copy_(bench.lens0, non_blocking=True)
+        graph.replay()
     clocks = ClockSampler(local if world > 1 else 0)
     clocks.start()
     bench.preroll(0.5)  # untimed steps so the sampler sees the clocks under this load
     barrier()
     torch.cuda.synchronize()
-    bench.run_timed(ev)
+    bench.run_timed(ev, graph)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
@@ -502,12 +551,13 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e2e_ms, h2d, d2h = bench.run_e2e(min(args.steps, 20), 3)
+        e2e_ms, h2d, d2h, e2e_graph = bench.run_e2e(min(args.steps, 20), 3, not args.no_graph)
         t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
         if world > 1:
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e = dict(value=bench.tokens * world / (t.item() / 1e3), unit="tokens/s", h2d_bytes_per_step=h2d,
-                   d2h_bytes_per_step=d2h, ms_per_step=t.item())
+                   d2h_bytes_per_step=d2h, ms_per_step=t.item(),
+                   launch="cuda-graph replay (copies included)" if e2e_graph else "eager launches")
 
     if rank == 0:
         peaks = load_peaks()
@@ -539,7 +589,10 @@ def main():
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype="bf16-in/fp32-acc", data="synthetic",
-                    config=dict(config_of(w), decode_path=args.decode_path), roofline=roofline,
+                    config=dict(config_of(w), decode_path=args.decode_path,
+                                launch="cuda-graph replay per step" if graph is not None else
+                                "eager launches" + (f" ({bench.graph_error})" if bench.graph_error else "")),
+                    roofline=roofline,
                     breakdown=dict(hash_ms=hash_ms, append_ms=append_ms, decode_ms=decode_ms,
                                    hash_roofline=hash_roof, decode_roofline=dec_roof,
                                    decode_only_tokens_per_s=bench.tokens / (decode_ms / 1e3),
