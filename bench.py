@@ -401,11 +401,38 @@ def traffic_record(kernel, workload, layout):
     rec = recs.get(f"{kernel}@{workload}:{layout}")
     if not rec:
         return None
-    import hashlib
     src = os.path.join(ROOT, rec["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
+    if not os.path.exists(src) or code_fingerprint(src) != rec["code_sha256"]:
         return None
     return rec["bytes_per_launch"]
+
+
+def code_fingerprint(path):
+    """sha256 of a C/CUDA source with its comments removed and whitespace
+    collapsed: it changes when the code changes, not when a comment does."""
+    import hashlib
+    text = open(path).read()
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":  # string or char literal, copied through verbatim
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    code = " ".join("".join(out).split())
+    return hashlib.sha256(code.encode()).hexdigest()
 
 
 # ------------------------------------------------------ oracle (CPU) ----

@@ -1,19 +1,24 @@
 // LSH-sampled decode attention for one layer (MagicPIG, Chen et al. 2024), sm_100a.
 //
-// Four kernels run back to back on one stream for every mp_decode_attend call:
+// Every mp_decode_attend call runs these kernels back to back on one stream
+// (programmatic dependent launch between them):
 //   qhash   SimHash codes of the query heads (fp32 projection of bf16 q onto W).
-//   scan    streams the table-major key codes of a context chunk with 16-byte
-//           loads, counts per token and per query head the tables whose code
-//           equals the query's (saturating at 2, bit-sliced), excludes the exact
-//           set D and compacts the sampled tokens (token id | head mask) with a
-//           warp-ballot / block prefix sum.
-//   attend  gathers the compacted K/V rows of a chunk into a cp.async shared
-//           memory ring, computes q.k for all query heads of the GQA group from
-//           one row load (bf16 mma.sync, fp32 accumulate), applies the -log u
-//           importance correction and runs an online softmax; one extra split
-//           per (b, kv head) handles D exactly (weight exp(s), no correction).
+//   scan    counts, per token and query head, the tables whose code equals the
+//           query's (bit-sliced counters saturating at 2), excludes the exact
+//           set D and compacts the sampled tokens (token id | head mask) in
+//           token order.  Byte codes: scan_k8_kernel, 16-byte streaming loads
+//           and a zero-byte test per 4 tokens.  Bit planes: scan_planes_kernel,
+//           persistent, 3-D TMA copies of 8 tables per stage into a ring,
+//           32 tokens per logic operation.
+//   attend  gathers the compacted K/V rows into a cp.async shared-memory
+//           ring, computes q.k for all query heads of the GQA group from one
+//           row load (bf16 mma.sync, fp32 accumulate), applies the -log u
+//           importance correction and runs an online softmax in base 2; one
+//           extra split per (b, kv head) handles D exactly (weight exp(s)).
 //   merge   log-sum-exp merge of the per-split partials into out / lse, plus
 //           n_sampled.
+// With bit planes the scan and the attention can instead run as one kernel,
+// fused_planes_kernel (opt-in, MP_PATH_FUSED).
 #include <math.h>
 
 #include <algorithm>

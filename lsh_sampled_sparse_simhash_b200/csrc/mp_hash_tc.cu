@@ -18,9 +18,12 @@
 //   warps 4..19 epilogue, four groups of four warps, each group one 64-column
 //               slice of every column tile: tcgen05.ld 32x32b (thread = key
 //               row, registers = columns), release of the accumulator, then
-//               sign test, pack, store off the MMA's critical path.
-//               K = 8: one byte per (table, token); K = 10: one warp ballot
-//               per column gives the 32-token bit-plane word.
+//               sign test, pack, store off the MMA's critical path.  Each
+//               thread packs 32 columns of its row into a word (saturating
+//               multiplies and a paired f32x2 FMA chain); byte codes then
+//               swap bytes within lane quads (4 tokens of one table per 32-bit
+//               store), bit planes transpose the 32x32 bit matrix across the
+//               warp (one plane word per lane).
 //
 // Column groups: W has L*K rows (hyperplanes); a group of at most 640 rows
 // (608 for K = 8, L = 75) stays resident; K = 10, L = 150 uses 3 groups of
