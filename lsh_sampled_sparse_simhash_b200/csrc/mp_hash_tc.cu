@@ -19,8 +19,9 @@
 //               slice of every column tile: tcgen05.ld 32x32b (thread = key
 //               row, registers = columns), release of the accumulator, then
 //               sign test, pack, store off the MMA's critical path.  Each
-//               thread packs 32 columns of its row into a word (saturating
-//               multiplies and a paired f32x2 FMA chain); byte codes then
+//               thread packs the sign bits of 32 columns of its row into a
+//               word (one funnel shift per column; the MMA negates the keys,
+//               so a set sign bit means a positive projection); byte codes then
 //               swap bytes within lane quads (4 tokens of one table per 32-bit
 //               store), bit planes transpose the 32x32 bit matrix across the
 //               warp (one plane word per lane).
@@ -120,10 +121,15 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// kind::f16 instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128.
+// kind::f16 instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128,
+// A (the keys) negated (bit 13).  The accumulator is then -(k . w_c), computed
+// exactly like k . w_c up to the sign (round-to-nearest is symmetric), and its
+// sign bit is 1 iff k . w_c > 0: a projection that cancels to zero gives +0,
+// sign 0, as the strict rule wants.
 __device__ __forceinline__ uint32_t idesc_bf16(int n)
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+    return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 13) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(kBM >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum)
@@ -153,46 +159,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// [x > 0] as 1.0f / 0.0f in one FMA-pipe instruction: a saturating product
-// by 2^126 sends every positive normal to 1 and zero, negatives and NaN to 0.
-// Flush-to-zero makes a subnormal projection (|x| < 2^-126) count as zero.
-__device__ __forceinline__ float positive_unit(uint32_t bits)
+// 32-bit word whose bit c is the sign bit of v[c]: with the keys negated in
+// the MMA (idesc_bf16), that bit is [k . w_c > 0].  One funnel shift per
+// column moves the sign into the running word; two independent chains of 16
+// columns halve the dependent latency.
+__device__ __forceinline__ uint32_t pack_signs32(const uint32_t *v)
 {
-    float r;
-    asm("mul.rn.ftz.sat.f32 %0, %1, 0f7E800000;" : "=f"(r) : "f"(__uint_as_float(bits)));
-    return r;
-}
-
-__device__ __forceinline__ uint64_t pair2(float lo, float hi)
-{
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
-// 16-bit integer whose bit c is [v[c] > 0], built on the FMA pipe: the sum
-// sum_c [v_c > 0] 2^c is exact in fp32.  The even and the odd bits are the two
-// lanes of one paired (f32x2) FMA chain, E = sum_i u_2i 4^i and
-// O = sum_i u_2i+1 4^i, which halves the chain's length; then 2 O + E, and
-// adding 2^23 puts the integer in the low bits of the float's bit pattern.
-__device__ __forceinline__ uint32_t pack_positive16(const uint32_t *v)
-{
-    uint64_t acc = pair2(positive_unit(v[14]), positive_unit(v[15]));
-    const uint64_t four = 0x4080000040800000ull;  // {4.0f, 4.0f}
+    uint32_t lo = 0u, hi = 0u;
 #pragma unroll
-    for (int i = 6; i >= 0; i--) {
-        const uint64_t u = pair2(positive_unit(v[2 * i]), positive_unit(v[2 * i + 1]));
-        asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(acc) : "l"(four), "l"(u));
+    for (int c = 15; c >= 0; c--) {
+        lo = __funnelshift_l(v[c], lo, 1);  // (lo << 1) | (v[c] >> 31)
+        hi = __funnelshift_l(v[16 + c], hi, 1);
     }
-    float e, o;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(e), "=f"(o) : "l"(acc));
-    return __float_as_uint(fmaf(o, 2.f, e) + 8388608.f);
-}
-
-// 32-bit word whose bit c is [v[c] > 0].
-__device__ __forceinline__ uint32_t pack_positive32(const uint32_t *v)
-{
-    return __byte_perm(pack_positive16(v), pack_positive16(v + 16), 0x5410);
+    return __byte_perm(lo, hi, 0x5410);
 }
 
 // Within each group of 4 lanes, transposes the 4x4 byte matrix whose row r
@@ -340,13 +319,14 @@ __device__ __forceinline__ void epilogue_slice(const Params &p, const TileDst &t
     for (int q = 0; q < NCH; q++) tmem_ld32(ta + 32 * q, v[q]);
     tmem_wait_ld();
     tc_fence_before();
-    mbar_arrive(empty_bar);  // values are in registers: free the accumulator
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar);  // the warp's values are in registers: free the accumulator
 #pragma unroll
     for (int q = 0; q < NCH; q++) {
         const int c32 = col0 + 32 * q;  // first global column of these 32
         if (!PLANES) {
             // 4 table bytes of this token -> 4 tokens of one table per lane
-            const uint32_t w = quad_transpose(pack_positive32(v[q]), sel1, sel2);
+            const uint32_t w = quad_transpose(pack_signs32(v[q]), sel1, sel2);
             const int l = (c32 >> 3) + (lane & 3);
             if (l < s.L) {
                 uint8_t *dst = td.bytes + (size_t)l * s.Ncap;
@@ -358,7 +338,7 @@ __device__ __forceinline__ void epilogue_slice(const Params &p, const TileDst &t
             }
         } else {
             // row word (bit c = column c32 + c) -> column word (bit t = token t)
-            const uint32_t rw = td.valid ? pack_positive32(v[q]) : 0u;
+            const uint32_t rw = td.valid ? pack_signs32(v[q]) : 0u;
             const uint32_t mine = warp_transpose32(rw, keep, rot);
             const uint32_t c = (uint32_t)(c32 + lane);
             if (td.warp_live && c < (uint32_t)s.LK) {
@@ -418,7 +398,8 @@ __device__ __forceinline__ void epilogue(const Params &p, const int *lens_sh, ui
                 epilogue_slice<PLANES, 1>(p, td, ta, empty, c0 + n0 + ch, lane, sel1, sel2, keep, rot);
             } else {
                 tc_fence_before();
-                mbar_arrive(empty);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty);
             }
         }
     }
@@ -456,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < kAccBufs; b++) {
             mbar_init(tmem_full(b), 1);
-            mbar_init(tmem_empty(b), 128 * kEpiGroups);
+            mbar_init(tmem_empty(b), 4 * kEpiGroups);  // one arrival per epilogue warp
         }
         static_assert(kAccBufs * kAccCols == 512, "TMEM holds 512 columns");
         mbar_init(w_full, 1);
