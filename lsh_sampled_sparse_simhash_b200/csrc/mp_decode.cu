@@ -126,41 +126,6 @@ __device__ __forceinline__ int clamp_len(const int32_t *seq_lens, int b, int max
     return n;
 }
 
-// Block-wide exclusive prefix sum over blockDim.x <= 1024 threads.
-__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int &total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = (blockDim.x + 31) >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int off = 0;
-    total = 0;
-    for (int w = 0; w < nwarp; w++) {
-        int t = warp_tot[w];
-        if (w < warp) off += t;
-        total += t;
-    }
-    return off + incl - v;
-}
-
-__device__ __forceinline__ int block_sum(int v, int *scratch)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = (blockDim.x + 31) >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    __syncthreads();
-    if (lane == 0) scratch[warp] = v;
-    __syncthreads();
-    int t = 0;
-    for (int w = 0; w < nwarp; w++) t += scratch[w];
-    return t;
-}
-
 // 16-byte read-only load that allocates in L1 (the plane scan touches each
 // 32-byte sector with two consecutive loads).
 __device__ __forceinline__ uint4 ld_cached_16(const void *p)
@@ -208,65 +173,53 @@ __device__ __forceinline__ uint32_t range_mask(int base, int lo, int hi, int wid
     return upto & ~((1u << a) - 1u);
 }
 
-// Compacts one thread's sampled tokens.  hm[g][w] bit i = token t0 + 32 w + i
-// is in S_g (NW words of WIDTH tokens; tokens outside [lo, hi) are masked).
-// Entries keep token order: thread-major, then word, then bit.
-template <int G, int NW, int WIDTH>
-__device__ __forceinline__ void compact_and_store(const Shape &s, int unit, int chunk, int nchunk,
-                                                  int chunk_tokens, int t0, int N, int lo, int hi,
-                                                  uint32_t (&hm)[G][NW], bool owner, const ScanOut &o,
-                                                  int *smem_scratch)
+// Candidate list of one chunk by one warp (lane = the WIDTH tokens at t0):
+// hm[g] bit i = token t0 + i is in S_g; tokens outside [lo, hi) are masked.
+// Entries keep token order (lane, then bit); CHUNK = tokens per list.
+template <int G, int WIDTH, int CHUNK>
+__device__ __forceinline__ void compact_warp(const Shape &s, int unit, int chunk, int nchunk, int t0, int N, int lo,
+                                             int hi, uint32_t (&hm)[G], const ScanOut &o, int lane)
 {
-    uint32_t any[NW];
-    int mine = 0;
-#pragma unroll
-    for (int w = 0; w < NW; w++) {
-        const uint32_t v = range_mask(t0 + 32 * w, lo, hi, WIDTH);
-        any[w] = 0u;
-#pragma unroll
-        for (int g = 0; g < G; g++) {
-            hm[g][w] &= v;
-            any[w] |= hm[g][w];
-        }
-        mine += __popc(any[w]);
-    }
-    int total;
-    int off = block_exclusive_scan(mine, smem_scratch, total);
-    uint32_t *dst = o.cand + ((size_t)unit * nchunk + chunk) * chunk_tokens;
-#pragma unroll
-    for (int w = 0; w < NW; w++) {
-        uint32_t m = any[w];
-        while (m) {
-            const int bit = __ffs(m) - 1;
-            m &= m - 1u;
-            uint32_t heads = 0u;
-#pragma unroll
-            for (int g = 0; g < G; g++) heads |= ((hm[g][w] >> bit) & 1u) << g;
-            dst[off++] = (uint32_t)(t0 + 32 * w + bit) | (heads << 24);
-        }
-    }
-    int32_t *cnt = o.cnt + ((size_t)unit * nchunk + chunk) * 16;
-    if (threadIdx.x == 0) cnt[0] = total;
+    const uint32_t v = range_mask(t0, lo, hi, WIDTH);
+    uint32_t any = 0u;
 #pragma unroll
     for (int g = 0; g < G; g++) {
-        int c = 0;
-#pragma unroll
-        for (int w = 0; w < NW; w++) c += __popc(hm[g][w]);
-        c = block_sum(c, smem_scratch + 32);
-        if (threadIdx.x == 0) cnt[1 + g] = c;
+        hm[g] &= v;
+        any |= hm[g];
     }
-    if (o.member_out && owner) {
+    const int mine = __popc(any);
+    int incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += t;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int off = incl - mine;
+    uint32_t *dst = o.cand + ((size_t)unit * nchunk + chunk) * CHUNK;
+    while (any) {
+        const int bit = __ffs(any) - 1;
+        any &= any - 1u;
+        uint32_t heads = 0u;
+#pragma unroll
+        for (int g = 0; g < G; g++) heads |= ((hm[g] >> bit) & 1u) << g;
+        dst[off++] = (uint32_t)(t0 + bit) | (heads << 24);
+    }
+    int32_t *cnt = o.cnt + ((size_t)unit * nchunk + chunk) * 16;
+    if (lane == 0) cnt[0] = total;
+#pragma unroll
+    for (int g = 0; g < G; g++) {
+        int c = __popc(hm[g]);
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) c += __shfl_xor_sync(0xffffffffu, c, d);
+        if (lane == 0) cnt[1 + g] = c;
+    }
+    if (o.member_out) {
         const int b = unit / s.Hkv, kvh = unit % s.Hkv;
+        for (int i = 0; i < WIDTH && t0 + i < N; i++)
 #pragma unroll
-        for (int w = 0; w < NW; w++) {
-            for (int i = 0; i < WIDTH; i++) {
-                const int tok = t0 + 32 * w + i;
-                if (tok >= N) break;
-#pragma unroll
-                for (int g = 0; g < G; g++)
-                    o.member_out[((size_t)b * s.Hq + kvh * G + g) * s.Ncap + tok] = (hm[g][w] >> i) & 1u;
-            }
-        }
+            for (int g = 0; g < G; g++)
+                o.member_out[((size_t)b * s.Hq + kvh * G + g) * s.Ncap + t0 + i] = (hm[g] >> i) & 1u;
     }
 }
 
@@ -314,7 +267,8 @@ __device__ __forceinline__ void combine_splits(uint32_t (&s1)[G][NW], uint32_t (
 // matches.  Zero bytes are found exactly with ((x & 0x7f..) + 0x7f..) | x,
 // whose byte top bit is 1 iff the byte is non-zero (the add runs on the FMA
 // pipe).  Two bit-sliced counters (seen >= 1, seen >= 2) live in the byte top
-// bits.
+// bits.  Warp 0 folds the other splits' counters and compacts the chunk's
+// candidates alone (warp-level scan, no block barrier); warps 1..7 exit.
 template <int G>
 __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
     Shape s, const uint8_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
@@ -323,8 +277,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
     extern __shared__ uint32_t dyn[];  // rep [L][G] (query code in 4 bytes), then split partials
     uint32_t *rep = dyn;
     uint32_t *part = dyn + ((s.L * G + 3) & ~3);
-    __shared__ int scratch[64];
     constexpr int TS = kSplitsK8, TG = kScanThreads / TS, NB = 8;
+    static_assert(TG == 32, "split ts = warp ts, token group tg = lane");
     const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
     const int unit = blockIdx.y, chunk = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
@@ -374,18 +328,19 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
         }
     }
     combine_splits<G, 4, TS>(s1, s2, part, ts, tg);
-    // Per-head 16-bit token masks from the byte top bits of the >= 2 counter.
-    uint32_t hm[G][1];
+    if (ts != 0) return;  // warp 0 (ts == 0, lane = tg) now holds the chunk's counters
+    // Per-head 16-bit token masks from the byte top bits of the >= 2 counter:
+    // the four top bits of a word, moved to bits 24..27 by one multiply.
+    uint32_t hm[G];
 #pragma unroll
     for (int g = 0; g < G; g++) {
         uint32_t m = 0u;
 #pragma unroll
-        for (int i = 0; i < 16; i++) m |= ((s2[g][i >> 2] >> (8 * (i & 3) + 7)) & 1u) << i;
-        hm[g][0] = ts == 0 ? m : 0u;
+        for (int j = 0; j < 4; j++) m |= ((((s2[g][j] >> 7) & 0x01010101u) * 0x01020408u) >> 24) << (4 * j);
+        hm[g] = m;
     }
     // Tokens eligible for S: [sink, N - window) and below N.
-    compact_and_store<G, 1, 16>(s, unit, chunk, nchunk, kChunkBytes, t0, N, s.sink, min(N - s.window, N), hm,
-                                ts == 0, o, scratch);
+    compact_warp<G, 16, kChunkBytes>(s, unit, chunk, nchunk, t0, N, s.sink, min(N - s.window, N), hm, o, tg);
 }
 
 // ------------------------------------------------------ scan, bit planes ----
@@ -458,55 +413,6 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, i
 __device__ __forceinline__ void consumer_barrier() { asm volatile("bar.sync 1, %0;" ::"n"(kScanThreads) : "memory"); }
 __device__ __forceinline__ void bar_sync_all(int id) { asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kScanThreads + 32) : "memory"); }
 __device__ __forceinline__ void bar_arrive_all(int id) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kScanThreads + 32) : "memory"); }
-
-// Candidate list of one item by one warp (lane = 32-token word at t0):
-// hm[g] bit i = token t0 + i is in S_g.  Entries keep token order.
-template <int G>
-__device__ __forceinline__ void compact_warp(const Shape &s, int unit, int chunk, int nchunk, int t0, int N, int lo,
-                                             int hi, uint32_t (&hm)[G], const ScanOut &o, int lane)
-{
-    const uint32_t v = range_mask(t0, lo, hi, 32);
-    uint32_t any = 0u;
-#pragma unroll
-    for (int g = 0; g < G; g++) {
-        hm[g] &= v;
-        any |= hm[g];
-    }
-    const int mine = __popc(any);
-    int incl = mine;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += t;
-    }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    int off = incl - mine;
-    uint32_t *dst = o.cand + ((size_t)unit * nchunk + chunk) * kChunkPlanes;
-    while (any) {
-        const int bit = __ffs(any) - 1;
-        any &= any - 1u;
-        uint32_t heads = 0u;
-#pragma unroll
-        for (int g = 0; g < G; g++) heads |= ((hm[g] >> bit) & 1u) << g;
-        dst[off++] = (uint32_t)(t0 + bit) | (heads << 24);
-    }
-    int32_t *cnt = o.cnt + ((size_t)unit * nchunk + chunk) * 16;
-    if (lane == 0) cnt[0] = total;
-#pragma unroll
-    for (int g = 0; g < G; g++) {
-        int c = __popc(hm[g]);
-#pragma unroll
-        for (int d = 16; d > 0; d >>= 1) c += __shfl_xor_sync(0xffffffffu, c, d);
-        if (lane == 0) cnt[1 + g] = c;
-    }
-    if (o.member_out) {
-        const int b = unit / s.Hkv, kvh = unit % s.Hkv;
-        for (int i = 0; i < 32 && t0 + i < N; i++)
-#pragma unroll
-            for (int g = 0; g < G; g++)
-                o.member_out[((size_t)b * s.Hq + kvh * G + g) * s.Ncap + t0 + i] = (hm[g] >> i) & 1u;
-    }
-}
 
 template <int G, int KB>
 __global__ void __launch_bounds__(kScanThreads + 32) scan_planes_kernel(
@@ -611,7 +517,7 @@ __global__ void __launch_bounds__(kScanThreads + 32) scan_planes_kernel(
                 }
                 if (ci + 1 < count) bar_arrive_all(3);  // item ci is read: the consumers may post item ci + 1
                 // tokens eligible for S: [sink, N - window) and below N
-                compact_warp<G>(s, cur.unit(s), cur.chunk, nchunk, cur.chunk * kChunkPlanes + lane * 32, cur.N,
+                compact_warp<G, 32, kChunkPlanes>(s, cur.unit(s), cur.chunk, nchunk, cur.chunk * kChunkPlanes + lane * 32, cur.N,
                                 s.sink, min(cur.N - s.window, cur.N), s2, o, lane);
                 cur.next(s, seq_lens, max_len);
             }
@@ -1604,10 +1510,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_planes_kernel(const __
 }
 
 // ----------------------------------------------------------------- merge ----
-// One block of 128 threads per (b, q head).  Pass 1: the global maximum of
-// the split maxima (threads stride over splits).  Pass 2: warp w folds splits
-// w, w + 4, ... with exp(m_j - M) weights (lane = 4 output dims, independent
-// loads unrolled), then the four warps are summed in shared memory.
+// One block of 128 threads per (b, q head).  Warp w folds splits w, w + 4,
+// ... (lane = 4 output dims) with a running maximum, rescaling its sums when
+// the maximum moves, so all loads go out in one pass (unrolled); the four
+// warps' (m, l, acc) are then combined in shared memory.
 template <int G>
 __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t *__restrict__ seq_lens,
                                                          int max_len, int nchunk, int span, int subs,
@@ -1635,54 +1541,61 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
     auto split_index = [&](int j) { return j < nsp ? j : dsp; };  // j in [0, nsp]
     const int last = has_d ? nsp : nsp - 1;                       // splits 0..last are read
 
-    // pass 1: M = max over live splits and D; sampled count
-    float m = -INFINITY;
+    // n_sampled: the chunks' per-head counts
     int ns = 0;
-    for (int j = tid; j <= last; j += blockDim.x) m = fmaxf(m, pm[base + split_index(j)]);
     for (int j = tid; j < nch; j += blockDim.x) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        ns += __shfl_xor_sync(0xffffffffu, ns, o);
+    // each warp folds splits warp, warp + 4, ... with a running maximum, so
+    // every load is issued in one pass (no separate pass for the maximum)
+    float m = -INFINITY, Ls = 0.f;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int j = warp; j <= last; j += 4) {
+        const size_t sp = base + split_index(j);
+        const float mj = pm[sp];
+        const float lj = pl[sp];
+        const float4 aj = reinterpret_cast<const float4 *>(pacc + sp * kHeadDim)[lane];
+        if (mj == -INFINITY) continue;  // an empty split (uniform across the warp)
+        if (mj > m) {
+            const float f = m == -INFINITY ? 0.f : fast_exp2(m - mj);
+            Ls *= f;
+            A.x *= f;
+            A.y *= f;
+            A.z *= f;
+            A.w *= f;
+            m = mj;
+        }
+        const float f = fast_exp2(mj - m);
+        Ls = fmaf(lj, f, Ls);
+        A.x = fmaf(aj.x, f, A.x);
+        A.y = fmaf(aj.y, f, A.y);
+        A.z = fmaf(aj.z, f, A.z);
+        A.w = fmaf(aj.w, f, A.w);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ns += __shfl_xor_sync(0xffffffffu, ns, o);
+    red_acc[warp][lane] = A;
     if (lane == 0) {
         red_m[warp] = m;
+        red_l[warp] = Ls;
         red_n[warp] = ns;
     }
     __syncthreads();
-    const float M = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
-
-    // pass 2
-    float Ls = 0.f;
-    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-#pragma unroll 4
-        for (int j = warp; j <= last; j += 4) {
-            const size_t sp = base + split_index(j);
-            const float mj = pm[sp];
-            const float f = mj == -INFINITY ? 0.f : fast_exp2(mj - M);
-            const float lj = pl[sp];
-            const float4 aj = reinterpret_cast<const float4 *>(pacc + sp * kHeadDim)[lane];
-            Ls = fmaf(lj, f, Ls);
-            A.x = fmaf(aj.x, f, A.x);
-            A.y = fmaf(aj.y, f, A.y);
-            A.z = fmaf(aj.z, f, A.z);
-            A.w = fmaf(aj.w, f, A.w);
-        }
-    }
-    red_acc[warp][lane] = A;
-    if (lane == 0) red_l[warp] = Ls;
-    __syncthreads();
     if (warp == 0) {
-        const float Lt = red_l[0] + red_l[1] + red_l[2] + red_l[3];
-        float4 o = red_acc[0][lane];
+        const float M = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+        float Lt = 0.f;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (M != -INFINITY) {
 #pragma unroll
-        for (int w = 1; w < 4; w++) {
-            const float4 t = red_acc[w][lane];
-            o.x += t.x;
-            o.y += t.y;
-            o.z += t.z;
-            o.w += t.w;
+            for (int w = 0; w < 4; w++) {
+                if (red_m[w] == -INFINITY) continue;
+                const float f = fast_exp2(red_m[w] - M);
+                const float4 t = red_acc[w][lane];
+                Lt = fmaf(red_l[w], f, Lt);
+                o.x = fmaf(t.x, f, o.x);
+                o.y = fmaf(t.y, f, o.y);
+                o.z = fmaf(t.z, f, o.z);
+                o.w = fmaf(t.w, f, o.w);
+            }
         }
         const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
         o.x *= inv;
