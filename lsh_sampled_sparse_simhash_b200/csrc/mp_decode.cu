@@ -62,23 +62,26 @@ __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__r
         }
         return;
     }
+    // this lane's W quarter row first: its load overlaps the q staging below
+    const int cl = tid >> 2, part = tid & 3;  // column within the block, quarter of the dims
+    const int c = l0 * s.K + cl;
+    const bool valid = cl < TB * s.K && c < s.LK;
+    uint4 w4[4];
+    if (valid) {
+        const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)c * kHeadDim + part * 32);
+#pragma unroll
+        for (int j = 0; j < 4; j++) w4[j] = __ldg(wr + j);
+    }
     for (int i = tid; i < G * kHeadDim; i += blockDim.x) {
         const int d = i % kHeadDim;
         qs[i / kHeadDim][d + (d >> 5)] = bf16_to_f32(q[(vec0 + i / kHeadDim) * kHeadDim + d]);
     }
     __syncthreads();
 
-    const int cl = tid >> 2, part = tid & 3;  // column within the block, quarter of the dims
-    const int c = l0 * s.K + cl;
-    const bool valid = cl < TB * s.K && c < s.LK;
     float acc[G];
 #pragma unroll
     for (int g = 0; g < G; g++) acc[g] = 0.f;
     if (valid) {
-        const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)c * kHeadDim + part * 32);
-        uint4 w4[4];
-#pragma unroll
-        for (int j = 0; j < 4; j++) w4[j] = __ldg(wr + j);
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             const uint32_t wv[4] = {w4[j].x, w4[j].y, w4[j].z, w4[j].w};
@@ -982,11 +985,26 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     const int unit = blockIdx.y, split = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
     grid_dependency_wait();
-    int N = a.seq_lens[b];
-    N = N < 0 ? 0 : (N > a.max_len ? a.max_len : N);
     const bool dsplit = split == a.ngroups * a.subs;
     const int grp = split / a.subs, sub = split % a.subs;
     const int c_begin = grp * a.span;
+    const uint32_t *lists = a.cand + ((size_t)unit * a.nchunk + c_begin) * a.chunk_tokens;
+    // A block that takes one chunk's whole list (span = subs = 1) reads the
+    // list's count and the first two tiles' entries together with the length:
+    // none of these loads waits for another (entries past the count are
+    // dropped below; they stay inside the chunk's list).
+    const bool direct = !dsplit && a.span == 1 && a.subs == 1;
+    int dcount = 0;
+    uint32_t pre0 = 0xFFFFFFFFu, pre1 = 0xFFFFFFFFu;
+    if (direct) {
+        if (tid == 0) dcount = a.cnt[((size_t)unit * a.nchunk + c_begin) * 16];
+        if (tid < kAttRows) {
+            pre0 = lists[tid];
+            pre1 = lists[kAttRows + tid];
+        }
+    }
+    int N = a.seq_lens[b];
+    N = N < 0 ? 0 : (N > a.max_len ? a.max_len : N);
     const int nch = (N + a.chunk_tokens - 1) / a.chunk_tokens;
     if (!dsplit && c_begin >= nch) return;
 
@@ -997,11 +1015,15 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     const int win0 = max(n_sink, N - s.window);
     const int nc = dsplit ? 0 : min(a.span, nch - c_begin);
     int nrows, e0 = 0;
-    const uint32_t *lists = a.cand + ((size_t)unit * a.nchunk + c_begin) * a.chunk_tokens;
     if (dsplit) {
         nrows = n_sink + (N - win0);
     } else {
-        if (warp == 0) {
+        if (direct) {
+            if (tid == 0) {
+                cpre[0] = 0;
+                cpre[1] = dcount;
+            }
+        } else if (warp == 0) {
             int run = 0;
             for (int j0 = 0; j0 < nc; j0 += 32) {
                 const int j = j0 + lane;
@@ -1067,8 +1089,13 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     };
 
     if (tid < kAttRows) {
-        if (ntiles > 0) ents[0][tid] = fetch1(0);
-        if (ntiles > 1) ents[1][tid] = fetch1(1);
+        if (direct) {
+            ents[0][tid] = tid < nrows ? pre0 : 0xFFFFFFFFu;
+            ents[1][tid] = kAttRows + tid < nrows ? pre1 : 0xFFFFFFFFu;
+        } else {
+            if (ntiles > 0) ents[0][tid] = fetch1(0);
+            if (ntiles > 1) ents[1][tid] = fetch1(1);
+        }
     }
     __syncthreads();  // entries of tiles 0 and 1, qinv
     if (ntiles > 0) issue(0, 0);
@@ -1510,6 +1537,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_planes_kernel(const __
 }
 
 // ----------------------------------------------------------------- merge ----
+constexpr int kMergeBatch = 8;  // splits per warp whose loads are in flight together
+
 // One block of 128 threads per (b, q head).  Warp w folds splits w, w + 4,
 // ... (lane = 4 output dims) with a running maximum, rescaling its sums when
 // the maximum moves, so all loads go out in one pass (unrolled); the four
@@ -1538,38 +1567,56 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
     const int nsp = ((nch + span - 1) / span) * subs;  // live chunk splits
     const int dsp = ngroups * subs;                     // the exact-set split (if has_d)
     const size_t base = (size_t)bh * (dsp + 1);
-    auto split_index = [&](int j) { return j < nsp ? j : dsp; };  // j in [0, nsp]
-    const int last = has_d ? nsp : nsp - 1;                       // splits 0..last are read
+    // split j in [0, dsp] holds a partial of this call iff j < nsp or it is
+    // the exact-set split; the loads below do not wait for that test (they
+    // stay inside the partial arrays), only the fold does
+    auto live = [&](int j) { return j < nsp || (has_d && j == dsp); };
 
     // n_sampled: the chunks' per-head counts
     int ns = 0;
     for (int j = tid; j < nch; j += blockDim.x) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
-    // each warp folds splits warp, warp + 4, ... with a running maximum, so
-    // every load is issued in one pass (no separate pass for the maximum)
+    // each warp folds splits warp, warp + 4, ... with a running maximum; the
+    // loads of kMergeBatch splits go out together before any of them is used
     float m = -INFINITY, Ls = 0.f;
     float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int j = warp; j <= last; j += 4) {
-        const size_t sp = base + split_index(j);
-        const float mj = pm[sp];
-        const float lj = pl[sp];
-        const float4 aj = reinterpret_cast<const float4 *>(pacc + sp * kHeadDim)[lane];
-        if (mj == -INFINITY) continue;  // an empty split (uniform across the warp)
-        if (mj > m) {
-            const float f = m == -INFINITY ? 0.f : fast_exp2(m - mj);
-            Ls *= f;
-            A.x *= f;
-            A.y *= f;
-            A.z *= f;
-            A.w *= f;
-            m = mj;
+    for (int j0 = warp; j0 <= dsp; j0 += 4 * kMergeBatch) {
+        float mj[kMergeBatch], lj[kMergeBatch];
+        float4 aj[kMergeBatch];
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; i++) {
+            const int j = j0 + 4 * i;
+            mj[i] = -INFINITY;
+            lj[i] = 0.f;
+            aj[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (j <= dsp) {
+                const size_t sp = base + j;
+                mj[i] = pm[sp];
+                lj[i] = pl[sp];
+                aj[i] = reinterpret_cast<const float4 *>(pacc + sp * kHeadDim)[lane];
+            }
         }
-        const float f = fast_exp2(mj - m);
-        Ls = fmaf(lj, f, Ls);
-        A.x = fmaf(aj.x, f, A.x);
-        A.y = fmaf(aj.y, f, A.y);
-        A.z = fmaf(aj.z, f, A.z);
-        A.w = fmaf(aj.w, f, A.w);
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; i++)
+            if (!live(j0 + 4 * i)) mj[i] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; i++) {
+            if (mj[i] == -INFINITY) continue;  // an empty or absent split (uniform across the warp)
+            if (mj[i] > m) {
+                const float f = m == -INFINITY ? 0.f : fast_exp2(m - mj[i]);
+                Ls *= f;
+                A.x *= f;
+                A.y *= f;
+                A.z *= f;
+                A.w *= f;
+                m = mj[i];
+            }
+            const float f = fast_exp2(mj[i] - m);
+            Ls = fmaf(lj[i], f, Ls);
+            A.x = fmaf(aj[i].x, f, A.x);
+            A.y = fmaf(aj[i].y, f, A.y);
+            A.z = fmaf(aj[i].z, f, A.z);
+            A.w = fmaf(aj[i].w, f, A.w);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ns += __shfl_xor_sync(0xffffffffu, ns, o);
