@@ -8,8 +8,9 @@
 // bits straight into the table-major code layout.
 //
 //   warp 0      TMA producer: the W column group (resident in shared memory,
-//               reloaded only when a CTA moves to the next group) and a
-//               2-stage ring of 128-row key tiles, 128B-swizzled.
+//               reloaded only when a CTA moves to the next group; one barrier
+//               per 256-column tile, so the first MMAs wait for one tile
+//               only) and a 2-stage ring of 128-row key tiles, 128B-swizzled.
 //   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, M = 128,
 //               N <= 256, K = 16, into one of two TMEM accumulators (N = 256
 //               keeps the operand traffic per flop within shared-memory
@@ -56,6 +57,7 @@ constexpr int kPrefetchAhead = 3;            // key tiles (of this block) kept i
 constexpr int kHalfBytes = kBM * 128;        // one 64-element (128 B) K half of a tile
 constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KB
 constexpr int kMaxGroupCols = 640;
+constexpr int kMaxWChunks = (kMaxGroupCols + kAccCols - 1) / kAccCols;  // column tiles of a group
 constexpr int kWBox = 32;                    // W rows per TMA box
 
 struct Params {
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const Params p)
 {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[16];  // 15 used
+    __shared__ __align__(8) uint64_t bars[24];
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_flag;
     __shared__ int lens_sh[kLensCache];
@@ -427,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto empty_a = [&](int s) { return bar0 + 8u * (2 + s); };     // 2,3
     auto tmem_full = [&](int b) { return bar0 + 8u * (4 + b); };   // 4..7
     auto tmem_empty = [&](int b) { return bar0 + 8u * (8 + b); };  // 8..11
-    const uint32_t w_full = bar0 + 8u * 12, w_empty = bar0 + 8u * 13, final_bar = bar0 + 8u * 14;
+    auto w_full = [&](int j) { return bar0 + 8u * (16 + j); };     // 16..18: W rows of column tile j
+    const uint32_t w_empty = bar0 + 8u * 13, final_bar = bar0 + 8u * 14;
 
     if (tid == 0) {
         abort_flag = 0;
@@ -440,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(tmem_empty(b), 4 * kEpiGroups);  // one arrival per epilogue warp
         }
         static_assert(kAccBufs * kAccCols == 512, "TMEM holds 512 columns");
-        mbar_init(w_full, 1);
+        for (int j = 0; j < kMaxWChunks; j++) mbar_init(w_full(j), 1);
         mbar_init(w_empty, 1);
         mbar_init(final_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -463,19 +466,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0;
         uint32_t empty_par[kStages] = {0, 0};
         int last_issued_par[kStages] = {-1, -1};
-        int cur_g = -1, w_loads = 0;
+        int cur_g = -1, w_loads = 0, w_rest = 0, w_width = 0, w_c0 = 0;
+        int w_last_par[kMaxWChunks];
+        for (int j = 0; j < kMaxWChunks; j++) w_last_par[j] = -1;
+        // W rows of column tile j of the group: one barrier per tile, so the
+        // first MMAs need only the first tile; every block starts at its own
+        // box of the tile, which spreads the blocks' simultaneous reads of the
+        // same W lines over the L2.
+        auto load_w_tile = [&](int j) {
+            const int n0 = j * kAccCols, cols = min(kAccCols, w_width - n0), nb = cols / kWBox;
+            mbar_expect_tx(w_full(j), (uint32_t)cols * 256u);
+            for (int i = 0; i < nb; i++) {
+                const int rb = (i + (int)blockIdx.x) % nb;
+                for (int kh = 0; kh < 2; kh++)
+                    tma_load_2d(w_smem + kh * w_half + (n0 + rb * kWBox) * 128, &tmap_w, w_full(j), kh * 64,
+                                w_c0 + n0 + rb * kWBox);
+            }
+            w_last_par[j] = (w_last_par[j] + 1) & 1;
+        };
         bool first_pass = true;
         for (ItemIter iter(p); iter.live(p) && !abort_flag; iter.next(p)) {
             const Item im = iter.item(p, lens_sh);
             if (im.skip) continue;
             if (im.group != cur_g) {
                 if (cur_g >= 0 && !mbar_wait(w_empty, (w_loads - 1) & 1, &abort_flag, p.status)) break;
-                int c0, width;
-                group_cols(p, im.group, c0, width);
-                mbar_expect_tx(w_full, (uint32_t)width * 256u);
-                for (int rb = 0; rb < width / kWBox; rb++)
-                    for (int kh = 0; kh < 2; kh++)
-                        tma_load_2d(w_smem + kh * w_half + rb * kWBox * 128, &tmap_w, w_full, kh * 64, c0 + rb * kWBox);
+                group_cols(p, im.group, w_c0, w_width);
+                load_w_tile(0);  // the rest after this item's key tile
+                w_rest = 1;
                 cur_g = im.group;
                 w_loads++;
             }
@@ -501,24 +518,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(a_smem + stage * kTileBytes + kHalfBytes, &tmap_keys, full_a(stage), 64, row0);
             last_issued_par[stage] = (last_issued_par[stage] + 1) & 1;
             stage ^= 1;
+            for (; w_rest > 0 && w_rest * kAccCols < w_width; w_rest++) load_w_tile(w_rest);
+            w_rest = 0;
         }
         // our own copies in flight must land before the CTA exits
         for (int st = 0; st < kStages; st++)
             if (last_issued_par[st] >= 0) mbar_wait(full_a(st), (uint32_t)last_issued_par[st], &abort_flag, p.status);
-        if (w_loads > 0) mbar_wait(w_full, (w_loads - 1) & 1, &abort_flag, p.status);
+        for (int j = 0; j < kMaxWChunks; j++)
+            if (w_last_par[j] >= 0) mbar_wait(w_full(j), (uint32_t)w_last_par[j], &abort_flag, p.status);
     } else if (warp == 1 && lane == 0) {
         // ----------------------------------------------------------- MMA ----
         int stage = 0, seq = 0;  // seq: column-tile sequence number; buffer seq % 4, use seq / 4
         uint32_t full_par[kStages] = {0, 0};
-        int cur_g = -1, w_uses = 0;
+        int cur_g = -1;
+        uint32_t w_ready = 0, w_par = 0;  // bit j: tile j of the current group landed / next parity
         for (ItemIter iter(p); iter.live(p) && !abort_flag; iter.next(p)) {
             const Item im = iter.item(p, lens_sh);
             if (im.skip) continue;
             if (im.group != cur_g) {
                 if (cur_g >= 0) mma_commit(w_empty);  // W free once the MMAs so far complete
-                if (!mbar_wait(w_full, w_uses & 1, &abort_flag, p.status)) break;
                 cur_g = im.group;
-                w_uses++;
+                w_ready = 0;
             }
             if (!mbar_wait(full_a(stage), full_par[stage], &abort_flag, p.status)) break;
             full_par[stage] ^= 1u;
@@ -529,6 +549,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int n0 = 0; n0 < width; n0 += kAccCols, seq++) {
                 const int nw = min(kAccCols, width - n0);
                 const int acc = seq & (kAccBufs - 1);
+                const int j = n0 / kAccCols;
+                if (!((w_ready >> j) & 1u)) {  // first use of W tile j in this group
+                    if (!mbar_wait(w_full(j), (w_par >> j) & 1u, &abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    w_par ^= 1u << j;
+                    w_ready |= 1u << j;
+                }
                 // wait for the epilogue to release use (seq / 4 - 1) of this buffer
                 if (!mbar_wait(tmem_empty(acc), ((seq / kAccBufs) & 1) ^ 1u, &abort_flag, p.status)) {
                     ok = false;
