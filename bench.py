@@ -178,8 +178,8 @@ class Bench:
         self.path = {"auto": mp.MP_PATH_AUTO, "split": mp.MP_PATH_SPLIT, "fused": mp.MP_PATH_FUSED}[path]
         self.graph_error = None
         fused = self.path == mp.MP_PATH_FUSED
-        # hash 1, append 2, decode: qhash + (scan, attention | fused) + merge
-        self.launches_per_step = 3 + (3 if fused else 4)
+        # hash 1, append 1, decode: qhash + (scan, attention | fused) + merge
+        self.launches_per_step = 2 + (3 if fused else 4)
 
     def hash(self):
         self.mp.hash_keys(self.shape, self.K, self.W, self.prefill, self.codes, seq_lens=self.lens0)

@@ -11,104 +11,128 @@
 
 namespace mp {
 
-constexpr int kAppendCols = 64;  // hyperplane columns per append block (4 lanes each)
+constexpr int kAppendCluster = 8;  // blocks per sequence (one thread-block cluster)
+constexpr int kAppendThreads = 1024;
 
 // --------------------------------------------------------------- append ----
-// grid (ceil(L / TB), B * Hkv), 256 threads: 4 lanes per hyperplane column
-// of a block of TB = 64 / K whole tables; each lane sums 32 exact bf16
-// products in fp32 and two shuffles add the quarters (bits can differ from
-// the tensor-core hash only where the projection is within fp32 rounding of
-// zero).
-__global__ void __launch_bounds__(256) append_kernel(Shape s, const uint16_t *__restrict__ k_new,
-                                                     const uint16_t *__restrict__ v_new,
-                                                     const uint16_t *__restrict__ W, uint16_t *kc, uint16_t *vc,
-                                                     void *codes, const int32_t *__restrict__ seq_lens,
-                                                     int32_t *status)
+// grid (kAppendCluster, B): one cluster of kAppendCluster blocks per sequence.
+// Block r takes tables [r T, r T + T) (T = ceil(L / kAppendCluster)) of all
+// Hkv kv heads of the sequence: its (column, head) pairs, head-minor, are
+// dealt to groups of four lanes (the heads of one column sit in neighbouring
+// lane groups and share the W row through L1); each lane sums 32 exact bf16
+// products in fp32, and two shuffles add the quarters (bits can differ from the
+// tensor-core hash only where the projection is within fp32 rounding of
+// zero).  Every block reads the position seq_lens[b] first and then arrives
+// on the cluster barrier; block 0 waits on it before writing seq_lens[b] + 1,
+// so the length moves only after every block of the sequence has read it.
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const uint16_t *__restrict__ k_new,
+                                                                const uint16_t *__restrict__ v_new,
+                                                                const uint16_t *__restrict__ W, uint16_t *kc,
+                                                                uint16_t *vc, void *codes, int32_t *seq_lens,
+                                                                int32_t *status)
 {
-    __shared__ float xs[kHeadDim];
-    __shared__ uint8_t bits[kAppendCols];
+    extern __shared__ float xs[];  // [Hkv][kHeadDim + 4] new keys (element d at d + d / 32), then bits
     const int tid = threadIdx.x;
-    const int unit = blockIdx.y;
-    const int b = unit / s.Hkv;
+    const int r = blockIdx.x, b = blockIdx.y;
+    const int T = (s.L + kAppendCluster - 1) / kAppendCluster;
+    const int l0 = min(s.L, r * T), l1 = min(s.L, l0 + T);
+    const int c_begin = l0 * s.K, ncol = (l1 - l0) * s.K;
+    uint8_t *bits = reinterpret_cast<uint8_t *>(xs + s.Hkv * (kHeadDim + 4));  // [Hkv][T K]
     grid_dependency_wait();
     const int pos = seq_lens[b];
-    if (pos < 0 || pos >= s.Ncap) {
-        if (blockIdx.x == 0 && unit % s.Hkv == 0 && tid == 0) set_status(status, MP_ERR_CAPACITY);
-        return;
-    }
-    const uint16_t *kn = k_new + (size_t)unit * kHeadDim;
-    if (blockIdx.x == 0 && tid < 32) {
-        const bool isv = tid >= 16;
-        const uint4 *src = reinterpret_cast<const uint4 *>((isv ? v_new : k_new) + (size_t)unit * kHeadDim);
-        uint4 *dst = reinterpret_cast<uint4 *>((isv ? vc : kc) + ((size_t)unit * s.Ncap + pos) * kHeadDim);
-        dst[tid & 15] = src[tid & 15];
-    }
-    if (tid < kHeadDim) xs[tid] = bf16_to_f32(kn[tid]);
-    __syncthreads();
-    const int TB = kAppendCols / s.K;
-    const int l0 = blockIdx.x * TB;
-    const int col = tid >> 2, part = tid & 3;  // column of the block, quarter of the dims
-    const int c = l0 * s.K + col;
-    const bool valid = col < TB * s.K && c < s.LK;
-    float dot = 0.f;
-    if (valid) {
-        const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)c * kHeadDim + part * 32);
-        const float *xp = xs + part * 32;
-#pragma unroll
-        for (int j8 = 0; j8 < 4; j8++) {
-            const uint4 w = __ldg(wr + j8);
-            dot = fmaf(xp[j8 * 8 + 0], bf16_lo(w.x), dot);
-            dot = fmaf(xp[j8 * 8 + 1], bf16_hi(w.x), dot);
-            dot = fmaf(xp[j8 * 8 + 2], bf16_lo(w.y), dot);
-            dot = fmaf(xp[j8 * 8 + 3], bf16_hi(w.y), dot);
-            dot = fmaf(xp[j8 * 8 + 4], bf16_lo(w.z), dot);
-            dot = fmaf(xp[j8 * 8 + 5], bf16_hi(w.z), dot);
-            dot = fmaf(xp[j8 * 8 + 6], bf16_lo(w.w), dot);
-            dot = fmaf(xp[j8 * 8 + 7], bf16_hi(w.w), dot);
+    asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");  // (release) this block has read pos
+    const bool ok = pos >= 0 && pos < s.Ncap;
+    if (!ok) {
+        if (r == 0 && tid == 0) set_status(status, MP_ERR_CAPACITY);
+    } else {
+        const size_t unit0 = (size_t)b * s.Hkv;
+        if (r == 0) {  // the K and V rows, 16 bytes per thread
+            for (int i = tid; i < s.Hkv * 32; i += blockDim.x) {
+                const int h = i >> 5, isv = (i >> 4) & 1, e = i & 15;
+                const uint4 *src = reinterpret_cast<const uint4 *>((isv ? v_new : k_new) + (unit0 + h) * kHeadDim);
+                uint4 *dst = reinterpret_cast<uint4 *>((isv ? vc : kc) + ((unit0 + h) * s.Ncap + pos) * kHeadDim);
+                dst[e] = src[e];
+            }
         }
-    }
-    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-    const bool bit = valid && dot > 0.f;
-    if (!s.planes) {
-        if (part == 0) bits[col] = bit;
+        for (int i = tid; i < s.Hkv * kHeadDim; i += blockDim.x) {
+            const int h = i / kHeadDim, d = i % kHeadDim;
+            xs[h * (kHeadDim + 4) + d + (d >> 5)] = bf16_to_f32(k_new[(unit0 + h) * kHeadDim + d]);
+        }
         __syncthreads();
-        if (tid < TB && l0 + tid < s.L) {
-            unsigned code = 0;
-            for (int bb = 0; bb < 8; bb++) code |= (unsigned)bits[tid * 8 + bb] << bb;
-            static_cast<uint8_t *>(codes)[((size_t)unit * s.L + l0 + tid) * s.Ncap + pos] = (uint8_t)code;
+        const int part = tid & 3;  // quarter of the dims
+        constexpr int kSlots = kAppendThreads / 4;
+        const int npairs = ncol * s.Hkv;
+        for (int pi = tid >> 2; pi < (npairs + kSlots - 1) / kSlots * kSlots; pi += kSlots) {
+            const bool valid = pi < npairs;
+            const int cl = valid ? pi / s.Hkv : 0, h = valid ? pi - cl * s.Hkv : 0;
+            float dot = 0.f;
+            if (valid) {
+                const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)(c_begin + cl) * kHeadDim + part * 32);
+                const float *xp = xs + h * (kHeadDim + 4) + part * 33;
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const uint4 w = __ldg(wr + j);
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        dot = fmaf(xp[j * 8 + 2 * e], bf16_lo(wv[e]), dot);
+                        dot = fmaf(xp[j * 8 + 2 * e + 1], bf16_hi(wv[e]), dot);
+                    }
+                }
+            }
+            dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+            dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+            if (valid && part == 0) bits[h * T * s.K + cl] = dot > 0.f;
         }
-    } else if (valid && part == 0) {
-        const int l = c / s.K, bb = c - l * s.K;
-        unsigned int *word =
-            static_cast<unsigned int *>(codes) + (((size_t)unit * s.L + l) * (s.Ncap >> 5) + (pos >> 5)) * s.K + bb;
-        const unsigned int m = 1u << (pos & 31);
-        if (bit)
-            atomicOr(word, m);
-        else
-            atomicAnd(word, ~m);
+        __syncthreads();
+        if (!s.planes) {
+            for (int i = tid; i < s.Hkv * (l1 - l0); i += blockDim.x) {
+                const int h = i / (l1 - l0), lt = i % (l1 - l0);
+                unsigned code = 0;
+                for (int bb = 0; bb < 8; bb++) code |= (unsigned)bits[h * T * s.K + lt * 8 + bb] << bb;
+                static_cast<uint8_t *>(codes)[((unit0 + h) * s.L + l0 + lt) * s.Ncap + pos] = (uint8_t)code;
+            }
+        } else {
+            const unsigned int m = 1u << (pos & 31);
+            for (int i = tid; i < s.Hkv * ncol; i += blockDim.x) {
+                const int h = i / ncol, cl = i % ncol;
+                const int c = c_begin + cl, l = c / s.K, bb = c - l * s.K;
+                unsigned int *word = static_cast<unsigned int *>(codes) +
+                                     (((unit0 + h) * s.L + l) * (s.Ncap >> 5) + (pos >> 5)) * s.K + bb;
+                if (bits[h * T * s.K + cl])
+                    atomicOr(word, m);
+                else
+                    atomicAnd(word, ~m);
+            }
+        }
     }
-}
-
-__global__ void bump_lengths_kernel(int B, int Ncap, int32_t *seq_lens)
-{
-    grid_dependency_wait();
-    for (int b = threadIdx.x; b < B; b += blockDim.x) {
-        const int p = seq_lens[b];
-        if (p >= 0 && p < Ncap) seq_lens[b] = p + 1;
-    }
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // (acquire) every block has read pos
+    if (ok && r == 0 && tid == 0) seq_lens[b] = pos + 1;
 }
 
 cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t *v_new, const uint16_t *W,
                           uint16_t *kc, uint16_t *vc, void *codes, int32_t *seq_lens, int32_t *status,
                           cudaStream_t st)
 {
-    const int TB = kAppendCols / s.K;
-    dim3 grid((s.L + TB - 1) / TB, s.B * s.Hkv);
-    cudaError_t e = launch_pdl(append_kernel, grid, dim3(256), 0, st, s, k_new, v_new, W, kc, vc, codes,
-                               (const int32_t *)seq_lens, status);
+    const int T = (s.L + kAppendCluster - 1) / kAppendCluster;
+    const size_t smem = (size_t)s.Hkv * (kHeadDim + 4) * sizeof(float) + (size_t)s.Hkv * T * s.K;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(append_kernel), (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(bump_lengths_kernel, dim3(1), dim3(256), 0, st, s.B, s.Ncap, seq_lens);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kAppendCluster, s.B);
+    cfg.blockDim = dim3(kAppendThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kAppendCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, append_kernel, s, k_new, v_new, W, kc, vc, codes, seq_lens, status);
 }
 
 }  // namespace mp
