@@ -42,6 +42,14 @@ __device__ __forceinline__ void grid_dependency_wait()
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// The two halves, for a kernel with work that does not depend on its
+// immediate predecessor.  Every kernel of this library lets its successor
+// launch only after its own wait has returned, so when a kernel starts, all
+// stream work before its predecessor is complete and visible: code before
+// grid_wait() may read that (cached codes, lengths), but nothing its
+// predecessor writes, and it writes no global memory.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {

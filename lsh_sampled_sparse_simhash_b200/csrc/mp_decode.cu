@@ -273,29 +273,49 @@ __device__ __forceinline__ void combine_splits(uint32_t (&s1)[G][NW], uint32_t (
 // bits.  Warp 0 folds the other splits' counters and compacts the chunk's
 // candidates alone (warp-level scan, no block barrier); warps 1..7 exit.
 template <int G>
-__global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
+__global__ void __launch_bounds__(kScanThreads, 3) scan_k8_kernel(
     Shape s, const uint8_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
     const int32_t *__restrict__ seq_lens, int max_len, int nchunk, ScanOut o)
 {
     extern __shared__ uint32_t dyn[];  // rep [L][G] (query code in 4 bytes), then split partials
     uint32_t *rep = dyn;
     uint32_t *part = dyn + ((s.L * G + 3) & ~3);
-    constexpr int TS = kSplitsK8, TG = kScanThreads / TS, NB = 8;
+    constexpr int TS = kSplitsK8, TG = kScanThreads / TS, NB = 4;
     static_assert(TG == 32, "split ts = warp ts, token group tg = lane");
     const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
     const int unit = blockIdx.y, chunk = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
-    grid_dependency_wait();
-    const int N = clamp_len(seq_lens, b, max_len, o.status, chunk == 0 && kvh == 0 && threadIdx.x == 0);
+    grid_launch_dependents();
+    // lengths and codes come from work before the query hash: read them first
+    const int N = clamp_len(seq_lens, b, max_len, o.status, false);
     const int c0 = chunk * kChunkBytes;
-    if (c0 >= N) return;
+    const bool reporter = chunk == 0 && kvh == 0 && threadIdx.x == 0;  // of a bad length of sequence b
+    if (c0 >= N) {
+        if (reporter) {
+            grid_wait();  // the status word is cleared by the query hash
+            clamp_len(seq_lens, b, max_len, o.status, true);
+        }
+        return;
+    }
+    const int t0 = c0 + tg * 16;
+    const uint8_t *base = codes + (size_t)unit * s.L * s.Ncap + t0;
+    uint4 wv[NB];
+    auto load_batch = [&](int lb) {
+#pragma unroll
+        for (int i = 0; i < NB; i++) {
+            const int l = lb + i * TS;
+            wv[i] = t0 < N && l < s.L ? ld_stream_16(base + (size_t)l * s.Ncap) : make_uint4(0, 0, 0, 0);
+        }
+    };
+    load_batch(ts);
+    grid_wait();  // the query codes are the query hash's output
+    if (reporter) clamp_len(seq_lens, b, max_len, o.status, true);
     for (int i = threadIdx.x; i < s.L * G; i += blockDim.x) {
         const int l = i / G, g = i % G;
         rep[i] = (qcodes[((size_t)b * s.Hq + kvh * G + g) * s.L + l] & 0xFFu) * 0x01010101u;
     }
     __syncthreads();
 
-    const int t0 = c0 + tg * 16;
     uint32_t s1[G][4], s2[G][4];
 #pragma unroll
     for (int g = 0; g < G; g++)
@@ -303,14 +323,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_k8_kernel(
         for (int j = 0; j < 4; j++) s1[g][j] = s2[g][j] = 0u;
 
     if (t0 < N) {
-        const uint8_t *base = codes + (size_t)unit * s.L * s.Ncap + t0;
         for (int lb = ts; lb < s.L; lb += NB * TS) {
-            uint4 wv[NB];
-#pragma unroll
-            for (int i = 0; i < NB; i++) {
-                const int l = lb + i * TS;
-                wv[i] = l < s.L ? ld_stream_16(base + (size_t)l * s.Ncap) : make_uint4(0, 0, 0, 0);
-            }
+            if (lb != ts) load_batch(lb);
 #pragma unroll
             for (int i = 0; i < NB; i++) {
                 const int l = lb + i * TS;
@@ -433,13 +447,17 @@ __global__ void __launch_bounds__(kScanThreads + 32) scan_planes_kernel(
     __shared__ __align__(8) uint64_t full[S], empty[S];
     __shared__ int range_sh[4];  // first item (b, kvh, chunk), item count
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    grid_dependency_wait();
+    // The lengths and the codes come from work before the query hash: the
+    // work split and the producer's first code stages go ahead of grid_wait(),
+    // which the consumers pass before reading the query codes and the
+    // compactor before writing the candidate lists.
+    grid_launch_dependents();
 
     if (threadIdx.x == 0) {
         // this block's contiguous share of the live items
         long long total = 0;
         for (int b = 0; b < s.B; b++) {
-            const int n = clamp_len(seq_lens, b, max_len, o.status, blockIdx.x == 0);
+            const int n = clamp_len(seq_lens, b, max_len, o.status, false);
             total += (long long)s.Hkv * ((n + kChunkPlanes - 1) / kChunkPlanes);
         }
         long long x = total * blockIdx.x / gridDim.x;
@@ -465,7 +483,13 @@ __global__ void __launch_bounds__(kScanThreads + 32) scan_planes_kernel(
     }
     __syncthreads();
     const int count = range_sh[3];
-    if (count <= 0) return;
+    if (count <= 0) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
+            grid_wait();  // the status word is cleared by the query hash
+            for (int b = 0; b < s.B; b++) clamp_len(seq_lens, b, max_len, o.status, true);
+        }
+        return;
+    }
     LiveCursor cur;
     cur.b = range_sh[0];
     cur.kvh = range_sh[1];
@@ -503,6 +527,11 @@ __global__ void __launch_bounds__(kScanThreads + 32) scan_planes_kernel(
             }
             if (it >= 1) {
                 const int ci = it - 1;
+                if (ci == 0) {
+                    grid_wait();
+                    if (blockIdx.x == 0 && lane == 0)
+                        for (int b = 0; b < s.B; b++) clamp_len(seq_lens, b, max_len, o.status, true);
+                }
                 bar_sync_all(2);  // the consumers' partials of item ci are in buffer ci & 1
                 const uint32_t *pp = part + (ci & 1) * (G * 2 * kScanThreads);
                 uint32_t s1[G], s2[G];
@@ -540,6 +569,7 @@ __global__ void __launch_bounds__(kScanThreads + 32) scan_planes_kernel(
     const int lane_off = box * NC * St::kBoxWords + ts * St::kBoxWords + in_box;  // words into a stage
     int e = 0, qm_unit = -1;
     bool dead = false;  // a copy never landed: stop waiting, keep the barriers in step
+    grid_wait();        // the query codes are the query hash's output
     for (int it = 0; it < count; it++, cur.next(s, seq_lens, max_len)) {
         const int unit = cur.unit(s);
         if (unit != qm_unit) {  // uniform over the consumers
