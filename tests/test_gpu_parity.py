@@ -327,6 +327,16 @@ def test_full_size_sampled_units(name):
     """The full workload in the benchmark's launch configuration (hash every
     key, append one token per sequence, decode); two (b, kv head) units are
     checked against the oracle on the oracle's own codes."""
+    _full_size(name, mp.MP_PATH_AUTO)
+
+
+@pytest.mark.parametrize("name", ["batch8_64k", "ragged16_planes"])
+def test_full_size_fused_path(name):
+    """The same at full size through the fused scan + attend kernel."""
+    _full_size(name, mp.MP_PATH_FUSED)
+
+
+def _full_size(name, path):
     w = WORKLOADS[name] if name in WORKLOADS else WORKLOADS[name.rsplit("_", 1)[0]].with_(code_layout="planes")
     inp = make_inputs(w)
     run = Run(w, inp)
@@ -358,8 +368,8 @@ def test_full_size_sampled_units(name):
     assert bad == 0
     run.set_codes(codes, units)
     qref, _ = oracle_query_codes(inp, w)
-    gpu = run.decode(qcodes_in=qref)
+    gpu = run.decode(qcodes_in=qref, path=path)
     assert gpu["status"] == 0
     ref = oracle_decode_units(inp2, w, units, codes, qref)
     worst = check_outputs(gpu, ref, w)
-    print(f"{name}: worst rel-L2 {worst:.2e}; mean |S_h| {gpu['ns'].mean():.0f}")
+    print(f"{name} (path {path}): worst rel-L2 {worst:.2e}; mean |S_h| {gpu['ns'].mean():.0f}")
