@@ -616,6 +616,7 @@ def main():
                         units=f"{int(lens_after.sum())} tokens x {w.n_kv_heads} kv heads; {union} union rows",
                         traffic=traffic_record("decode", w.name, config_of(w)["code_layout"]))
         dec_roof["frac"] = dec_roof["achieved"] / dec_roof["peak"]
+        dec_roof["frac_of_nominal_8tbs"] = dec_roof["achieved"] / 8000.0  # nominal HBM3e figure, for context
         dominant = hash_roof if hash_ms >= decode_ms else dec_roof
         roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
         roofline["kernel"] = dominant["kernel"]
