@@ -1005,7 +1005,9 @@ template <int G>
 __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ uint32_t meta[kAttStages][kAttRows];  // headmask | exact << 8
+    constexpr int kWarpRows = kAttRows / 4;                   // rows of a tile per warp
+    constexpr int kWarpStage = kWarpRows * kRowStride * 2;    // one warp's K rows then V rows
+    __shared__ uint32_t meta[4][kAttStages][kWarpRows];       // per warp: headmask | exact << 8
     __shared__ float ucos[4][16 * G];                // per warp: cos of pairs needing log u
     __shared__ float uval[4][16 * G];                // per warp: their log u
     __shared__ float qinv[G];
@@ -1028,9 +1030,9 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     uint32_t pre0 = 0xFFFFFFFFu, pre1 = 0xFFFFFFFFu;
     if (direct) {
         if (tid == 0) dcount = a.cnt[((size_t)unit * a.nchunk + c_begin) * 16];
-        if (tid < kAttRows) {
-            pre0 = lists[tid];
-            pre1 = lists[kAttRows + tid];
+        if (lane < kWarpRows) {  // the warp's rows of tiles 0 and 1
+            pre0 = lists[warp * kWarpRows + lane];
+            pre1 = lists[kAttRows + warp * kWarpRows + lane];
         }
     }
     int N = a.seq_lens[b];
@@ -1086,14 +1088,18 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     const uint16_t *vbase = a.vc + (size_t)unit * s.Ncap * kHeadDim;
     const int ntiles = (nrows + kAttRows - 1) / kAttRows;
 
-    // Candidate entries: threads 0..63 each read the entry of one row of a tile
-    // two tiles ahead (its load overlaps the current tile's arithmetic) and
-    // leave it in a 2-slot shared ring; the copy issue reads its 8 rows there.
+    // Each warp owns rows 16 warp .. 16 warp + 15 of every 64-row tile and runs
+    // its own entry ring and 2-stage cp.async ring, so the warps of a block
+    // meet only at the start (span prefix, q norms) and at the end (merge of
+    // their states), never per tile.  Lanes 0..15 read the entries of the
+    // warp's rows two tiles ahead (the load overlaps the current tile's
+    // arithmetic) into a 2-slot ring; the copy issue reads its rows there.
     static_assert(kAttStages == 2, "entry ring sized for one tile of copies in flight");
-    __shared__ uint32_t ents[2][kAttRows];
-    int jc = 0;  // chunk of this thread's next candidate (rows are visited in increasing order)
+    __shared__ uint32_t ents[4][2][kWarpRows];
+    uint8_t *wring = smem + warp * (kAttStages * kWarpStage);
+    int jc = 0;  // chunk of this lane's next candidate (rows are visited in increasing order)
     auto fetch1 = [&](int tile) -> uint32_t {
-        const int e = tile * kAttRows + tid;
+        const int e = tile * kAttRows + warp * kWarpRows + lane;
         if (e >= nrows) return 0xFFFFFFFFu;
         if (dsplit) return (uint32_t)(e < n_sink ? e : win0 + (e - n_sink));
         const int r = e0 + e;
@@ -1102,32 +1108,32 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     };
 
     auto issue = [&](int tile, int stage) {
-        uint8_t *ks_ = smem + stage * kStageBytes;
-        uint8_t *vs_ = ks_ + kAttRows * kRowStride;
-        const int col = tid & 15;
+        uint8_t *ks_ = wring + stage * kWarpStage;
+        uint8_t *vs_ = ks_ + kWarpRows * kRowStride;
+        const int col = lane & 15;
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const int r = (tid >> 4) + 8 * i;
-            const uint32_t ent = ents[tile & 1][r];
+        for (int i = 0; i < kWarpRows / 2; i++) {
+            const int r = (lane >> 4) + 2 * i;
+            const uint32_t ent = ents[warp][tile & 1][r];
             const bool ok = ent != 0xFFFFFFFFu;
             const int tok = ok ? (int)(ent & 0xFFFFFFu) : 0;
             const size_t off = (size_t)tok * kHeadDim + col * 8;
             cp_async_16(ks_ + r * kRowStride + col * 16, kbase + off, ok ? 16 : 0);
             cp_async_16(vs_ + r * kRowStride + col * 16, vbase + off, ok ? 16 : 0);
-            if (col == 0) meta[stage][r] = ok ? (dsplit ? dmeta : (ent >> 24)) : 0u;
+            if (col == 0) meta[warp][stage][r] = ok ? (dsplit ? dmeta : (ent >> 24)) : 0u;
         }
     };
 
-    if (tid < kAttRows) {
+    if (lane < kWarpRows) {
         if (direct) {
-            ents[0][tid] = tid < nrows ? pre0 : 0xFFFFFFFFu;
-            ents[1][tid] = kAttRows + tid < nrows ? pre1 : 0xFFFFFFFFu;
+            ents[warp][0][lane] = warp * kWarpRows + lane < nrows ? pre0 : 0xFFFFFFFFu;
+            ents[warp][1][lane] = kAttRows + warp * kWarpRows + lane < nrows ? pre1 : 0xFFFFFFFFu;
         } else {
-            if (ntiles > 0) ents[0][tid] = fetch1(0);
-            if (ntiles > 1) ents[1][tid] = fetch1(1);
+            if (ntiles > 0) ents[warp][0][lane] = fetch1(0);
+            if (ntiles > 1) ents[warp][1][lane] = fetch1(1);
         }
     }
-    __syncthreads();  // entries of tiles 0 and 1, qinv
+    __syncthreads();  // qinv (and this warp's entries of tiles 0 and 1)
     if (ntiles > 0) issue(0, 0);
     cp_async_commit();
     attn_set_qinv<G>(w, qinv, lane);
@@ -1135,17 +1141,17 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     for (int tile = 0; tile < ntiles; tile++) {
         if (tile + 1 < ntiles) issue(tile + 1, (tile + 1) % kAttStages);
         cp_async_commit();
-        const bool fetcher = tid < kAttRows && tile + 2 < ntiles;
+        const bool fetcher = lane < kWarpRows && tile + 2 < ntiles;
         const uint32_t pend = fetcher ? fetch1(tile + 2) : 0u;
         cp_async_wait<kAttStages - 1>();
-        __syncthreads();
+        __syncwarp();
         const int stage = tile % kAttStages;
-        const uint8_t *ks_ = smem + stage * kStageBytes;
-        const uint8_t *vs_ = ks_ + kAttRows * kRowStride;
-
-        attn_tile<G>(w, ks_, vs_, meta[stage], warp, lane, a.scale, a.lu, ucos[warp], uval[warp]);
-        if (fetcher) ents[tile & 1][tid] = pend;  // slot of tile + 2, read after the barrier
-        __syncthreads();  // stage may be refilled next iteration
+        const uint8_t *ks_ = wring + stage * kWarpStage;
+        // the warp's own 16 rows, addressed as warp 0 of a tile
+        attn_tile<G>(w, ks_, ks_ + kWarpRows * kRowStride, meta[warp][stage], 0, lane, a.scale, a.lu, ucos[warp],
+                     uval[warp]);
+        if (fetcher) ents[warp][tile & 1][lane] = pend;  // slot of tile + 2, read after the next __syncwarp
+        __syncwarp();  // the stage may be refilled next iteration
     }
     cp_async_wait<0>();
     __syncthreads();
