@@ -31,14 +31,22 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
                                                                 uint16_t *vc, void *codes, int32_t *seq_lens,
                                                                 int32_t *status)
 {
-    extern __shared__ float xs[];  // [Hkv][kHeadDim + 4] new keys (element d at d + d / 32), then bits
+    // shared: this block's W rows [T K][kHeadDim] bf16, the new keys
+    // [Hkv][kHeadDim + 4] fp32 (element d at d + d / 32), the bits [Hkv][T K]
+    extern __shared__ __align__(16) uint8_t sm_raw[];
     const int tid = threadIdx.x;
     const int r = blockIdx.x, b = blockIdx.y;
     const int T = (s.L + kAppendCluster - 1) / kAppendCluster;
     const int l0 = min(s.L, r * T), l1 = min(s.L, l0 + T);
     const int c_begin = l0 * s.K, ncol = (l1 - l0) * s.K;
-    uint8_t *bits = reinterpret_cast<uint8_t *>(xs + s.Hkv * (kHeadDim + 4));  // [Hkv][T K]
+    uint16_t *wsm = reinterpret_cast<uint16_t *>(sm_raw);
+    float *xs = reinterpret_cast<float *>(sm_raw + (size_t)T * s.K * kHeadDim * 2);
+    uint8_t *bits = reinterpret_cast<uint8_t *>(xs + s.Hkv * (kHeadDim + 4));
     grid_dependency_wait();
+    // the block's W rows into shared memory first: they do not wait for the position
+    for (int i = tid; i < ncol * (kHeadDim / 8); i += blockDim.x)
+        cp_async_16(wsm + (size_t)i * 8, W + (size_t)c_begin * kHeadDim + (size_t)i * 8, 16);
+    cp_async_commit();
     const int pos = seq_lens[b];
     asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");  // (release) this block has read pos
     const bool ok = pos >= 0 && pos < s.Ncap;
@@ -58,6 +66,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
             const int h = i / kHeadDim, d = i % kHeadDim;
             xs[h * (kHeadDim + 4) + d + (d >> 5)] = bf16_to_f32(k_new[(unit0 + h) * kHeadDim + d]);
         }
+        cp_async_wait<0>();
         __syncthreads();
         const int part = tid & 3;  // quarter of the dims
         constexpr int kSlots = kAppendThreads / 4;
@@ -67,11 +76,11 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
             const int cl = valid ? pi / s.Hkv : 0, h = valid ? pi - cl * s.Hkv : 0;
             float dot = 0.f;
             if (valid) {
-                const uint4 *wr = reinterpret_cast<const uint4 *>(W + (size_t)(c_begin + cl) * kHeadDim + part * 32);
+                const uint4 *wr = reinterpret_cast<const uint4 *>(wsm + (size_t)cl * kHeadDim + part * 32);
                 const float *xp = xs + h * (kHeadDim + 4) + part * 33;
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
-                    const uint4 w = __ldg(wr + j);
+                    const uint4 w = wr[j];
                     const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
@@ -106,6 +115,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
             }
         }
     }
+    cp_async_wait<0>();  // (the error path leaves no copy in flight either)
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // (acquire) every block has read pos
     if (ok && r == 0 && tid == 0) seq_lens[b] = pos + 1;
 }
@@ -115,7 +125,8 @@ cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t 
                           cudaStream_t st)
 {
     const int T = (s.L + kAppendCluster - 1) / kAppendCluster;
-    const size_t smem = (size_t)s.Hkv * (kHeadDim + 4) * sizeof(float) + (size_t)s.Hkv * T * s.K;
+    const size_t smem = (size_t)T * s.K * kHeadDim * 2 + (size_t)s.Hkv * (kHeadDim + 4) * sizeof(float) +
+                        (size_t)s.Hkv * T * s.K;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(append_kernel), (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
