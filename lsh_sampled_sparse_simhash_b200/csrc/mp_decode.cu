@@ -29,11 +29,13 @@
 namespace mp {
 
 // ------------------------------------------------------------------ qhash ---
-// grid (ceil(L / TB), B * Hkv), 256 threads.  A block covers TB = 64 / K whole
-// tables (64 or 60 hyperplane columns); four lanes share a column, each summing
-// 32 of the 128 products for all G heads of the kv group (one W load serves G
-// heads), then two shuffles finish the sums.
+// grid (ceil(L / TB), ceil(units / UG)), 256 threads.  A block covers TB =
+// 64 / K whole tables (64 or 60 hyperplane columns) for UG units (kv heads of
+// sequences); four lanes share a column, each summing 32 of the 128 products
+// for all G heads of each unit (one W load serves UG G query vectors), then
+// two shuffles finish the sums.
 constexpr int kQhashCols = 64;
+constexpr int kQhashVecs = 32;  // query vectors a block can stage (UG G)
 
 inline int qhash_tables_per_block(int K) { return kQhashCols / K; }
 
@@ -41,24 +43,24 @@ template <int G>
 __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__restrict__ q,
                                                     const uint16_t *__restrict__ W,
                                                     const uint16_t *__restrict__ qcodes_in,
-                                                    uint16_t *__restrict__ qcodes, int32_t *status)
+                                                    uint16_t *__restrict__ qcodes, int32_t *status, int ug)
 {
-    __shared__ float qs[G][kHeadDim + 4];  // element d at d + d / 32: the 4 quarters hit distinct banks
-    __shared__ uint8_t bits[G][kQhashCols];
+    __shared__ float qs[kQhashVecs][kHeadDim + 4];  // element d at d + d / 32: the 4 quarters hit distinct banks
+    __shared__ uint8_t bits[kQhashVecs][kQhashCols];
     const int tid = threadIdx.x;
-    const int unit = blockIdx.y;
-    const int b = unit / s.Hkv, kvh = unit % s.Hkv;
+    const int units = s.B * s.Hkv;
+    const int u0 = blockIdx.y * ug, nu = min(ug, units - u0);  // units u0 .. u0 + nu - 1
     const int TB = kQhashCols / s.K;
     const int l0 = blockIdx.x * TB;
-    const size_t vec0 = (size_t)b * s.Hq + (size_t)kvh * G;
+    const size_t vec0 = (size_t)u0 * G;  // query vectors of a unit are consecutive: (b Hkv + kvh) G + g
 
     grid_dependency_wait();
     if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *status = 0;
 
     if (qcodes_in) {
-        for (int i = tid; i < G * TB; i += blockDim.x) {
-            int g = i / TB, l = l0 + i % TB;
-            if (l < s.L) qcodes[(vec0 + g) * s.L + l] = qcodes_in[(vec0 + g) * s.L + l];
+        for (int i = tid; i < nu * G * TB; i += blockDim.x) {
+            const int v = i / TB, l = l0 + i % TB;
+            if (l < s.L) qcodes[(vec0 + v) * s.L + l] = qcodes_in[(vec0 + v) * s.L + l];
         }
         return;
     }
@@ -72,49 +74,69 @@ __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__r
 #pragma unroll
         for (int j = 0; j < 4; j++) w4[j] = __ldg(wr + j);
     }
-    for (int i = tid; i < G * kHeadDim; i += blockDim.x) {
+    for (int i = tid; i < nu * G * kHeadDim; i += blockDim.x) {
         const int d = i % kHeadDim;
         qs[i / kHeadDim][d + (d >> 5)] = bf16_to_f32(q[(vec0 + i / kHeadDim) * kHeadDim + d]);
     }
     __syncthreads();
 
-    float acc[G];
+    for (int u = 0; u < nu; u++) {
+        float acc[G];
 #pragma unroll
-    for (int g = 0; g < G; g++) acc[g] = 0.f;
-    if (valid) {
+        for (int g = 0; g < G; g++) acc[g] = 0.f;
+        if (valid) {
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const uint32_t wv[4] = {w4[j].x, w4[j].y, w4[j].z, w4[j].w};
+            for (int j = 0; j < 4; j++) {
+                const uint32_t wv[4] = {w4[j].x, w4[j].y, w4[j].z, w4[j].w};
 #pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const int dd = part * 33 + j * 8 + 2 * e;  // padded index of dim part * 32 + j * 8 + 2 e
-                const float w0 = bf16_lo(wv[e]), w1 = bf16_hi(wv[e]);
+                for (int e = 0; e < 4; e++) {
+                    const int dd = part * 33 + j * 8 + 2 * e;  // padded index of dim part * 32 + j * 8 + 2 e
+                    const float w0 = bf16_lo(wv[e]), w1 = bf16_hi(wv[e]);
 #pragma unroll
-                for (int g = 0; g < G; g++) {
-                    acc[g] = fmaf(w0, qs[g][dd], acc[g]);
-                    acc[g] = fmaf(w1, qs[g][dd + 1], acc[g]);
+                    for (int g = 0; g < G; g++) {
+                        acc[g] = fmaf(w0, qs[u * G + g][dd], acc[g]);
+                        acc[g] = fmaf(w1, qs[u * G + g][dd + 1], acc[g]);
+                    }
                 }
             }
         }
-    }
 #pragma unroll
-    for (int g = 0; g < G; g++) {
-        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
-        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 2);
-    }
-    if (part == 0) {
+        for (int g = 0; g < G; g++) {
+            acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
+            acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 2);
+        }
+        if (part == 0) {
 #pragma unroll
-        for (int g = 0; g < G; g++) bits[g][cl] = valid && acc[g] > 0.f;
-    }
-    __syncthreads();
-    if (tid < G * TB) {
-        const int g = tid / TB, tl = tid % TB, l = l0 + tl;
-        if (l < s.L) {
-            unsigned code = 0;
-            for (int bb = 0; bb < s.K; bb++) code |= (unsigned)bits[g][tl * s.K + bb] << bb;
-            qcodes[(vec0 + g) * s.L + l] = (uint16_t)code;
+            for (int g = 0; g < G; g++) bits[u * G + g][cl] = valid && acc[g] > 0.f;
         }
     }
+    __syncthreads();
+    for (int i = tid; i < nu * G * TB; i += blockDim.x) {
+        const int v = i / TB, tl = i % TB, l = l0 + tl;
+        if (l < s.L) {
+            unsigned code = 0;
+            for (int bb = 0; bb < s.K; bb++) code |= (unsigned)bits[v][tl * s.K + bb] << bb;
+            qcodes[(vec0 + v) * s.L + l] = (uint16_t)code;
+        }
+    }
+}
+
+// Units per query-hash block: the most (up to kQhashVecs / G query vectors)
+// that still leave at least two blocks per SM.
+static int qhash_units_per_block(const Shape &s, int G)
+{
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                      cudaSuccess)
+            sms = 148;
+    }
+    const int TB = qhash_tables_per_block(s.K);
+    const long long ntiles = (s.L + TB - 1) / TB, units = (long long)s.B * s.Hkv;
+    int ug = 1;
+    while (2 * ug * G <= kQhashVecs && ntiles * ((units + 2 * ug - 1) / (2 * ug)) >= 2LL * sms) ug *= 2;
+    return ug;
 }
 
 // ------------------------------------------------------- scan helpers -------
@@ -1861,10 +1883,10 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     const int units = s.B * s.Hkv;
     cudaError_t e;
     {
-        const int TB = qhash_tables_per_block(s.K);
-        dim3 grid((s.L + TB - 1) / TB, units);
+        const int TB = qhash_tables_per_block(s.K), ug = qhash_units_per_block(s, G);
+        dim3 grid((s.L + TB - 1) / TB, (units + ug - 1) / ug);
         e = launch_pdl(qhash_kernel<G>, grid, dim3(256), 0, st, s, q, W,
-                       (const uint16_t *)(dbg ? dbg->qcodes_in : nullptr), ws.qcodes, ws.status);
+                       (const uint16_t *)(dbg ? dbg->qcodes_in : nullptr), ws.qcodes, ws.status, ug);
         if (e != cudaSuccess) return e;
     }
     ScanOut so{ws.cand, ws.cnt, dbg ? dbg->member_out : nullptr, ws.status, 1u};
@@ -1972,16 +1994,17 @@ cudaError_t launch_decode(const Shape &s, const uint16_t *q, const uint16_t *W, 
 cudaError_t launch_hash_queries(const Shape &s, const uint16_t *q, const uint16_t *W, uint16_t *qcodes,
                                 cudaStream_t st)
 {
-    const int TB = qhash_tables_per_block(s.K);
-    dim3 grid((s.L + TB - 1) / TB, s.B * s.Hkv);
+    const int TB = qhash_tables_per_block(s.K), units = s.B * s.Hkv;
     const uint16_t *none = nullptr;
     int32_t *no_status = nullptr;
+    if (s.G != 1 && s.G != 2 && s.G != 4 && s.G != 8) return cudaErrorInvalidValue;
+    const int ug = qhash_units_per_block(s, s.G);
+    dim3 grid((s.L + TB - 1) / TB, (units + ug - 1) / ug);
     switch (s.G) {
-    case 1: return launch_pdl(qhash_kernel<1>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status);
-    case 2: return launch_pdl(qhash_kernel<2>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status);
-    case 4: return launch_pdl(qhash_kernel<4>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status);
-    case 8: return launch_pdl(qhash_kernel<8>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status);
-    default: return cudaErrorInvalidValue;
+    case 1: return launch_pdl(qhash_kernel<1>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug);
+    case 2: return launch_pdl(qhash_kernel<2>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug);
+    case 4: return launch_pdl(qhash_kernel<4>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug);
+    default: return launch_pdl(qhash_kernel<8>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug);
     }
 }
 
