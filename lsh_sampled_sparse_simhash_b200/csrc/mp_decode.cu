@@ -1596,13 +1596,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_planes_kernel(const __
 
 // ----------------------------------------------------------------- merge ----
 constexpr int kMergeBatch = 8;  // splits per warp whose loads are in flight together
+constexpr int kMergeWarps = 8;  // 8 kMergeBatch = 64 splits per head in one round of loads
 
-// One block of 128 threads per (b, q head).  Warp w folds splits w, w + 4,
-// ... (lane = 4 output dims) with a running maximum, rescaling its sums when
-// the maximum moves, so all loads go out in one pass (unrolled); the four
-// warps' (m, l, acc) are then combined in shared memory.
+// One block of kMergeWarps warps per (b, q head).  Warp w folds splits w,
+// w + kMergeWarps, ... (lane = 4 output dims) with a running maximum,
+// rescaling its sums when the maximum moves, so all loads go out in one pass
+// (unrolled); the warps' (m, l, acc) are then combined in shared memory.
 template <int G>
-__global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t *__restrict__ seq_lens,
+__global__ void __launch_bounds__(32 * kMergeWarps) merge_kernel(Shape s, const int32_t *__restrict__ seq_lens,
                                                          int max_len, int nchunk, int span, int subs,
                                                          int ngroups, int chunk_tokens,
                                                          const float *__restrict__ pm,
@@ -1611,9 +1612,9 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
                                                          const int32_t *__restrict__ cnt, float *out,
                                                          float *lse, int32_t *n_sampled, int has_d)
 {
-    __shared__ float red_m[4], red_l[4];
-    __shared__ int red_n[4];
-    __shared__ float4 red_acc[4][32];
+    __shared__ float red_m[kMergeWarps], red_l[kMergeWarps];
+    __shared__ int red_n[kMergeWarps];
+    __shared__ float4 red_acc[kMergeWarps][32];
     const int bh = blockIdx.x;
     const int b = bh / s.Hq, h = bh % s.Hq, kvh = h / G, g = h % G;
     const int unit = b * s.Hkv + kvh;
@@ -1637,12 +1638,12 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
     // loads of kMergeBatch splits go out together before any of them is used
     float m = -INFINITY, Ls = 0.f;
     float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = warp; j0 <= dsp; j0 += 4 * kMergeBatch) {
+    for (int j0 = warp; j0 <= dsp; j0 += kMergeWarps * kMergeBatch) {
         float mj[kMergeBatch], lj[kMergeBatch];
         float4 aj[kMergeBatch];
 #pragma unroll
         for (int i = 0; i < kMergeBatch; i++) {
-            const int j = j0 + 4 * i;
+            const int j = j0 + kMergeWarps * i;
             mj[i] = -INFINITY;
             lj[i] = 0.f;
             aj[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1655,7 +1656,7 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
         }
 #pragma unroll
         for (int i = 0; i < kMergeBatch; i++)
-            if (!live(j0 + 4 * i)) mj[i] = -INFINITY;
+            if (!live(j0 + kMergeWarps * i)) mj[i] = -INFINITY;
 #pragma unroll
         for (int i = 0; i < kMergeBatch; i++) {
             if (mj[i] == -INFINITY) continue;  // an empty or absent split (uniform across the warp)
@@ -1686,12 +1687,14 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
     }
     __syncthreads();
     if (warp == 0) {
-        const float M = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+        float M = red_m[0];
+#pragma unroll
+        for (int w = 1; w < kMergeWarps; w++) M = fmaxf(M, red_m[w]);
         float Lt = 0.f;
         float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < 4; w++) {
+            for (int w = 0; w < kMergeWarps; w++) {
                 if (red_m[w] == -INFINITY) continue;
                 const float f = fast_exp2(red_m[w] - M);
                 const float4 t = red_acc[w][lane];
@@ -1710,7 +1713,10 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(Shape s, const int32_t 
         reinterpret_cast<float4 *>(out + (size_t)bh * kHeadDim)[lane] = o;
         if (lane == 0) {
             lse[bh] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;  // partials keep log2 units
-            n_sampled[bh] = red_n[0] + red_n[1] + red_n[2] + red_n[3];
+            int nt = 0;
+#pragma unroll
+            for (int w = 0; w < kMergeWarps; w++) nt += red_n[w];
+            n_sampled[bh] = nt;
         }
     }
 }
@@ -1966,7 +1972,7 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     }
     // partials: per chunk (fused) or per split of the plan, then the exact set
     const int m_span = fused ? 1 : sp.span, m_subs = fused ? 1 : sp.subs, m_groups = fused ? nchunk : sp.ngroups;
-    e = launch_pdl(merge_kernel<G>, dim3(s.B * s.Hq), dim3(kHeadDim), 0, st, s, seq_lens, max_len, nchunk, m_span,
+    e = launch_pdl(merge_kernel<G>, dim3(s.B * s.Hq), dim3(32 * kMergeWarps), 0, st, s, seq_lens, max_len, nchunk, m_span,
                    m_subs, m_groups, C, (const float *)ws.pm, (const float *)ws.pl, (const float *)ws.pacc,
                    (const int32_t *)ws.cnt, out, lse, n_sampled, fused ? 0 : 1);
     if (e != cudaSuccess) return e;
