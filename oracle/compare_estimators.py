@@ -15,6 +15,7 @@ and reports the relative L2 error against exact attention and the fraction
 of planted needle keys each token set contains.
 
     python -m oracle.compare_estimators --workload llama8b_16k --units 2
+    python -m oracle.compare_estimators --workload tiny --units 1 --sweep
 """
 from __future__ import annotations
 
@@ -64,9 +65,13 @@ def compare_unit(w, q_bits, W_bits, b: int, kvh: int, n: int, rng: np.random.Gen
     return rows
 
 
-def compare(name: str, units: int, seed: int = 0):
+def compare(name: str, units: int, seed: int = 0, **overrides):
+    """Rows of compare_unit over `units` evenly picked units of workload
+    `name` (fields replaced by `overrides`, e.g. k_bits, n_tables)."""
     import workloads
     w = workloads.get(name)
+    if overrides:
+        w = w.with_(**overrides)
     q_bits = workloads.queries_of(w)
     W_bits = workloads.hyperplanes_of(w)
     lens = workloads.seq_lens_of(w)
@@ -91,15 +96,40 @@ def summary(rows):
     return out
 
 
+SWEEP_K = (6, 8, 10)
+SWEEP_L = (25, 50, 75, 100, 150, 200)
+
+
+def sweep(name: str, units: int, seed: int = 0, ks=SWEEP_K, ls=SWEEP_L):
+    """Budget, errors and needle recall of the three estimators over a grid
+    of (K bits, L tables) on one workload: more tables sample more tokens,
+    more bits per table fewer."""
+    out = {}
+    for K in ks:
+        for L in ls:
+            _, rows = compare(name, units, seed, k_bits=K, n_tables=L)
+            out[(K, L)] = summary(rows)
+    return out
+
+
 def main():
     p = argparse.ArgumentParser()
     p.add_argument("--workload", action="append", default=None)
     p.add_argument("--units", type=int, default=2)
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--sweep", action="store_true", help="grid over K in 6, 8, 10 and L in 25 .. 200")
     args = p.parse_args()
     build()
     res = {}
     for name in args.workload or ["tiny", "llama8b_16k"]:
+        if args.sweep:
+            print(f"{name}: K L budget/N magicpig topk oracle_sampling recall_magicpig recall_topk", flush=True)
+            for (K, L), r in sweep(name, args.units, args.seed).items():
+                print(f"{name}: {K} {L} {r['budget_fraction']:.4f} {r['magicpig']['mean_rel_l2']:.3g} "
+                      f"{r['topk']['mean_rel_l2']:.3g} {r['oracle_sampling']['mean_rel_l2']:.3g} "
+                      f"{r['needle_recall']['magicpig']:.2f} {r['needle_recall']['topk']:.2f}", flush=True)
+                res[(name, K, L)] = r
+            continue
         w, rows = compare(name, args.units, args.seed)
         res[name] = summary(rows)
         print(name, json.dumps(res[name]), flush=True)

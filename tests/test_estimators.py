@@ -72,3 +72,18 @@ def test_comparison_runs_on_the_single_head_workload():
     assert s["needle_recall"]["magicpig"] == 1.0
     assert s["magicpig"]["mean_rel_l2"] < 1e-2
     assert 0 < s["budget_fraction"] < 0.5
+
+
+def test_budget_grows_with_tables_and_shrinks_with_bits():
+    """The sampling probability u = P[Bin(L, p^K) >= 2] grows with the number
+    of tables L and falls with the bits per table K, and so must MagicPIG's
+    budget |S_h| on the same keys (the codes of the first L' tables are the
+    same for every L >= L' only in distribution, so the check is on the
+    spread-out grid points)."""
+    from oracle.compare_estimators import sweep
+    r = sweep("tiny", 1, ks=(6, 10), ls=(25, 200))
+    b = {kl: v["budget_fraction"] for kl, v in r.items()}
+    assert b[(6, 200)] > b[(6, 25)] and b[(10, 200)] > b[(10, 25)]
+    assert b[(6, 25)] > b[(10, 25)] and b[(6, 200)] > b[(10, 200)]
+    # needles are q + small noise: every setting keeps them
+    assert all(v["needle_recall"]["magicpig"] == 1.0 for v in r.values())
