@@ -29,7 +29,9 @@
 //
 // Column groups: W has L*K rows (hyperplanes); a group of at most 640 rows
 // (608 for K = 8, L = 75) stays resident; K = 10, L = 150 uses 3 groups of
-// <= 512 and re-reads each key tile once per group.
+// <= 512.  Each block keeps one group for the whole launch, and the blocks of
+// the different groups walk the same key tiles side by side, so a key tile
+// is read from DRAM once and from L2 by the other groups' blocks.
 //
 // Every wait on an mbarrier is bounded (1 s of %globaltimer); on expiry the
 // kernel records MP_ERR_CUDA in the status word, skips the rest of its work,
@@ -71,7 +73,7 @@ struct Params {
     int ngroups;
     int gsize;       // columns per group (multiple of 32)
     int gpad_max;    // padded width of the widest group (multiple of 32)
-    int total_items; // ngroups * units * n_mt
+    int total_items; // units * n_mt (every block hashes its items for its own column group)
     uint32_t kmagic; // floor(2^32 / K) + 1: c / K = umulhi(c, kmagic) while c K < 2^32
     uint32_t hmagic; // floor(2^32 / Hkv) + 1: batch of unit u = umulhi(u, hmagic)
 };
@@ -243,48 +245,45 @@ __device__ __forceinline__ Item make_item(const Params &p, int group, int unit, 
     return r;
 }
 
+// A block keeps one column group for the whole launch: block x takes group
+// x % ngroups and, of the (unit, tile) items, x / ngroups + k S for k = 0,
+// 1, ... (S = gridDim.x / ngroups; the grid is a multiple of ngroups).  The
+// ngroups blocks x = ngroups j + g walk the same key tiles side by side, so
+// each tile comes from DRAM once and from L2 for the other groups, and W is
+// loaded once per block.
+__device__ __forceinline__ int block_group(const Params &p) { return (int)blockIdx.x % p.ngroups; }
+__device__ __forceinline__ int item_stride(const Params &p) { return (int)gridDim.x / p.ngroups; }
+
 __device__ __forceinline__ Item item_of(const Params &p, int it, const int *lens_sh)
 {
-    const int units = p.s.B * p.s.Hkv;
-    const int rem = it % (units * p.n_mt);
-    return make_item(p, it / (units * p.n_mt), rem / p.n_mt, rem % p.n_mt, lens_sh);
+    return make_item(p, block_group(p), it / p.n_mt, it % p.n_mt, lens_sh);
 }
 
-// The items of this block, blockIdx.x + k gridDim.x for k = 0, 1, ..., in
-// (group, unit, tile) form, advanced with carries instead of divisions.
+// The (unit, tile) items of this block, advanced with carries instead of
+// divisions.
 struct ItemIter {
     int it, group, unit, mt;
-    int dg, du, dm;  // gridDim.x in the same mixed radix
+    int step, du, dm;  // the stride in the same mixed radix
     __device__ __forceinline__ explicit ItemIter(const Params &p)
     {
-        const int units = p.s.B * p.s.Hkv;
-        it = blockIdx.x;
+        group = block_group(p);
+        it = (int)blockIdx.x / p.ngroups;
         mt = it % p.n_mt;
-        unit = (it / p.n_mt) % units;
-        group = it / (p.n_mt * units);
-        const int g = gridDim.x;
-        dm = g % p.n_mt;
-        du = (g / p.n_mt) % units;
-        dg = g / (p.n_mt * units);
+        unit = it / p.n_mt;
+        step = item_stride(p);
+        dm = step % p.n_mt;
+        du = step / p.n_mt;
     }
     __device__ __forceinline__ bool live(const Params &p) const { return it < p.total_items; }
     __device__ __forceinline__ void next(const Params &p)
     {
-        const int units = p.s.B * p.s.Hkv;
-        it += gridDim.x;
+        it += step;
         mt += dm;
-        int carry = 0;
+        unit += du;
         if (mt >= p.n_mt) {
             mt -= p.n_mt;
-            carry = 1;
+            unit++;
         }
-        unit += du + carry;
-        carry = 0;
-        if (unit >= units) {
-            unit -= units;
-            carry = 1;
-        }
-        group += dg + carry;
     }
     __device__ __forceinline__ Item item(const Params &p, const int *lens_sh) const
     {
@@ -502,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // later tiles of this block into L2: the first pass covers 2..kPrefetchAhead
             // items ahead, every later pass the one newly kPrefetchAhead ahead
             for (int ahead = first_pass ? 2 : kPrefetchAhead; ahead <= kPrefetchAhead; ahead++) {
-                const int it2 = iter.it + ahead * (int)gridDim.x;
+                const int it2 = iter.it + ahead * item_stride(p);
                 if (it2 < p.total_items) {
                     const Item i2 = item_of(p, it2, lens_sh);
                     if (!i2.skip) {
@@ -672,7 +671,7 @@ cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint
     p.ngroups = (s.LK + kMaxGroupCols - 1) / kMaxGroupCols;
     p.gsize = (((s.LK + p.ngroups - 1) / p.ngroups) + 31) & ~31;
     p.gpad_max = p.gsize;
-    p.total_items = p.ngroups * s.B * s.Hkv * p.n_mt;
+    p.total_items = s.B * s.Hkv * p.n_mt;  // (unit, tile) items, each hashed for every group
     p.kmagic = (uint32_t)((1ull << 32) / (uint64_t)s.K) + 1u;
     p.hmagic = (uint32_t)((1ull << 32) / (uint64_t)s.Hkv) + 1u;
     CUtensorMap mk, mw;
@@ -681,7 +680,7 @@ cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint
     const int smem = 1024 + 2 * p.gpad_max * 128 + kStages * kTileBytes;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(hash_keys_tc_kernel), smem);
     if (e != cudaSuccess) return e;
-    const int grid = min(num_sms(), p.total_items);
+    const int grid = p.ngroups * min(num_sms() / p.ngroups, p.total_items);
     return launch_pdl(hash_keys_tc_kernel, dim3(grid), dim3(kThreads), smem, st, mk, mw, p);
 }
 
