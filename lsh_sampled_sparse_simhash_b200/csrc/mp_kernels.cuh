@@ -41,9 +41,11 @@ bool encode_tensor_map(CUtensorMap *m, CUtensorMapDataType type, int rank, const
 cudaError_t ensure_smem(const void *func, int bytes);
 
 // Launches with programmatic stream serialization: the kernel may be
-// scheduled while its predecessor in the stream is still running; every
-// kernel of this library calls grid_dependency_wait() before touching
-// memory, so ordering is unchanged and only the launch latency is hidden.
+// scheduled while its predecessor in the stream is still running.  Every
+// kernel of this library waits for its predecessor (griddepcontrol.wait)
+// before it reads anything the predecessor writes and before it writes global
+// memory, and lets its own successor launch only after that wait, so ordering
+// is unchanged and only launch latency is hidden (see grid_wait()).
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                        Args... args)
