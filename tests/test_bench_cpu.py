@@ -1,0 +1,59 @@
+"""Host-side pieces of bench.py that decide what the JSON line reports: the
+code fingerprint that keys the committed DRAM-traffic records (it must follow
+the code and ignore comments and layout), the traffic lookup itself, and the
+packing of the end-to-end step's inputs into one buffer."""
+import json
+import os
+
+import numpy as np
+
+import bench
+
+
+def _write(tmp_path, name, text):
+    p = tmp_path / name
+    p.write_text(text)
+    return str(p)
+
+
+def test_fingerprint_ignores_comments_and_whitespace(tmp_path):
+    a = _write(tmp_path, "a.cu", "int f(int x) {\n  return x + 1; // add one\n}\n/* block\n comment */\n")
+    b = _write(tmp_path, "b.cu", "// header\nint f(int x)\n{\n\treturn x + 1;\n}\n")
+    assert bench.code_fingerprint(a) == bench.code_fingerprint(b)
+
+
+def test_fingerprint_follows_the_code(tmp_path):
+    a = _write(tmp_path, "a.cu", "int f(int x) { return x + 1; }\n")
+    b = _write(tmp_path, "b.cu", "int f(int x) { return x + 2; }\n")
+    assert bench.code_fingerprint(a) != bench.code_fingerprint(b)
+
+
+def test_fingerprint_keeps_comment_markers_inside_strings(tmp_path):
+    a = _write(tmp_path, "a.cu", 'const char *s = "a // b";\n')
+    b = _write(tmp_path, "b.cu", 'const char *s = "a ";\n')
+    assert bench.code_fingerprint(a) != bench.code_fingerprint(b)
+
+
+def test_traffic_lookup_follows_the_fingerprint():
+    """A committed record is reported while its source's code is the one the
+    capture was taken on, and null once the code has changed."""
+    recs = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    assert recs
+    for key, rec in recs.items():
+        kernel, rest = key.split("@")
+        workload, layout = rest.split(":")
+        src = os.path.join(bench.ROOT, rec["source"])
+        fresh = bench.code_fingerprint(src) == rec["code_sha256"]
+        assert bench.traffic_record(kernel, workload, layout) == (rec["bytes_per_launch"] if fresh else None), key
+    assert bench.traffic_record("hash_keys", "no_such_workload", "bytes") is None
+
+
+def test_packed_inputs_round_trip():
+    arrays = [np.arange(5, dtype=np.int16), np.arange(7, dtype=np.int32) - 3, np.linspace(0, 1, 3, dtype=np.float32)]
+    buf = bench._pack_host(arrays)
+    off = 0
+    for a in arrays:
+        assert off % 256 == 0
+        np.testing.assert_array_equal(buf[off:off + a.nbytes].view(a.dtype), a)
+        off += (a.nbytes + 255) // 256 * 256
+    assert buf.nbytes == off
