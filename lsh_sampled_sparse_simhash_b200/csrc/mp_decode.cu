@@ -695,20 +695,25 @@ struct LogU {
     float K, L, lnC2, a3, a4, a5;
 };
 
+// log u for a pair of cosine c.  The plain log and exp are the hardware
+// approximations (__logf, __expf: a few ulp, a few 1e-6 relative at these
+// arguments), which moves log u by ~1e-5 at most, far inside the output
+// tolerance; acos and the log1p / expm1 terms, where cancellation matters,
+// keep the accurate library functions.
 __device__ __forceinline__ float log_sampling_prob(float c, const LogU &u)
 {
     c = fminf(1.f, fmaxf(-1.f, c));
     float p = 1.f - acosf(c) * 0.318309886183790671538f;
     p = fmaxf(p, 1e-30f);
-    const float lx = u.K * logf(p);
-    const float x = expf(lx);
+    const float lx = u.K * __logf(p);
+    const float x = __expf(lx);
     if (x < 1e-3f) {
         const float r = x / (1.f - x);
         const float tail = u.a3 * r * (1.f + u.a4 * r * (1.f + u.a5 * r));
         return u.lnC2 + 2.f * lx + (u.L - 2.f) * log1pf(-x) + log1pf(tail);
     }
     const float y = (u.L - 1.f) * log1pf(-x) + log1pf((u.L - 1.f) * x);
-    return logf(-expm1f(y));
+    return __logf(-expm1f(y));
 }
 
 constexpr int kAttThreads = 128;
