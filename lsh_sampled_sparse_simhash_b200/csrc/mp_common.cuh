@@ -135,23 +135,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t a, uint32_t parity)
     return mbar_try_wait(a, parity) || mbar_wait_bounded_slow(a, parity);
 }
 
-// One contiguous global -> shared copy on the async (TMA) engine, completing
-// `bytes` of the transaction count of mbarrier `bar`.  dst, src and bytes are
-// multiples of 16.
-__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-
-// Pulls `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
-// without waiting for it: the later real load then finds it there.
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 // Orders this thread's earlier generic-proxy shared-memory accesses before its
 // later async-proxy ones (a buffer that was read is about to be refilled).
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
