@@ -71,21 +71,31 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
         const int part = tid & 3;  // quarter of the dims
         constexpr int kSlots = kAppendThreads / 4;
         const int npairs = ncol * s.Hkv;
+        // this lane's quarter of its head's key, in registers: the slot
+        // stride is a multiple of Hkv whenever Hkv divides kSlots, and then
+        // the head of a lane never changes between its pairs
+        float kx[32];
+        int hcur = -1;
         for (int pi = tid >> 2; pi < (npairs + kSlots - 1) / kSlots * kSlots; pi += kSlots) {
             const bool valid = pi < npairs;
             const int cl = valid ? pi / s.Hkv : 0, h = valid ? pi - cl * s.Hkv : 0;
+            if (valid && h != hcur) {
+                const float *xp = xs + h * (kHeadDim + 4) + part * 33;
+#pragma unroll
+                for (int i = 0; i < 32; i++) kx[i] = xp[i];
+                hcur = h;
+            }
             float dot = 0.f;
             if (valid) {
                 const uint4 *wr = reinterpret_cast<const uint4 *>(wsm + (size_t)cl * kHeadDim + part * 32);
-                const float *xp = xs + h * (kHeadDim + 4) + part * 33;
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
                     const uint4 w = wr[j];
                     const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
-                        dot = fmaf(xp[j * 8 + 2 * e], bf16_lo(wv[e]), dot);
-                        dot = fmaf(xp[j * 8 + 2 * e + 1], bf16_hi(wv[e]), dot);
+                        dot = fmaf(kx[j * 8 + 2 * e], bf16_lo(wv[e]), dot);
+                        dot = fmaf(kx[j * 8 + 2 * e + 1], bf16_hi(wv[e]), dot);
                     }
                 }
             }
