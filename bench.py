@@ -1,14 +1,22 @@
 #!/usr/bin/env python
 """Benchmark of one LSH-sampled decode layer-step (MagicPIG hot path) on B200.
 
-A step = every row of the hot path over one batch of synthetic input:
-  mp_hash_keys   SimHash of every cached key (tcgen05 tensor-core GEMM with a
-                 sign-packing epilogue),
-  mp_append_token  one new token per sequence (K/V row + codes, length + 1),
-  mp_decode_attend query hash, collision scan + compaction, sampled attention
-                 with the -log u correction, exact sink/window set, LSE merge.
-Metric: decode context tokens scanned per second per layer-step
-(sum over sequences of the post-append length, divided by the step time).
+A step is one decode of every sequence of the batch:
+  mp_append_token   one new token per sequence (K/V row + its SimHash codes,
+                    length + 1),
+  mp_decode_attend  query hash, collision scan + compaction, sampled attention
+                    with the -log u correction, exact sink/window set, LSE merge,
+over the post-append context.  The key-hash build of the cached keys
+(mp_hash_keys, a tcgen05 tensor-core GEMM) is a prefill cost: it is timed on
+its own (`breakdown.hash_*`, against the bf16 tensor peak), except for the
+16k-token Llama-3.1-8B-shaped layer, whose step specification hashes every
+cached key, so there the step is hash + append + decode.
+
+Metric: decode context tokens scanned per second per layer-step: the sum over
+sequences of the post-append length, divided by the step's device time;
+`roofline` is the step's algorithmic HBM bytes (key codes + the unique
+sampled K/V rows + the exact-set rows) over the same time, against the
+measured HBM copy bandwidth.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
@@ -31,13 +39,22 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "llama8b_16k"
+DEFAULT_WORKLOAD = "ragged16"
+HASH_IN_STEP = ("llama8b_16k",)  # workloads whose step hashes every cached key
 FLUSH_BYTES = 256 << 20  # > 126 MB L2
 METRIC = "decode context-tokens scanned/s per layer-step"
 HASH_IMPL = "tcgen05-bf16"   # implementation of mp_hash_keys in this build
+# The pages' own system-level claim, reported as context only (other
+# hardware, other system: CPU-side sampled attention next to GPU attention).
+PAGES_CLAIM = dict(
+    claim="MagicPIG decoding throughput 1.76-4.99x over GPU-only attention",
+    hardware="CPU + GPU: Intel CPUs with AVX512 (AVX512_BF16 for bf16) for the sampled attention; "
+             "GPU model not stated",
+    source="sourcepulse project page, 'Highlighted Details' and 'Quick Start & Requirements'",
+    role="context, not the target")
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
@@ -46,13 +63,14 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-overlap", action="store_true", help="skip the streamed-prefill overlap measurement")
     p.add_argument("--code-layout", default=None, choices=["auto", "bytes", "planes"],
                    help="key-code layout (default: the workload's, i.e. bytes for K=8, planes for K=10)")
     p.add_argument("--no-graph", action="store_true",
                    help="launch every timed step eagerly instead of replaying a captured CUDA graph")
     p.add_argument("--decode-path", default="auto", choices=["auto", "split", "fused"],
                    help="decode kernels: auto, split (scan then attention) or fused (one kernel; bit planes)")
-    return p.parse_args()
+    return p.parse_args(argv)
 
 
 def load_peaks():
@@ -86,8 +104,39 @@ def workload_for_rank(name, rank, code_layout=None):
     return w.with_(seed=w.seed + 7919 * rank) if rank else w
 
 
+def hash_in_step(w) -> bool:
+    return w.name in HASH_IN_STEP
+
+
 def step_tokens(lens_after):
     return int(np.sum(lens_after))
+
+
+def decode_bytes(w, lens_after, union_rows):
+    """Algorithmic HBM bytes of one decode over post-append lengths: the key
+    codes of every (token, kv head) (L*K/8 bytes each), the unique sampled
+    K/V rows and the exact-set rows (512 bytes per row: k + v, bf16)."""
+    LK = w.n_tables * w.k_bits
+    code_bytes = int(np.sum(lens_after)) * w.n_kv_heads * LK // 8
+    d_rows = sum(min(w.sink, int(n)) + int(n) - max(min(w.sink, int(n)), int(n) - w.window)
+                 for n in lens_after) * w.n_kv_heads
+    return code_bytes + (union_rows + d_rows) * 2 * w.head_dim * 2, code_bytes, d_rows
+
+
+def step_description(w):
+    if hash_in_step(w):
+        return "hash all cached keys + append 1 token/sequence + LSH-sampled decode"
+    return "append 1 token/sequence + LSH-sampled decode (key-hash build timed apart)"
+
+
+def config_of(w):
+    """The workload, identical on both arms (no launch or kernel-path keys)."""
+    return dict(workload=w.name, batch=w.batch, q_heads=w.n_q_heads, kv_heads=w.n_kv_heads,
+                head_dim=w.head_dim, context=w.context, ragged_min=w.ragged_min or None, k_bits=w.k_bits,
+                n_tables=w.n_tables, sink=w.sink, window=w.window, planted_per_kv_head=w.n_planted,
+                code_layout=w.code_layout if w.code_layout != "auto" else ("bytes" if w.k_bits == 8 else "planes"),
+                step=step_description(w),
+                l2="flushed between timed steps (256 MiB write)", parallelism="replicas (1 rank = 1 GPU)")
 
 
 # ------------------------------------------------------------- clocks ----
@@ -177,9 +226,13 @@ class Bench:
         self.tokens = step_tokens(inp["seq_lens"] + 1)
         self.path = {"auto": mp.MP_PATH_AUTO, "split": mp.MP_PATH_SPLIT, "fused": mp.MP_PATH_FUSED}[path]
         self.graph_error = None
+        self.with_hash = hash_in_step(w)
         fused = self.path == mp.MP_PATH_FUSED
-        # hash 1, append 1, decode: qhash + (scan, attention | fused) + merge
-        self.launches_per_step = 2 + (3 if fused else 4)
+        # append 1, decode: qhash + (scan, attention | fused) + merge; hash 1 if in the step
+        self.launches_per_step = 1 + (3 if fused else 4) + (1 if self.with_hash else 0)
+        # prefill: the codes of the cached keys (the step's append adds the new token's)
+        self.hash()
+        torch.cuda.synchronize()
 
     def hash(self):
         self.mp.hash_keys(self.shape, self.K, self.W, self.prefill, self.codes, seq_lens=self.lens0)
@@ -191,11 +244,16 @@ class Bench:
         self.mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
                               self.out, self.lse, self.ns, self.ws, path=self.path)
 
-    def step(self):
-        self.lens.copy_(self.lens0, non_blocking=True)
-        self.hash()
+    def calls(self):
+        """The library calls of one step (the lengths are reset before it)."""
+        if self.with_hash:
+            self.hash()
         self.append()
         self.decode()
+
+    def step(self):
+        self.lens.copy_(self.lens0, non_blocking=True)
+        self.calls()
 
     def union_rows(self):
         """Unique sampled (token, kv head) rows of one decode (for the bytes roofline)."""
@@ -207,38 +265,43 @@ class Bench:
                               self.out, self.lse, self.ns, self.ws, member_out=mem, path=self.path)
         torch.cuda.synchronize()
         m = mem.view(w.batch, w.n_kv_heads, w.group, w.capacity).amax(dim=2)
-        return int(m.sum().item()), float(self.ns.float().mean().item())
+        u = int(m.sum().item())
+        del mem, m
+        return u, float(self.ns.float().mean().item())
 
-    def timed(self, steps, warmup):
-        torch = self.torch
+    def warm(self, warmup):
         for _ in range(warmup):
             self.flush.zero_()
             self.step()
-        torch.cuda.synchronize()
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
-        return ev
+        self.torch.cuda.synchronize()
 
-    def preroll(self, seconds):
+    def events(self, steps, n=2):
+        torch = self.torch
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(n)] for _ in range(steps)]
+
+    def preroll(self, seconds, graph=None):
         torch = self.torch
         t0 = time.perf_counter()
         while time.perf_counter() - t0 < seconds:
             for _ in range(8):
                 self.flush.zero_()
-                self.step()
+                self.lens.copy_(self.lens0, non_blocking=True)
+                if graph is not None:
+                    graph.replay()
+                else:
+                    self.calls()
             torch.cuda.synchronize()
 
     def capture(self):
-        """Captures one step (hash, append, decode: every kernel of the step,
-        programmatic launch edges included) in a CUDA graph; None if capture
-        is not possible here."""
+        """Captures one step's calls (every kernel of the step, programmatic
+        launch edges included) in a CUDA graph; None if capture is not
+        possible here."""
         torch = self.torch
         try:
             torch.cuda.synchronize()
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                self.hash()
-                self.append()
-                self.decode()
+                self.calls()
             torch.cuda.synchronize()
             return g
         except Exception as exc:  # report the eager fallback in the JSON line
@@ -249,7 +312,7 @@ class Bench:
     def run_timed(self, ev, graph=None):
         """K steps, one event pair per step (no events between the calls, which
         would serialise the programmatic launch chain); with a graph, each step
-        is one replay of the captured hash + append + decode."""
+        is one replay of the captured calls.  L2 flushed before each step."""
         for e in ev:
             self.flush.zero_()
             self.lens.copy_(self.lens0, non_blocking=True)
@@ -257,24 +320,26 @@ class Bench:
             if graph is not None:
                 graph.replay()
             else:
-                self.hash()
-                self.append()
-                self.decode()
+                self.calls()
             e[1].record()
 
-    def run_breakdown(self, ev):
-        """K more steps with an event between every call: per-call device time
-        for the roofline of each kernel."""
-        for e in ev:
-            self.flush.zero_()
-            self.lens.copy_(self.lens0, non_blocking=True)
-            e[0].record()
-            self.hash()
-            e[1].record()
-            self.append()
-            e[2].record()
-            self.decode()
-            e[3].record()
+    def run_breakdown(self, steps):
+        """Per-call device times (events around each call, L2 flushed before
+        each call): the key-hash build, the append and the decode."""
+        torch = self.torch
+        res = {"hash": [], "append": [], "decode": []}
+        for _ in range(steps):
+            for name, fn in (("hash", self.hash), ("append", self.append), ("decode", self.decode)):
+                if name == "append":
+                    self.lens.copy_(self.lens0, non_blocking=True)
+                self.flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                res[name].append((e0, e1))
+        torch.cuda.synchronize()
+        return {k: statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in res.items()}
 
     def prefill_overlap(self, iters=10):
         """Streamed prefill beside decoding: a block of R tokens per unit hashed
@@ -323,10 +388,10 @@ class Bench:
     def run_e2e(self, steps, warmup, use_graph=True):
         """Public API with host buffers: per step, one H2D copy of the step's
         inputs (q, k_new, v_new, lengths, packed) from pinned memory, the
-        three calls, and one D2H copy of out / lse / n_sampled (packed) into
-        pinned memory; device-timed.  The H2D copy runs on a second stream
-        next to the hash of the cached keys, which does not read those inputs;
-        the append waits for both."""
+        step's calls, and one D2H copy of out / lse / n_sampled (packed) into
+        pinned memory; device-timed.  When the step hashes the cached keys,
+        the H2D copy runs on a second stream beside that hash (which does not
+        read those inputs) and the append waits for both."""
         torch = self.torch
         hin = torch.from_numpy(self.in_host).pin_memory()
         hout = torch.empty(self.out_dev.shape, dtype=torch.uint8).pin_memory()
@@ -336,11 +401,14 @@ class Bench:
 
         def one_step():
             main = torch.cuda.current_stream()
-            side.wait_stream(main)
-            with torch.cuda.stream(side):
+            if self.with_hash:
+                side.wait_stream(main)
+                with torch.cuda.stream(side):
+                    self.in_dev.copy_(hin, non_blocking=True)
+                self.hash()
+                main.wait_stream(side)
+            else:
                 self.in_dev.copy_(hin, non_blocking=True)
-            self.hash()
-            main.wait_stream(side)
             self.append()
             self.decode()
             hout.copy_(self.out_dev, non_blocking=True)
@@ -444,73 +512,116 @@ def code_fingerprint(path):
 
 # ------------------------------------------------------ oracle (CPU) ----
 
-def oracle_unit_step(inp, w, b, kh):
-    """The fp64 oracle over one (b, kv head) unit of a step: SimHash of the
-    unit's post-append keys, query codes of its heads, then the decode."""
-    import oracle
-    n = int(inp["seq_lens"][b]) + 1
-    G = w.group
-    Kc = inp["K"][b, kh, :n].copy()
-    Kc[n - 1] = inp["k_new"][b, kh]
-    Vc = inp["V"][b, kh, :n].copy()
-    Vc[n - 1] = inp["v_new"][b, kh]
-    kc = oracle.simhash(Kc, inp["W"], w.k_bits, w.n_tables)
-    q = inp["q"][b:b + 1, kh * G:(kh + 1) * G]
-    qc = oracle.simhash(q, inp["W"], w.k_bits, w.n_tables)
-    oracle.decode(q, Kc[None, None], Vc[None, None], kc[None, None], qc, np.array([n], np.int32),
-                  Kbits=w.k_bits, L=w.n_tables, sink=w.sink, window=w.window)
-    return n
+class OracleSample:
+    """The fp64 oracle on (sequence, kv head) units of the workload, one unit
+    per step, cycling over a fixed set of units.  The unit's cached-key codes are the
+    prefill (computed once, untimed, like the GPU arm's key-hash build); a
+    step is what the GPU step does for the unit: SimHash of the appended key
+    (and, for the workload whose step hashes every cached key, of all of
+    them), the query codes of the unit's heads, the collision scan and the
+    estimator over the post-append context.  A unit is 1/Hkv of a sequence,
+    so its tokens count (N_b + 1) / Hkv toward the metric."""
+
+    SAMPLE_UNITS = 4
+
+    def __init__(self, w, inp=None):
+        import oracle
+        from workloads import hyperplanes_of, new_token_of, queries_of, seq_lens_of
+        oracle.build()
+        self.oracle, self.w = oracle, w
+        self.W = inp["W"] if inp is not None else hyperplanes_of(w)
+        self.q = inp["q"] if inp is not None else queries_of(w)
+        self.lens = inp["seq_lens"] if inp is not None else seq_lens_of(w)
+        self.k_new, self.v_new = (inp["k_new"], inp["v_new"]) if inp is not None else new_token_of(w)
+        self.inp = inp
+        # a fixed set of units spread over the batch (and so over its length
+        # mix), each prepared once and then cycled through
+        n = min(self.SAMPLE_UNITS, w.batch * w.n_kv_heads)
+        self.units = [((i * w.batch) // n, i % w.n_kv_heads) for i in range(n)]
+        self.cache = {}
+
+    def _unit(self, b, kh):
+        if (b, kh) not in self.cache:
+            from workloads import unit_keys_values
+            w, n = self.w, int(self.lens[b])
+            if self.inp is not None:
+                Kc, Vc = self.inp["K"][b, kh, :n], self.inp["V"][b, kh, :n]
+            else:
+                Kc, Vc = unit_keys_values(w, self.q, b, kh, n)
+            Kc = np.concatenate([Kc, self.k_new[b, kh][None]])
+            Vc = np.concatenate([Vc, self.v_new[b, kh][None]])
+            codes = None if hash_in_step(w) else self.oracle.simhash(Kc[:n], self.W, w.k_bits, w.n_tables)
+            self.cache[(b, kh)] = (Kc, Vc, codes)
+        return self.cache[(b, kh)]
+
+    def unit_step(self, b, kh):
+        """Timed part of one unit-step; returns its metric tokens."""
+        o, w = self.oracle, self.w
+        Kc, Vc, codes = self._unit(b, kh)
+        n = Kc.shape[0]
+        t0 = time.perf_counter()
+        if codes is None:
+            kc = o.simhash(Kc, self.W, w.k_bits, w.n_tables)
+        else:
+            kc = np.concatenate([codes, o.simhash(Kc[n - 1:], self.W, w.k_bits, w.n_tables)])
+        G = w.group
+        q = self.q[b:b + 1, kh * G:(kh + 1) * G]
+        qc = o.simhash(q, self.W, w.k_bits, w.n_tables)
+        o.decode(q, Kc[None, None], Vc[None, None], kc[None, None], qc, np.array([n], np.int32),
+                 Kbits=w.k_bits, L=w.n_tables, sink=w.sink, window=w.window)
+        return time.perf_counter() - t0, n / w.n_kv_heads
+
+    def describe(self):
+        extra = "SimHash of all its cached keys, " if hash_in_step(self.w) else \
+            "SimHash of the appended key (cached-key codes precomputed, untimed), "
+        lens = [int(self.lens[b]) + 1 for b, _ in self.units]
+        return (f"one (sequence, kv head) unit per step, cycling over units {self.units} (lengths {lens}): "
+                f"{extra}query codes, collision scan and estimator over the post-append context; a unit counts "
+                f"(N_b + 1) / {self.w.n_kv_heads} tokens")
 
 
 def oracle_rate(inp, w, budget_s):
-    """Units of the step in (b, kv head) order until ~budget_s of CPU work;
-    the rate is scaled to the whole step by token count."""
-    import oracle
-    units = [(b, kh) for b in range(w.batch) for kh in range(w.n_kv_heads)]
-    total_unit_tokens = sum(int(inp["seq_lens"][b]) + 1 for b, _ in units)
-    done_tokens, t0, k = 0, time.perf_counter(), 0
-    while time.perf_counter() - t0 < budget_s:
-        b, kh = units[k % len(units)]
-        done_tokens += oracle_unit_step(inp, w, b, kh)
+    """cpu_baseline of our arm: oracle unit-steps until ~budget_s of timed
+    CPU work; tokens/s over the timed parts."""
+    smp = OracleSample(w, inp)
+    done_tokens, busy, k = 0.0, 0.0, 0
+    while busy < budget_s and k < 200:
+        b, kh = smp.units[k % len(smp.units)]
+        dt, tok = smp.unit_step(b, kh)
+        busy += dt
+        done_tokens += tok
         k += 1
-    dt = time.perf_counter() - t0
-    est_step = dt * total_unit_tokens / done_tokens
-    value = step_tokens(inp["seq_lens"] + 1) / est_step
-    sample = (f"{k} (b, kv-head) unit-steps of the {len(units)} in one step ({done_tokens} unit-tokens: SimHash "
-              f"of the unit's keys + collision scan + estimator), scaled to the full step by token count")
-    return value, dict(kind="oracle", cores=oracle.num_threads(), sample=sample, seconds=round(dt, 2))
+    sample = f"{k} unit-steps ({smp.describe()})"
+    return done_tokens / busy, dict(kind="oracle", cores=smp.oracle.num_threads(), sample=sample,
+                                   seconds=round(busy, 2))
 
 
 def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands, on the host cores,
+    each step one bounded sample of the workload (one unit-step); rank 0
+    only."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import oracle
-    from workloads import make_inputs
-    oracle.build()
-    w = workload_for_rank(args.workload, 0)
-    inp = make_inputs(w)
-    G = w.group
-    units = [(b, kh) for b in range(w.batch) for kh in range(w.n_kv_heads)]
-    total_unit_tokens = sum(int(inp["seq_lens"][b]) + 1 for b, _ in units)
-    rates = []
+    w = workload_for_rank(args.workload, 0, args.code_layout)
+    smp = OracleSample(w)
+    times, toks = [], []
     for i in range(args.warmup + args.steps):
-        b, kh = units[i % len(units)]
-        t0 = time.perf_counter()
-        n = oracle_unit_step(inp, w, b, kh)
-        dt = time.perf_counter() - t0
+        b, kh = smp.units[i % len(smp.units)]
+        dt, tok = smp.unit_step(b, kh)
         if i >= args.warmup:
-            rates.append(step_tokens(inp["seq_lens"] + 1) / (dt * total_unit_tokens / n))
-    value = statistics.mean(rates)
+            times.append(dt)
+            toks.append(tok)
+    value = sum(toks) / sum(times)
     unit = "tokens/s"
     line = dict(impl="reference", metric=METRIC, value=value, unit=unit, n_gpus=args.gpus, steps=args.steps,
-                warmup=args.warmup, ms_per_step=1e3 * step_tokens(inp["seq_lens"] + 1) / value,
-                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
-                config=config_of(w),
-                cpu_baseline=dict(value=value, unit=unit, cores=oracle.num_threads(), kind="oracle",
-                                  sample="each step: one (b, kv-head) unit (hash of its keys + collision scan "
-                                         "+ estimator), scaled to the full step by token count"),
-                e2e=dict(value=value, unit=unit, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+                warmup=args.warmup, ms_per_step=1e3 * statistics.mean(times), higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic", config=config_of(w),
+                step_sample=smp.describe(),
+                cpu_baseline=dict(value=value, unit=unit, cores=smp.oracle.num_threads(), kind="oracle",
+                                  sample=smp.describe()),
+                e2e=dict(value=value, unit=unit, h2d_bytes_per_step=0, d2h_bytes_per_step=0),
+                context=PAGES_CLAIM)
     print(json.dumps(line, default=_jsonable), flush=True)
 
 
@@ -518,15 +629,6 @@ def _jsonable(o):
     if hasattr(o, "item"):
         return o.item()
     raise TypeError(type(o).__name__)
-
-
-def config_of(w):
-    return dict(workload=w.name, batch=w.batch, q_heads=w.n_q_heads, kv_heads=w.n_kv_heads,
-                head_dim=w.head_dim, context=w.context, ragged_min=w.ragged_min or None, k_bits=w.k_bits,
-                n_tables=w.n_tables, sink=w.sink, window=w.window, planted_per_kv_head=w.n_planted,
-                code_layout=w.code_layout if w.code_layout != "auto" else ("bytes" if w.k_bits == 8 else "planes"),
-                step="hash all cached keys + append 1 token/sequence + LSH-sampled decode",
-                l2="flushed between timed steps (256 MiB write)", parallelism="replicas (1 rank = 1 GPU)")
 
 
 # --------------------------------------------------------------- main ----
@@ -558,15 +660,16 @@ def main():
         if world > 1:
             dist.barrier()
 
-    ev = bench.timed(args.steps, args.warmup)
+    bench.warm(args.warmup)
     graph = None if args.no_graph else bench.capture()
     for _ in range(3 if graph is not None else 0):  # warm replays
         bench.flush.zero_()
         bench.lens.copy_(bench.lens0, non_blocking=True)
         graph.replay()
+    ev = bench.events(args.steps)
     clocks = ClockSampler(local if world > 1 else 0)
     clocks.start()
-    bench.preroll(0.5)  # untimed steps so the sampler sees the clocks under this load
+    bench.preroll(0.5, graph)  # untimed steps so the sampler sees the clocks under this load
     barrier()
     torch.cuda.synchronize()
     bench.run_timed(ev, graph)
@@ -574,12 +677,7 @@ def main():
     barrier()
     clk = clocks.stop()
     step_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    evb = bench.timed(args.steps, 0)
-    bench.run_breakdown(evb)
-    torch.cuda.synchronize()
-    hash_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evb)
-    append_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evb)
-    decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evb)
+    per_call = bench.run_breakdown(args.steps)
     total_ms, all_tokens = reduce_over_ranks(sum(step_ms), bench.tokens * args.steps, device, world)
     value = all_tokens / (total_ms / 1e3)
 
@@ -595,45 +693,65 @@ def main():
 
     if rank == 0:
         peaks = load_peaks()
-        B = w.batch
+        layout = config_of(w)["code_layout"]
         lens_after = bench.inp["seq_lens"] + 1
+        dec_bytes, code_bytes, d_rows = decode_bytes(w, lens_after, union)
         LK = w.n_tables * w.k_bits
-        code_bytes = int(lens_after.sum()) * w.n_kv_heads * LK // 8
-        d_rows = sum(min(w.sink, n) + n - max(min(w.sink, n), n - w.window) for n in lens_after) * w.n_kv_heads
-        dec_bytes = code_bytes + (union + d_rows) * 2 * w.head_dim * 2
         hash_rows = int(bench.inp["seq_lens"].sum()) * w.n_kv_heads
         hash_flops = 2.0 * hash_rows * w.head_dim * LK
+        hash_ms, append_ms, decode_ms = per_call["hash"], per_call["append"], per_call["decode"]
         if HASH_IMPL.startswith("tcgen05"):
             hash_bound, hash_peak, hash_unit = "tensor", peaks["bf16"], "TFLOP/s"
         else:  # fp32 FMA pipe: 148 SMs x 128 lanes x 2 flop x max SM clock
             hash_bound, hash_peak, hash_unit = "alu", 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12, "TFLOP/s"
-        hash_roof = dict(kernel="mp_hash_keys", bound=hash_bound, achieved=hash_flops / (hash_ms / 1e3) / 1e12,
-                         peak=hash_peak, unit=hash_unit, algorithmic=hash_flops, units=f"{hash_rows} key rows",
-                         traffic=traffic_record("hash_keys", w.name, config_of(w)["code_layout"]))
+        hash_roof = dict(kernel="mp_hash_keys (tcgen05 key-hash build)", bound=hash_bound,
+                         achieved=hash_flops / (hash_ms / 1e3) / 1e12, peak=hash_peak, unit=hash_unit,
+                         peak_source=peaks["source"] + " bf16 burst", algorithmic=hash_flops,
+                         units=f"{hash_rows} key rows x {LK} columns",
+                         traffic=traffic_record("hash_keys", w.name, layout))
         hash_roof["frac"] = hash_roof["achieved"] / hash_roof["peak"]
-        dec_roof = dict(kernel="mp_decode_attend", bound="hbm", achieved=dec_bytes / (decode_ms / 1e3) / 1e9,
-                        peak=peaks["hbm"], unit="GB/s", algorithmic=dec_bytes,
-                        units=f"{int(lens_after.sum())} tokens x {w.n_kv_heads} kv heads; {union} union rows",
-                        traffic=traffic_record("decode", w.name, config_of(w)["code_layout"]))
+        dec_units = f"{int(lens_after.sum())} tokens x {w.n_kv_heads} kv heads; {union} union rows; {d_rows} exact rows"
+        dec_roof = dict(kernel="mp_decode_attend (qhash + scan + attend + merge)", bound="hbm",
+                        achieved=dec_bytes / (decode_ms / 1e3) / 1e9, peak=peaks["hbm"], unit="GB/s",
+                        algorithmic=dec_bytes, units=dec_units,
+                        traffic=traffic_record("decode", w.name, layout))
         dec_roof["frac"] = dec_roof["achieved"] / dec_roof["peak"]
         dec_roof["frac_of_nominal_8tbs"] = dec_roof["achieved"] / 8000.0  # nominal HBM3e figure, for context
-        dominant = hash_roof if hash_ms >= decode_ms else dec_roof
-        roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
-        roofline["kernel"] = dominant["kernel"]
-        roofline["peak_source"] = peaks["source"]
+        ms_step = total_ms / args.steps
+        if bench.with_hash:
+            # the step's largest part is the hash; the HBM-bound decode is
+            # reported from its own events (breakdown loop)
+            roofline = {k: dec_roof[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+            roofline["kernel"] = dec_roof["kernel"] + ", timed alone"
+        else:
+            ach = dec_bytes / (ms_step / 1e3) / 1e9
+            roofline = dict(bound="hbm", achieved=ach, peak=peaks["hbm"], unit="GB/s", frac=ach / peaks["hbm"],
+                            traffic=dec_roof["traffic"],
+                            kernel="decode step: mp_append_token + mp_decode_attend (qhash + scan + attend + "
+                                   "merge), timed over the timed region")
+        roofline["peak_source"] = peaks["source"] + " HBM copy"
+        roofline["algorithmic_bytes"] = dec_bytes
+        roofline["bytes"] = dict(codes=code_bytes, union_rows=union, exact_rows=d_rows, row_bytes=2 * w.head_dim * 2)
+        roofline["frac_of_nominal_8tbs"] = roofline["achieved"] / 8000.0
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
-                    warmup=args.warmup, ms_per_step=total_ms / args.steps, higher_is_better=True,
+                    warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype="bf16-in/fp32-acc", data="synthetic",
-                    config=dict(config_of(w), decode_path=args.decode_path,
-                                launch="cuda-graph replay per step" if graph is not None else
+                    config=config_of(w),
+                    launch=dict(decode_path=args.decode_path,
+                                mode="cuda-graph replay per step" if graph is not None else
                                 "eager launches" + (f" ({bench.graph_error})" if bench.graph_error else "")),
                     roofline=roofline,
                     breakdown=dict(hash_ms=hash_ms, append_ms=append_ms, decode_ms=decode_ms,
+                                   hash_in_step=bench.with_hash,
                                    hash_roofline=hash_roof, decode_roofline=dec_roof,
                                    decode_only_tokens_per_s=bench.tokens / (decode_ms / 1e3),
-                                   mean_sampled_per_head=mean_ns, union_rows=union),
-                    gpu_launches=bench.launches_per_step * args.steps, clocks=clk, e2e=e2e)
-        line["prefill_overlap"] = bench.prefill_overlap()
+                                   mean_sampled_per_head=mean_ns, union_rows=union,
+                                   note="per-call times: events around each call alone, L2 flushed before "
+                                        "each; the step is one graph replay with the launches overlapped"),
+                    gpu_launches=bench.launches_per_step * args.steps, clocks=clk, e2e=e2e,
+                    context=PAGES_CLAIM)
+        if not args.no_overlap:
+            line["prefill_overlap"] = bench.prefill_overlap()
         if world == 1 and not args.no_cpu_baseline:
             v, info = oracle_rate(bench.inp, w, budget_s=10.0)
             line["cpu_baseline"] = dict(value=v, unit="tokens/s", **info)

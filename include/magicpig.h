@@ -22,8 +22,11 @@
  *
  * Conventions for every call:
  *   - Tensors are caller-owned device buffers (bf16 is passed as raw 16-bit
- *     patterns).  The library allocates nothing and keeps no global state
- *     beyond a per-device cache of function attributes.
+ *     patterns).  The library allocates nothing.  Its global state is a
+ *     per-device cache of function attributes and, for
+ *     mp_decode_attend_noalloc only, one fixed 16 MiB scratch array in device
+ *     memory on every GPU that loads the library (with its address cached per
+ *     device).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) except mp_read_status, which synchronises.
  *   - Return value: MP_OK or a negative MP_ERR_* from host-side validation
@@ -187,10 +190,10 @@ int mp_decode_attend(const mp_shape *shape, const void *q, const void *W, const 
 /*
  * mp_decode_attend without a caller-provided workspace.  The method has no
  * counterpart of this call: it exists for callers that cannot allocate device
- * memory where they decode — code inside a CUDA-graph capture region, runtimes
- * whose memory pools are sealed after start-up, plugins that only receive
- * tensors from a host framework.  Same arguments, results and device checks as
- * mp_decode_attend, minus the workspace and the test hooks.
+ * memory where they decode — runtimes whose memory pools are sealed after
+ * start-up, plugins that only receive tensors from a host framework and may
+ * not call cudaMalloc themselves.  Same arguments, results and device checks
+ * as mp_decode_attend, minus the workspace and the test hooks.
  *   - Scratch is one fixed array of 16 MiB compiled into the library; every
  *     GPU that loads the library holds it until the process exits.
  *   - Problems whose workspace (mp_decode_workspace_bytes) exceeds 16 MiB are
@@ -198,7 +201,10 @@ int mp_decode_attend(const mp_shape *shape, const void *q, const void *W, const 
  *     128k-token sequence with 8 kv heads and K = 8 fits).
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it: make that first call before any
- *     stream capture begins.
+ *     stream capture begins.  The cached address belongs to the device's
+ *     current context: after a device reset (cudaDeviceReset) it is stale, and
+ *     the library must be unloaded and loaded again before this call is used
+ *     on that device.
  *   - Every call shares the array: calls whose executions overlap on the GPU
  *     (several streams or host threads on one device) race and must be
  *     serialised by the caller.  The array's contents carry over between calls;

@@ -1,18 +1,20 @@
 // Decode entry point that needs no caller-provided workspace.
 //
 // mp_decode_attend takes a device workspace that the caller allocates.  Some
-// callers cannot allocate device memory at the point where they decode: code
-// running inside a CUDA-graph capture region (allocation would break the
-// capture), runtimes whose memory pools are sealed after start-up, and
-// plugins that only ever receive tensors from a host framework and may not
-// call cudaMalloc themselves.  mp_decode_attend_noalloc serves them: its
-// scratch space is a fixed, file-scope device array compiled into the library.
+// callers cannot allocate device memory at the point where they decode:
+// runtimes whose memory pools are sealed after start-up, and plugins that only
+// ever receive tensors from a host framework and may not call cudaMalloc
+// themselves.  mp_decode_attend_noalloc serves them: its scratch space is a
+// fixed, file-scope device array compiled into the library.
 //
 // The array is kNoAllocScratchBytes (16 MiB) on every GPU that loads the
 // library, for the life of the process.  Host code cannot use the array's name
 // as a device address, so the first call on each device (with that device
 // current) looks the address up with cudaGetSymbolAddress and caches it; make
-// that first call before any stream capture begins.  All calls share the one
+// that first call before any stream capture begins.  The cached address is
+// that of the device's current context: after cudaDeviceReset it is stale and
+// the library has to be reloaded before this entry point is used again on
+// that device.  All calls share the one
 // array: calls whose executions overlap on the GPU (two streams, or two host
 // threads on the same device) race on it and must be serialised by the caller.
 // Nothing in the array has to start at zero: the first kernel of every call

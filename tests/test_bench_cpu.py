@@ -57,3 +57,43 @@ def test_packed_inputs_round_trip():
         np.testing.assert_array_equal(buf[off:off + a.nbytes].view(a.dtype), a)
         off += (a.nbytes + 255) // 256 * 256
     assert buf.nbytes == off
+
+
+def test_both_arms_report_the_same_config():
+    """The GPU arm and the reference arm print config_of(workload) unchanged:
+    it names the workload only (no launch mode or kernel path)."""
+    import workloads
+    w = workloads.get(bench.DEFAULT_WORKLOAD)
+    cfg = bench.config_of(w)
+    assert cfg["workload"] == "ragged16" and cfg["code_layout"] == "bytes"
+    assert not {"launch", "decode_path", "mode"} & set(cfg)
+    assert cfg == bench.config_of(workloads.get("ragged16"))
+
+
+def test_step_contents_per_workload():
+    """Only the 16k Llama-shaped layer hashes every cached key inside the
+    step; elsewhere the key-hash build is timed apart."""
+    import workloads
+    assert bench.hash_in_step(workloads.get("llama8b_16k"))
+    for name in ("ragged16", "batch8_64k", "batch4_128k", "ragged4", "tiny"):
+        assert not bench.hash_in_step(workloads.get(name))
+
+
+def test_decode_bytes_hand_count():
+    """Two sequences of 100 and 3 tokens, K=8, L=75, sink 4 + window 64,
+    2 kv heads, 10 union rows: codes 103 x 2 x 75 B; exact rows: 68 for the
+    long sequence (4 + 64) and all 3 of the short one, per kv head."""
+    import workloads
+    w = workloads.get("tiny").with_(n_kv_heads=2, n_q_heads=2)
+    total, codes, d_rows = bench.decode_bytes(w, np.array([100, 3]), 10)
+    assert codes == 103 * 2 * 75
+    assert d_rows == (68 + 3) * 2
+    assert total == codes + (10 + d_rows) * 512
+
+
+def test_oracle_sample_units_spread_over_the_batch():
+    import workloads
+    w = workloads.get("ragged16")
+    smp = bench.OracleSample(w)
+    assert smp.units == [(0, 0), (4, 1), (8, 2), (12, 3)]
+    assert "(N_b + 1) / 8" in smp.describe()

@@ -1,6 +1,6 @@
 """mp_decode_attend_noalloc: the decode entry point for callers that cannot
-allocate device memory where they decode (inside a CUDA-graph capture, with a
-sealed memory pool, or as a plugin that only receives tensors).  It must give
+allocate device memory where they decode (a runtime with a memory pool sealed
+after start-up, or a plugin that only receives tensors).  It must give
 the same results as mp_decode_attend, which uses a caller-allocated workspace,
 on consecutive calls that share the library's fixed scratch array.
 
