@@ -177,17 +177,7 @@ struct ScanOut {
     int32_t *cnt;        // [B*Hkv][nchunk][16]: [0] union count, [1+g] per-head count
     uint8_t *member_out; // nullable [B][Hq][Ncap]
     int32_t *status;
-    uint32_t one;        // 1, opaque to the compiler (see add_fma)
 };
-
-// a + c computed as a * one + c: an integer multiply-add runs on the FMA pipe,
-// leaving the ALU pipe to the logic operations of the byte scan.
-__device__ __forceinline__ uint32_t add_fma(uint32_t a, uint32_t one, uint32_t c)
-{
-    uint32_t r;
-    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(one), "r"(c));
-    return r;
-}
 
 // Bits [lo - base, hi - base) of a `width`-bit token word starting at token `base`.
 __device__ __forceinline__ uint32_t range_mask(int base, int lo, int hi, int width)
@@ -248,138 +238,143 @@ __device__ __forceinline__ void compact_warp(const Shape &s, int unit, int chunk
     }
 }
 
-// Table-split partial counters: thread (ts, tg) with ts > 0 leaves its two
-// bit-sliced counters (seen >= 1, seen >= 2) for its token group in shared
-// memory; the ts == 0 thread of the same group folds them in:
-//   s2 = s2 | s2' | (s1 & s1'),  s1 = s1 | s1'.
-template <int G, int NW, int TS>
-__device__ __forceinline__ void combine_splits(uint32_t (&s1)[G][NW], uint32_t (&s2)[G][NW], uint32_t *part, int ts,
-                                               int tg)
+// -------------------------------------------------- scan, byte codes (K = 8) ----
+// Byte codes [unit][L][Ncap].  A warp owns a 512-token chunk of one unit for
+// all L tables (lane = 16 consecutive tokens, one 16-byte streaming load per
+// table), so no partial counts ever cross warps; a block is 8 consecutive
+// chunks of one unit and shares only the query codes.
+//
+// Each 16-bit half of a register holds one token's code byte c as the bit
+// pattern 0x6000 | c, a normal fp16 number (512 + c/2), so two tokens are
+// compared with one packed half compare against the query's 0x6000 | q:
+// set.eq.f16x2 yields 1.0 per matching half, and add.f16x2 sums the matches
+// per (token, head) exactly (at most L <= 255 < 2048).  Compare and add both
+// run on the FMA pipe; the byte split (one lop3 for the even bytes, one prmt
+// for the odd bytes of a word) is shared by the G heads.  A token is in S_h
+// iff its count reaches 2.
+__device__ __forceinline__ uint32_t h2_even_bytes(uint32_t w)  // halves 0x6000 | byte 0, 0x6000 | byte 2
 {
-    constexpr int TG = kScanThreads / TS;
-    if (ts > 0) {
-#pragma unroll
-        for (int g = 0; g < G; g++)
-#pragma unroll
-            for (int j = 0; j < NW; j++) {
-                part[((g * NW + j) * 2 + 0) * kScanThreads + threadIdx.x] = s1[g][j];
-                part[((g * NW + j) * 2 + 1) * kScanThreads + threadIdx.x] = s2[g][j];
-            }
-    }
-    __syncthreads();
-    if (ts == 0) {
-#pragma unroll 1
-        for (int t = 1; t < TS; t++) {
-#pragma unroll
-            for (int g = 0; g < G; g++)
-#pragma unroll
-                for (int j = 0; j < NW; j++) {
-                    const uint32_t a1 = part[((g * NW + j) * 2 + 0) * kScanThreads + t * TG + tg];
-                    const uint32_t a2 = part[((g * NW + j) * 2 + 1) * kScanThreads + t * TG + tg];
-                    s2[g][j] |= a2 | (s1[g][j] & a1);
-                    s1[g][j] |= a1;
-                }
-        }
-    }
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(0x00FF00FFu), "r"(0x60006000u));  // (w & b) | c
+    return r;
+}
+__device__ __forceinline__ uint32_t h2_odd_bytes(uint32_t w)  // halves 0x6000 | byte 1, 0x6000 | byte 3
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, 0x4341;" : "=r"(r) : "r"(w), "r"(0x60606060u));
+    return r;
+}
+__device__ __forceinline__ void h2_count_eq(uint32_t &cnt, uint32_t x, uint32_t q)  // cnt += (x == q) per half
+{
+    uint32_t m;
+    asm("set.eq.f16x2.f16x2 %0, %1, %2;" : "=r"(m) : "r"(x), "r"(q));
+    asm("add.rn.f16x2 %0, %0, %1;" : "+r"(cnt) : "r"(m));
+}
+// Bits 0 and 1 of the result: halves of `cnt` at or above 2.0.
+__device__ __forceinline__ uint32_t h2_at_least_2(uint32_t cnt)
+{
+    uint32_t m;
+    asm("set.ge.u32.f16x2 %0, %1, %2;" : "=r"(m) : "r"(cnt), "r"(0x40004000u));  // 0xFFFF per true half (2.0)
+    return (m & 1u) | ((m >> 15) & 2u);
 }
 
-// -------------------------------------------------- scan, byte codes (K = 8) ----
-// Byte codes [unit][L][Ncap].  A 512-token chunk per block of 256 threads:
-// 32 token groups of 16 tokens (one 16-byte load per table) x 8 table splits
-// (tables ts, ts + 8, ...; up to 8 loads in flight per thread), merged in
-// shared memory.  Per 4-token word and
-// head: x = codes ^ (qcode * 0x01010101); a byte of x is zero iff that token
-// matches.  Zero bytes are found exactly with ((x & 0x7f..) + 0x7f..) | x,
-// whose byte top bit is 1 iff the byte is non-zero (the add runs on the FMA
-// pipe).  Two bit-sliced counters (seen >= 1, seen >= 2) live in the byte top
-// bits.  Warp 0 folds the other splits' counters and compacts the chunk's
-// candidates alone (warp-level scan, no block barrier); warps 1..7 exit.
+constexpr int kByteWarps = 8;   // chunks (warps) per block
+constexpr int kByteRing = 12;   // tables in each warp's shared-memory ring (11 copies in flight)
+
+// Each lane copies its own 16 code bytes of a table into its slot of the
+// warp's ring (cp.async, 16 bytes, bypassing L1) and reads back only that
+// slot, so the ring needs no barrier: cp.async.wait_group makes a lane's own
+// copies visible to it, and a slot is refilled (same lane, program order,
+// after __syncwarp) only once its bytes have been consumed.
 template <int G>
-__global__ void __launch_bounds__(kScanThreads, 3) scan_k8_kernel(
+__global__ void __launch_bounds__(32 * kByteWarps, G >= 8 ? 2 : 4) scan_bytes_kernel(
     Shape s, const uint8_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
     const int32_t *__restrict__ seq_lens, int max_len, int nchunk, ScanOut o)
 {
-    extern __shared__ uint32_t dyn[];  // rep [L][G] (query code in 4 bytes), then split partials
-    uint32_t *rep = dyn;
-    uint32_t *part = dyn + ((s.L * G + 3) & ~3);
-    constexpr int TS = kSplitsK8, TG = kScanThreads / TS, NB = 4;
-    static_assert(TG == 32, "split ts = warp ts, token group tg = lane");
-    const int ts = threadIdx.x / TG, tg = threadIdx.x % TG;
-    const int unit = blockIdx.y, chunk = blockIdx.x;
+    extern __shared__ __align__(16) uint32_t scan_smem[];  // ring [8 warps][kByteRing][512 B], then qpat [L][G]
+    constexpr int D = kByteRing;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t *ring = reinterpret_cast<uint8_t *>(scan_smem) + (size_t)warp * D * kChunkBytes + lane * 16;
+    uint32_t *qpat = scan_smem + kByteWarps * D * kChunkBytes / 4;  // (0x6000 | q) in both halves
+    const int unit = blockIdx.y, chunk = blockIdx.x * kByteWarps + warp;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
     grid_launch_dependents();
     // lengths and codes come from work before the query hash: read them first
     const int N = clamp_len(seq_lens, b, max_len, o.status, false);
-    const int c0 = chunk * kChunkBytes;
-    const bool reporter = chunk == 0 && kvh == 0 && threadIdx.x == 0;  // of a bad length of sequence b
-    if (c0 >= N) {
+    const bool reporter = blockIdx.x == 0 && kvh == 0 && threadIdx.x == 0;  // of a bad length of sequence b
+    if (blockIdx.x * kByteWarps * kChunkBytes >= N) {  // the whole block is past the sequence
         if (reporter) {
             grid_wait();  // the status word is cleared by the query hash
             clamp_len(seq_lens, b, max_len, o.status, true);
         }
         return;
     }
-    const int t0 = c0 + tg * 16;
-    const uint8_t *base = codes + (size_t)unit * s.L * s.Ncap + t0;
-    uint4 wv[NB];
-    auto load_batch = [&](int lb) {
-#pragma unroll
-        for (int i = 0; i < NB; i++) {
-            const int l = lb + i * TS;
-            wv[i] = t0 < N && l < s.L ? ld_stream_16(base + (size_t)l * s.Ncap) : make_uint4(0, 0, 0, 0);
-        }
+    const int c0 = chunk * kChunkBytes;
+    const int t0 = c0 + lane * 16;
+    const bool live = c0 < N;  // warp-uniform
+    const bool mine = t0 < N;  // lanes past the sequence copy nothing (their counts are masked)
+    const uint8_t *src = codes + (size_t)unit * s.L * s.Ncap + t0;
+    auto copy = [&](int l) {
+        if (mine && l < s.L) cp_async_16(ring + (l % D) * kChunkBytes, src + (size_t)l * s.Ncap, 16);
+        cp_async_commit();  // one group per table, empty past L, so the group count stays uniform
     };
-    load_batch(ts);
+    if (live)
+        for (int l = 0; l < D - 1; l++) copy(l);
     grid_wait();  // the query codes are the query hash's output
     if (reporter) clamp_len(seq_lens, b, max_len, o.status, true);
     for (int i = threadIdx.x; i < s.L * G; i += blockDim.x) {
         const int l = i / G, g = i % G;
-        rep[i] = (qcodes[((size_t)b * s.Hq + kvh * G + g) * s.L + l] & 0xFFu) * 0x01010101u;
+        qpat[i] = ((qcodes[((size_t)b * s.Hq + kvh * G + g) * s.L + l] & 0xFFu) | 0x6000u) * 0x00010001u;
     }
     __syncthreads();
+    if (!live) return;
 
-    uint32_t s1[G][4], s2[G][4];
+    // cnt[g][j][0]: tokens 4j and 4j + 2 (even bytes of word j), [1]: 4j + 1, 4j + 3
+    uint32_t cnt[G][4][2];
 #pragma unroll
     for (int g = 0; g < G; g++)
 #pragma unroll
-        for (int j = 0; j < 4; j++) s1[g][j] = s2[g][j] = 0u;
+        for (int j = 0; j < 4; j++) cnt[g][j][0] = cnt[g][j][1] = 0u;
 
-    if (t0 < N) {
-        for (int lb = ts; lb < s.L; lb += NB * TS) {
-            if (lb != ts) load_batch(lb);
+#pragma unroll 2
+    for (int l = 0; l < s.L; l++) {
+        cp_async_wait<D - 2>();  // table l has landed (groups 0 .. l complete)
+        const uint4 v = *reinterpret_cast<const uint4 *>(ring + (l % D) * kChunkBytes);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t ev[4], od[4];
 #pragma unroll
-            for (int i = 0; i < NB; i++) {
-                const int l = lb + i * TS;
-                if (l >= s.L) break;
-                const uint32_t w[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+        for (int j = 0; j < 4; j++) {
+            ev[j] = h2_even_bytes(w[j]);
+            od[j] = h2_odd_bytes(w[j]);
+        }
+        __syncwarp();
+        copy(l + D - 1);  // into the slot of table l - 1, consumed in the previous iteration
 #pragma unroll
-                for (int g = 0; g < G; g++) {
-                    const uint32_t r = rep[l * G + g];
+        for (int g = 0; g < G; g++) {
+            const uint32_t q = qpat[l * G + g];
 #pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        const uint32_t x = w[j] ^ r;
-                        const uint32_t nz = add_fma(x & 0x7F7F7F7Fu, o.one, 0x7F7F7F7Fu) | x;
-                        s2[g][j] |= s1[g][j] & ~nz;
-                        s1[g][j] |= ~nz;
-                    }
-                }
+            for (int j = 0; j < 4; j++) {
+                h2_count_eq(cnt[g][j][0], ev[j], q);
+                h2_count_eq(cnt[g][j][1], od[j], q);
             }
         }
     }
-    combine_splits<G, 4, TS>(s1, s2, part, ts, tg);
-    if (ts != 0) return;  // warp 0 (ts == 0, lane = tg) now holds the chunk's counters
-    // Per-head 16-bit token masks from the byte top bits of the >= 2 counter:
-    // the four top bits of a word, moved to bits 24..27 by one multiply.
+    cp_async_wait<0>();
+    // Per-head 16-bit token masks: bit 4j + {0, 1, 2, 3} = tokens of word j.
     uint32_t hm[G];
 #pragma unroll
     for (int g = 0; g < G; g++) {
         uint32_t m = 0u;
 #pragma unroll
-        for (int j = 0; j < 4; j++) m |= ((((s2[g][j] >> 7) & 0x01010101u) * 0x01020408u) >> 24) << (4 * j);
+        for (int j = 0; j < 4; j++) {
+            const uint32_t e = h2_at_least_2(cnt[g][j][0]), od = h2_at_least_2(cnt[g][j][1]);
+            // e: bit 0 = token 4j, bit 1 = token 4j + 2; od: the same for 4j + 1, 4j + 3
+            m |= ((e & 1u) | ((od & 1u) << 1) | ((e & 2u) << 1) | ((od & 2u) << 2)) << (4 * j);
+        }
         hm[g] = m;
     }
     // Tokens eligible for S: [sink, N - window) and below N.
-    compact_warp<G, 16, kChunkBytes>(s, unit, chunk, nchunk, t0, N, s.sink, min(N - s.window, N), hm, o, tg);
+    compact_warp<G, 16, kChunkBytes>(s, unit, chunk, nchunk, t0, N, s.sink, min(N - s.window, N), hm, o, lane);
 }
 
 // ------------------------------------------------------ scan, bit planes ----
@@ -1900,7 +1895,7 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
                        (const uint16_t *)(dbg ? dbg->qcodes_in : nullptr), ws.qcodes, ws.status, ug);
         if (e != cudaSuccess) return e;
     }
-    ScanOut so{ws.cand, ws.cnt, dbg ? dbg->member_out : nullptr, ws.status, 1u};
+    ScanOut so{ws.cand, ws.cnt, dbg ? dbg->member_out : nullptr, ws.status};
     const LogU lu = make_logu(s);
     const float scale = 1.0f / sqrtf((float)s.d);
     const int path = dbg ? dbg->path : MP_PATH_AUTO;
@@ -1932,12 +1927,12 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
         if (!fused && path == MP_PATH_FUSED) return cudaErrorNotSupported;
     }
     if (nchunk > 0 && !fused) {
-        dim3 grid(nchunk, units);
-        const size_t part = (size_t)2 * G * 4 * kScanThreads * sizeof(uint32_t);       // byte scan: 4 words
         if (!s.planes) {
-            const size_t sm = (size_t)((s.L * G + 3) & ~3) * sizeof(uint32_t) + part;
-            if ((e = ensure_smem(reinterpret_cast<const void *>(scan_k8_kernel<G>), (int)sm)) != cudaSuccess) return e;
-            e = launch_pdl(scan_k8_kernel<G>, grid, dim3(kScanThreads), sm, st, s,
+            const size_t sm = (size_t)kByteWarps * kByteRing * kChunkBytes + (size_t)s.L * G * sizeof(uint32_t);
+            if ((e = ensure_smem(reinterpret_cast<const void *>(scan_bytes_kernel<G>), (int)sm)) != cudaSuccess)
+                return e;
+            dim3 grid((nchunk + kByteWarps - 1) / kByteWarps, units);
+            e = launch_pdl(scan_bytes_kernel<G>, grid, dim3(32 * kByteWarps), sm, st, s,
                            static_cast<const uint8_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
                            nchunk, so);
         } else if (s.K == 8) {
