@@ -154,6 +154,8 @@ int mp_append_token(const mp_shape *shape, const void *k_new, const void *v_new,
 #define MP_PATH_SPLIT 1    /* collision scan, then sampled attention (two kernels) */
 #define MP_PATH_FUSED 2    /* one kernel scans and attends (bit-plane codes, G <= 4);
                               MP_ERR_SHAPE where it does not apply */
+#define MP_PATH_TC 3       /* collision scan, then sampled attention on the tcgen05 tensor cores
+                              (scores, key norms and P.V in TMEM; persistent, one CTA per SM) */
 
 /* Test hooks of mp_decode_attend (all nullable / zero). */
 typedef struct mp_decode_debug {

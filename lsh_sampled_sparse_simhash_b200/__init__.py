@@ -36,6 +36,7 @@ from ._binding import (  # noqa: F401
     MP_PATH_AUTO,
     MP_PATH_SPLIT,
     MP_PATH_FUSED,
+    MP_PATH_TC,
 )
 
 __all__ = [

@@ -23,6 +23,7 @@ MP_CODES_PLANES = 2
 MP_PATH_AUTO = 0
 MP_PATH_SPLIT = 1
 MP_PATH_FUSED = 2
+MP_PATH_TC = 3
 
 
 class MagicPIGError(RuntimeError):

@@ -175,7 +175,7 @@ int mp_decode_attend(const mp_shape *shape, const void *q, const void *W, const 
     if (debug) {
         if ((debug->qcodes_in && !aligned16(debug->qcodes_in)) || (debug->qcodes_out && !aligned16(debug->qcodes_out)))
             return MP_ERR_ALIGN;
-        if (debug->path < MP_PATH_AUTO || debug->path > MP_PATH_FUSED) return MP_ERR_ARG;
+        if (debug->path < MP_PATH_AUTO || debug->path > MP_PATH_TC) return MP_ERR_ARG;
         if (debug->path == MP_PATH_FUSED && (!s.planes || s.G > 4)) return MP_ERR_SHAPE;
     }
     return cuda_status(launch_decode(s, static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(W), codes,

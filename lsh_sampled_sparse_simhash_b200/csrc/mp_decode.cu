@@ -25,6 +25,7 @@
 
 #include "mp_common.cuh"
 #include "mp_kernels.cuh"
+#include "mp_logu.cuh"
 
 namespace mp {
 
@@ -55,7 +56,10 @@ __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__r
     const size_t vec0 = (size_t)u0 * G;  // query vectors of a unit are consecutive: (b Hkv + kvh) G + g
 
     grid_dependency_wait();
-    if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *status = 0;
+    if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) {
+        status[0] = 0;  // the call's status word
+        status[1] = 0;  // the attention kernel's work counter
+    }
 
     if (qcodes_in) {
         for (int i = tid; i < nu * G * TB; i += blockDim.x) {
@@ -284,17 +288,24 @@ constexpr int kByteRing = 12;   // tables in each warp's shared-memory ring (11 
 // Each lane copies its own 16 code bytes of a table into its slot of the
 // warp's ring (cp.async, 16 bytes, bypassing L1) and reads back only that
 // slot, so the ring needs no barrier: cp.async.wait_group makes a lane's own
-// copies visible to it, and a slot is refilled (same lane, program order,
-// after __syncwarp) only once its bytes have been consumed.
+// copies visible to it, and a slot is refilled by the same lane only after
+// the words read from it have been used (the refill is issued after the
+// instructions that consume them).  The query patterns of a table are one
+// 16-byte shared load for up to four heads.
 template <int G>
-__global__ void __launch_bounds__(32 * kByteWarps, G >= 8 ? 2 : 4) scan_bytes_kernel(
+#ifndef MP_SCAN_BLOCKS_PER_SM
+#define MP_SCAN_BLOCKS_PER_SM 4
+#endif
+__global__ void __launch_bounds__(32 * kByteWarps, G >= 8 ? 2 : MP_SCAN_BLOCKS_PER_SM) scan_bytes_kernel(
     Shape s, const uint8_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
     const int32_t *__restrict__ seq_lens, int max_len, int nchunk, ScanOut o)
 {
-    extern __shared__ __align__(16) uint32_t scan_smem[];  // ring [8 warps][kByteRing][512 B], then qpat [L][G]
+    extern __shared__ __align__(16) uint32_t scan_smem[];  // ring [8 warps][kByteRing][512 B], then qpat [L][GP]
     constexpr int D = kByteRing;
+    constexpr int GP = G < 4 ? 4 : G;  // query patterns per table, padded to whole 16-byte loads
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint8_t *ring = reinterpret_cast<uint8_t *>(scan_smem) + (size_t)warp * D * kChunkBytes + lane * 16;
+    const uint32_t ring0 = smem_u32(scan_smem) + (uint32_t)(warp * D * kChunkBytes + lane * 16);
+    const uint32_t ring_end = ring0 + D * kChunkBytes;
     uint32_t *qpat = scan_smem + kByteWarps * D * kChunkBytes / 4;  // (0x6000 | q) in both halves
     const int unit = blockIdx.y, chunk = blockIdx.x * kByteWarps + warp;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
@@ -314,17 +325,21 @@ __global__ void __launch_bounds__(32 * kByteWarps, G >= 8 ? 2 : 4) scan_bytes_ke
     const bool live = c0 < N;  // warp-uniform
     const bool mine = t0 < N;  // lanes past the sequence copy nothing (their counts are masked)
     const uint8_t *src = codes + (size_t)unit * s.L * s.Ncap + t0;
-    auto copy = [&](int l) {
-        if (mine && l < s.L) cp_async_16(ring + (l % D) * kChunkBytes, src + (size_t)l * s.Ncap, 16);
-        cp_async_commit();  // one group per table, empty past L, so the group count stays uniform
-    };
-    if (live)
-        for (int l = 0; l < D - 1; l++) copy(l);
+    uint32_t wr = ring0;  // slot of the next copy
+    if (live) {
+        for (int l = 0; l < D - 1; l++) {
+            if (mine && l < s.L) cp_async_16_s(wr, src, 16);
+            cp_async_commit();  // one group per table, empty past L, so the group count stays uniform
+            src += s.Ncap;
+            wr += kChunkBytes;
+        }
+    }
     grid_wait();  // the query codes are the query hash's output
     if (reporter) clamp_len(seq_lens, b, max_len, o.status, true);
-    for (int i = threadIdx.x; i < s.L * G; i += blockDim.x) {
-        const int l = i / G, g = i % G;
-        qpat[i] = ((qcodes[((size_t)b * s.Hq + kvh * G + g) * s.L + l] & 0xFFu) | 0x6000u) * 0x00010001u;
+    for (int i = threadIdx.x; i < s.L * GP; i += blockDim.x) {
+        const int l = i / GP, g = i % GP;
+        qpat[i] = g < G ? ((qcodes[((size_t)b * s.Hq + kvh * G + g) * s.L + l] & 0xFFu) | 0x6000u) * 0x00010001u
+                        : 0u;
     }
     __syncthreads();
     if (!live) return;
@@ -336,10 +351,14 @@ __global__ void __launch_bounds__(32 * kByteWarps, G >= 8 ? 2 : 4) scan_bytes_ke
 #pragma unroll
         for (int j = 0; j < 4; j++) cnt[g][j][0] = cnt[g][j][1] = 0u;
 
-#pragma unroll 2
+    uint32_t rd = ring0;  // slot of table l
+    const uint4 *qp = reinterpret_cast<const uint4 *>(qpat);
     for (int l = 0; l < s.L; l++) {
         cp_async_wait<D - 2>();  // table l has landed (groups 0 .. l complete)
-        const uint4 v = *reinterpret_cast<const uint4 *>(ring + (l % D) * kChunkBytes);
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(rd)
+                     : "memory");
+        rd = rd + kChunkBytes == ring_end ? ring0 : rd + kChunkBytes;
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t ev[4], od[4];
 #pragma unroll
@@ -347,17 +366,27 @@ __global__ void __launch_bounds__(32 * kByteWarps, G >= 8 ? 2 : 4) scan_bytes_ke
             ev[j] = h2_even_bytes(w[j]);
             od[j] = h2_odd_bytes(w[j]);
         }
-        __syncwarp();
-        copy(l + D - 1);  // into the slot of table l - 1, consumed in the previous iteration
+        // the refill of the slot of table l - 1, whose words were used last iteration
+        if (mine && l + D - 1 < s.L) cp_async_16_s(wr, src, 16);
+        cp_async_commit();
+        src += s.Ncap;
+        wr = wr + kChunkBytes == ring_end ? ring0 : wr + kChunkBytes;
+        uint32_t q[GP];
 #pragma unroll
-        for (int g = 0; g < G; g++) {
-            const uint32_t q = qpat[l * G + g];
+        for (int k = 0; k < GP / 4; k++) {
+            const uint4 t = qp[l * (GP / 4) + k];
+            q[4 * k] = t.x;
+            q[4 * k + 1] = t.y;
+            q[4 * k + 2] = t.z;
+            q[4 * k + 3] = t.w;
+        }
+#pragma unroll
+        for (int g = 0; g < G; g++)
 #pragma unroll
             for (int j = 0; j < 4; j++) {
-                h2_count_eq(cnt[g][j][0], ev[j], q);
-                h2_count_eq(cnt[g][j][1], od[j], q);
+                h2_count_eq(cnt[g][j][0], ev[j], q[g]);
+                h2_count_eq(cnt[g][j][1], od[j], q[g]);
             }
-        }
     }
     cp_async_wait<0>();
     // Per-head 16-bit token masks: bit 4j + {0, 1, 2, 3} = tokens of word j.
@@ -679,38 +708,6 @@ __global__ void __launch_bounds__(kScanThreads + 32) scan_planes_kernel(
 }
 
 // ---------------------------------------------------------------- attend ----
-// log u for the at-least-2-of-L rule, u = P[Binomial(L, x) >= 2], x = p^K,
-// p = 1 - arccos(c)/pi.  Small x: u = C(L,2) x^2 (1-x)^(L-2) * (1 + a3 r (1 +
-// a4 r (1 + a5 r))) with r = x / (1-x), a_j = (L-j+1)/j (binomial ratios),
-// truncated after j = 5 (relative error < 2e-6 for x < 1e-3, L <= 255).
-// Otherwise u = 1 - exp(y), y = (L-1) log1p(-x) + log1p((L-1) x) (the closed
-// form 1 - (1-x)^L - L x (1-x)^(L-1) rearranged so that expm1 keeps u's
-// relative precision).
-struct LogU {
-    float K, L, lnC2, a3, a4, a5;
-};
-
-// log u for a pair of cosine c.  The plain log and exp are the hardware
-// approximations (__logf, __expf: a few ulp, a few 1e-6 relative at these
-// arguments), which moves log u by ~1e-5 at most, far inside the output
-// tolerance; acos and the log1p / expm1 terms, where cancellation matters,
-// keep the accurate library functions.
-__device__ __forceinline__ float log_sampling_prob(float c, const LogU &u)
-{
-    c = fminf(1.f, fmaxf(-1.f, c));
-    float p = 1.f - acosf(c) * 0.318309886183790671538f;
-    p = fmaxf(p, 1e-30f);
-    const float lx = u.K * __logf(p);
-    const float x = __expf(lx);
-    if (x < 1e-3f) {
-        const float r = x / (1.f - x);
-        const float tail = u.a3 * r * (1.f + u.a4 * r * (1.f + u.a5 * r));
-        return u.lnC2 + 2.f * lx + (u.L - 2.f) * log1pf(-x) + log1pf(tail);
-    }
-    const float y = (u.L - 1.f) * log1pf(-x) + log1pf((u.L - 1.f) * x);
-    return __logf(-expm1f(y));
-}
-
 constexpr int kAttThreads = 128;
 constexpr int kMaxSpan = 64;                // scan chunks per attention block, at most
 constexpr int kAttRows = 64;                // rows per tile (4 warps x 16)
@@ -1804,6 +1801,7 @@ static LogU make_logu(const Shape &s)
     u.a3 = (float)((L - 2.0) / 3.0);
     u.a4 = (float)((L - 3.0) / 4.0);
     u.a5 = (float)((L - 4.0) / 5.0);
+    u.a6 = (float)((L - 5.0) / 6.0);
     return u;
 }
 
@@ -1928,7 +1926,7 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     }
     if (nchunk > 0 && !fused) {
         if (!s.planes) {
-            const size_t sm = (size_t)kByteWarps * kByteRing * kChunkBytes + (size_t)s.L * G * sizeof(uint32_t);
+            const size_t sm = (size_t)kByteWarps * kByteRing * kChunkBytes + (size_t)s.L * std::max(G, 4) * sizeof(uint32_t);
             if ((e = ensure_smem(reinterpret_cast<const void *>(scan_bytes_kernel<G>), (int)sm)) != cudaSuccess)
                 return e;
             dim3 grid((nchunk + kByteWarps - 1) / kByteWarps, units);
@@ -1964,11 +1962,34 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
 
     aa.lu = lu;
     aa.scale = scale;
-    if (!fused) {
+    if (!fused && path != MP_PATH_TC) {
         const int sm = kAttStages * kStageBytes;
         if ((e = ensure_smem(reinterpret_cast<const void *>(attend_kernel<G>), sm)) != cudaSuccess) return e;
         dim3 grid(sp.nsplit, units);
         if ((e = launch_pdl(attend_kernel<G>, grid, dim3(kAttThreads), sm, st, aa)) != cudaSuccess) return e;
+    } else if (!fused) {
+        AttendTcArgs ta;
+        ta.s = s;
+        ta.q = q;
+        ta.kc = kc;
+        ta.vc = vc;
+        ta.seq_lens = seq_lens;
+        ta.max_len = max_len;
+        ta.nchunk = nchunk;
+        ta.span = sp.span;
+        ta.subs = sp.subs;
+        ta.nsplit = sp.nsplit;
+        ta.chunk_tokens = C;
+        ta.cand = ws.cand;
+        ta.cnt = ws.cnt;
+        ta.work_counter = ws.status + 1;
+        ta.status = ws.status;
+        ta.pm = ws.pm;
+        ta.pl = ws.pl;
+        ta.pacc = ws.pacc;
+        ta.lu = lu;
+        ta.scale = scale;
+        if ((e = launch_attend_tc(ta, st)) != cudaSuccess) return e;
     }
     // partials: per chunk (fused) or per split of the plan, then the exact set
     const int m_span = fused ? 1 : sp.span, m_subs = fused ? 1 : sp.subs, m_groups = fused ? nchunk : sp.ngroups;

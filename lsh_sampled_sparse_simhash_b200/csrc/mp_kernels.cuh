@@ -7,6 +7,7 @@
 #include <initializer_list>
 
 #include "mp_common.cuh"
+#include "mp_logu.cuh"
 
 namespace mp {
 
@@ -30,6 +31,27 @@ cudaError_t launch_decode(const Shape &s, const uint16_t *q, const uint16_t *W, 
                           float *out, float *lse, int32_t *n_sampled, void *workspace,
                           const mp_decode_debug *dbg, cudaStream_t st);
 size_t decode_workspace_bytes(const Shape &s, int max_len);
+
+// Sampled attention on the tensor cores (mp_attend_tc.cu): every work item of
+// the split plan (units x nsplit; split nsplit - 1 of a unit is its exact set
+// D) leaves one (m, l, acc) partial per query head in pm / pl / pacc
+// [B*Hq][nsplit] (acc: [..][128]); m and l are in log2 units.  work_counter
+// must be 0 when the kernel starts (the query hash clears it).
+struct AttendTcArgs {
+    Shape s;
+    const uint16_t *q, *kc, *vc;
+    const int32_t *seq_lens;
+    int max_len, nchunk, span, subs, nsplit, chunk_tokens;
+    const uint32_t *cand;  // [B*Hkv][nchunk][chunk_tokens] token | headmask << 24
+    const int32_t *cnt;    // [B*Hkv][nchunk][16], [0] = candidates of the chunk
+    int32_t *work_counter;
+    int32_t *status;
+    float *pm, *pl, *pacc;
+    LogU lu;
+    float scale;  // 1 / sqrt(d)
+};
+cudaError_t launch_attend_tc(const AttendTcArgs &a, cudaStream_t st);
+size_t attend_tc_smem_bytes();
 
 // A tiled TMA descriptor for a rank-`rank` tensor (dims and box innermost
 // first, byte strides of dims 1..rank-1), no interleave, zero fill out of

@@ -114,7 +114,7 @@ def test_decode_path_selector_checked(lib):
     Rejected on the host, so nothing launches."""
     A = 1 << 12  # aligned fake device pointers (never dereferenced)
     for lay, G, path, want in [(1, 4, 2, mp.MP_ERR_SHAPE), (2, 8, 2, mp.MP_ERR_SHAPE), (2, 4, 7, mp.MP_ERR_ARG),
-                               (2, 4, -1, mp.MP_ERR_ARG)]:
+                               (2, 4, 4, mp.MP_ERR_ARG), (2, 4, -1, mp.MP_ERR_ARG)]:
         s = good_shape(code_layout=lay, n_q_heads=2 * G)
         need = ctypes.c_size_t()
         assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 1024, ctypes.byref(need)) == 0

@@ -11,8 +11,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from gpu_harness import (Run, check_outputs, code_mismatch, dev, host, oracle_decode_units,
                          oracle_query_codes, oracle_unit_codes)
+from layout import unpack_codes
 from workloads import WORKLOADS, f32_to_bf16_bits, make_inputs
 
 import lsh_sampled_sparse_simhash_b200 as mp
@@ -92,6 +94,44 @@ def test_decode_same_codes_matches_oracle(case):
     worst = check_outputs(gpu, ref, w)
     print(f"{case}: worst rel-L2 {worst:.2e}, sampled per head {gpu['ns'].mean():.1f}")
     assert gpu["ns"].sum() > 0 or w.context <= w.sink + w.window
+
+
+@pytest.mark.parametrize("case", list(SMALL_CASES))
+def test_tc_attention_path_matches_oracle(case):
+    """The tcgen05 sampled-attention kernel (MP_PATH_TC: scores, key norms and
+    P.V on the tensor cores, accumulators in TMEM) on the oracle's codes: same
+    S_h and n_sampled, outputs within tolerance."""
+    w = SMALL_CASES[case]
+    run = Run(w)
+    units, codes, _ = oracle_codes_all(run)
+    run.set_codes(codes, units)
+    qref, _ = oracle_query_codes(run.inp, w)
+    gpu = run.decode(qcodes_in=qref, path=mp.MP_PATH_TC)
+    assert gpu["status"] == 0
+    ref = oracle_decode_units(run.inp, w, units, codes, qref)
+    check_outputs(gpu, ref, w)
+
+
+def test_tc_attention_ragged_lengths_and_boundaries():
+    """MP_PATH_TC over lengths that hit its tile and item boundaries: empty,
+    all-exact (N <= sink + window), one past a 128-row tile of candidates, and
+    long sequences whose candidate lists span several tiles."""
+    w = SMALL_CASES["g4_k8_ragged_tail"].with_(name="tcb", batch=6, context=9000, seed=2014)
+    inp = make_inputs(w)
+    inp["seq_lens"] = np.array([0, 50, 129, 2049, 9000, 4500], np.int32)
+    for b, n in enumerate(inp["seq_lens"]):
+        inp["K"][b, :, n:] = 0
+        inp["V"][b, :, n:] = 0
+    run = Run(w, inp)
+    units = all_units(w)
+    codes = [oracle_unit_codes(inp, w, b, kh, int(inp["seq_lens"][b]))[0] for b, kh in units]
+    run.set_codes(codes, units)
+    qref, _ = oracle_query_codes(inp, w)
+    gpu = run.decode(qcodes_in=qref, path=mp.MP_PATH_TC)
+    assert gpu["status"] == 0
+    ref = oracle_decode_units(inp, w, units, codes, qref)
+    check_outputs(gpu, ref, w)
+    assert np.isneginf(gpu["lse"][0]).all() and not gpu["out"][0].any()
 
 
 PLANE_CASES = ["g4_k10", "g2_k10_short", "g4_k8_planes", "g1_k8_planes_short"]
@@ -325,8 +365,7 @@ FULL = ["llama8b_16k", "batch8_64k", "batch4_128k", "ragged16", "ragged16_planes
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_sampled_units(name):
     """The full workload in the benchmark's launch configuration (hash every
-    key, append one token per sequence, decode); two (b, kv head) units are
-    checked against the oracle on the oracle's own codes."""
+    key, append one token per sequence, decode)."""
     _full_size(name, mp.MP_PATH_AUTO)
 
 
@@ -336,7 +375,28 @@ def test_full_size_fused_path(name):
     _full_size(name, mp.MP_PATH_FUSED)
 
 
+def test_full_size_tc_attention_path():
+    """The same at full size (ragged16, byte codes) through the tcgen05
+    sampled-attention kernel."""
+    _full_size("ragged16", mp.MP_PATH_TC)
+
+
+def _spread(units, lens, n):
+    """n units spread over the length range, the shortest and longest included."""
+    order = sorted(units, key=lambda u: (int(lens[u[0]]), u))
+    idx = sorted({int(round(i * (len(order) - 1) / max(n - 1, 1))) for i in range(n)})
+    return [order[i] for i in idx]
+
+
 def _full_size(name, path):
+    """Checks at full size, on every (sequence, kv head) unit:
+      - key codes: 1024 sampled tokens and the appended token of every unit
+        against the oracle's SimHash (bit-exact except near-zero bits);
+      - candidate sets and n_sampled of every unit against the oracle's
+        collision rule on the same codes (the GPU's key codes, the oracle's
+        query codes), bit-exact;
+      - out / lse of 8 units spread over the length range (shortest and
+        longest included) against the fp64 estimator on the same codes."""
     w = WORKLOADS[name] if name in WORKLOADS else WORKLOADS[name.rsplit("_", 1)[0]].with_(code_layout="planes")
     inp = make_inputs(w)
     run = Run(w, inp)
@@ -346,30 +406,41 @@ def _full_size(name, path):
     torch.cuda.synchronize()
     new_lens = host(run.lens)
     assert (new_lens == inp["seq_lens"] + 1).all()
-    # host copy of the post-append cache for the sampled units
-    units = [(0, 0), (w.batch - 1, w.n_kv_heads - 1)]
-    inp2 = dict(inp)
-    inp2["seq_lens"] = new_lens
-    K2 = inp["K"].copy()
-    V2 = inp["V"].copy()
+    # the post-append cache on the host (rows past each length are zero, so
+    # writing the appended row in place gives exactly that state)
     for b in range(w.batch):
-        K2[b, :, inp["seq_lens"][b]] = inp["k_new"][b]
-        V2[b, :, inp["seq_lens"][b]] = inp["v_new"][b]
-    inp2["K"], inp2["V"] = K2, V2
-    codes, bad = [], 0
-    rng = np.random.default_rng(0)
-    for b, kh in units:
-        n = int(new_lens[b])
-        c, m = oracle_unit_codes(inp2, w, b, kh, n)
-        codes.append(c)
-        pick = rng.choice(n, size=min(n, 4096), replace=False)
-        x, _ = code_mismatch(run.codes_logical(b, kh, n)[pick], c[pick], m[pick], w.k_bits)
-        bad += x
-    assert bad == 0
-    run.set_codes(codes, units)
+        inp["K"][b, :, inp["seq_lens"][b]] = inp["k_new"][b]
+        inp["V"][b, :, inp["seq_lens"][b]] = inp["v_new"][b]
+    inp["seq_lens"] = new_lens
     qref, _ = oracle_query_codes(inp, w)
     gpu = run.decode(qcodes_in=qref, path=path)
     assert gpu["status"] == 0
-    ref = oracle_decode_units(inp2, w, units, codes, qref)
+    codes_h = host(run.codes)
+    if run.shape.planes:
+        codes_h = codes_h.view(np.uint32)
+    units = all_units(w)
+    keep = set(_spread(units, new_lens, 8))
+    kept = {}
+    rng = np.random.default_rng(0)
+    bad = exempt = 0
+    G = w.group
+    for b, kh in units:
+        n = int(new_lens[b])
+        g = unpack_codes(codes_h[b, kh], w.k_bits, w.n_tables, n, run.shape.planes)
+        pick = np.unique(np.concatenate([rng.choice(n - 1, size=min(n - 1, 1024), replace=False), [n - 1]]))
+        ref, margin = oracle.simhash(inp["K"][b, kh, pick], inp["W"], w.k_bits, w.n_tables, margin=True)
+        x, e = code_mismatch(g[pick], ref, margin, w.k_bits)
+        bad += x
+        exempt += e
+        hs = slice(kh * G, (kh + 1) * G)
+        mem, ns = oracle.collide(g, qref[b, hs], w.sink, w.window)
+        np.testing.assert_array_equal(gpu["member"][b, hs, :n], mem, err_msg=f"member b={b} kh={kh}")
+        np.testing.assert_array_equal(gpu["ns"][b, hs], ns, err_msg=f"n_sampled b={b} kh={kh}")
+        if (b, kh) in keep:
+            kept[(b, kh)] = g
+    assert bad == 0, f"{bad} key-code bits differ beyond the near-zero tolerance ({exempt} exempt)"
+    picked = sorted(kept)
+    ref = oracle_decode_units(inp, w, picked, [kept[u] for u in picked], qref)
     worst = check_outputs(gpu, ref, w)
-    print(f"{name} (path {path}): worst rel-L2 {worst:.2e}; mean |S_h| {gpu['ns'].mean():.0f}")
+    print(f"{name} (path {path}): {len(units)} units' candidate sets exact; worst rel-L2 {worst:.2e} over "
+          f"{len(picked)} units; mean |S_h| {gpu['ns'].mean():.0f}; {exempt} near-zero code bits exempt")
