@@ -68,8 +68,9 @@ def parse(argv=None):
                    help="key-code layout (default: the workload's, i.e. bytes for K=8, planes for K=10)")
     p.add_argument("--no-graph", action="store_true",
                    help="launch every timed step eagerly instead of replaying a captured CUDA graph")
-    p.add_argument("--decode-path", default="auto", choices=["auto", "split", "fused"],
-                   help="decode kernels: auto, split (scan then attention) or fused (one kernel; bit planes)")
+    p.add_argument("--decode-path", default="auto", choices=["auto", "split", "fused", "tc"],
+                   help="decode kernels: auto, split (scan then attention), fused (one kernel; bit planes) or tc "
+                        "(scan then the tcgen05 attention kernel)")
     return p.parse_args(argv)
 
 
@@ -224,7 +225,8 @@ class Bench:
         self.out, self.lse, self.ns = _views(self.out_dev, step_out)
         self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
         self.tokens = step_tokens(inp["seq_lens"] + 1)
-        self.path = {"auto": mp.MP_PATH_AUTO, "split": mp.MP_PATH_SPLIT, "fused": mp.MP_PATH_FUSED}[path]
+        self.path = {"auto": mp.MP_PATH_AUTO, "split": mp.MP_PATH_SPLIT, "fused": mp.MP_PATH_FUSED,
+                     "tc": mp.MP_PATH_TC}[path]
         self.graph_error = None
         self.with_hash = hash_in_step(w)
         fused = self.path == mp.MP_PATH_FUSED

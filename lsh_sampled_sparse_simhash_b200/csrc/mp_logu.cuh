@@ -24,7 +24,9 @@ struct LogU {
 // approximations (__logf, __expf: a few ulp, a few 1e-6 relative at these
 // arguments), which moves log u by ~1e-5 at most, far inside the output
 // tolerance; acos and the log1p / expm1 terms, where cancellation matters,
-// keep the accurate library functions.
+// keep the accurate library functions.  Both forms share one log1p of (-x) and one
+// log1p of a form-dependent argument, so a warp whose lanes take different
+// forms evaluates log1p twice, not three times.
 __device__ __forceinline__ float log_sampling_prob(float c, const LogU &u)
 {
     c = fminf(1.f, fmaxf(-1.f, c));
@@ -32,13 +34,13 @@ __device__ __forceinline__ float log_sampling_prob(float c, const LogU &u)
     p = fmaxf(p, 1e-30f);
     const float lx = u.K * __logf(p);
     const float x = __expf(lx);
-    if (x < 1e-3f) {
-        const float r = x / (1.f - x);
-        const float tail = u.a3 * r * (1.f + u.a4 * r * (1.f + u.a5 * r * (1.f + u.a6 * r)));
-        return u.lnC2 + 2.f * lx + (u.L - 2.f) * log1pf(-x) + log1pf(tail);
-    }
-    const float y = (u.L - 1.f) * log1pf(-x) + log1pf((u.L - 1.f) * x);
-    return __logf(-expm1f(y));
+    const bool small = x < 1e-3f;
+    const float r = __fdividef(x, 1.f - x);
+    const float tail = u.a3 * r * (1.f + u.a4 * r * (1.f + u.a5 * r * (1.f + u.a6 * r)));
+    const float l1 = log1pf(-x);
+    const float l2 = log1pf(small ? tail : (u.L - 1.f) * x);
+    if (small) return u.lnC2 + 2.f * lx + (u.L - 2.f) * l1 + l2;
+    return __logf(-expm1f((u.L - 1.f) * l1 + l2));
 }
 
 }  // namespace mp

@@ -134,6 +134,37 @@ def test_tc_attention_ragged_lengths_and_boundaries():
     assert np.isneginf(gpu["lse"][0]).all() and not gpu["out"][0].any()
 
 
+def test_ragged_batch_of_many_units():
+    """A mid-size ragged batch (16 sequences x 8 kv heads, lengths 1500 to
+    8192): every unit's candidate set against the oracle's collision rule on
+    the same codes, and the outputs of units spread over the length range."""
+    w = TINY.with_(name="pipe", batch=16, n_q_heads=32, n_kv_heads=8, context=8192, ragged_min=1500,
+                   n_planted=16, seed=2015)
+    inp = make_inputs(w)
+    run = Run(w, inp)
+    run.hash_keys()
+    qref, _ = oracle_query_codes(inp, w)
+    gpu = run.decode(qcodes_in=qref)
+    assert gpu["status"] == 0
+    units = all_units(w)
+    G = w.group
+    lens = inp["seq_lens"]
+    keep = set(_spread(units, lens, 6))
+    kept = {}
+    for b, kh in units:
+        n = int(lens[b])
+        g = run.codes_logical(b, kh, n)
+        hs = slice(kh * G, (kh + 1) * G)
+        mem, ns = oracle.collide(g, qref[b, hs], w.sink, w.window)
+        np.testing.assert_array_equal(gpu["member"][b, hs, :n], mem, err_msg=f"member b={b} kh={kh}")
+        np.testing.assert_array_equal(gpu["ns"][b, hs], ns)
+        if (b, kh) in keep:
+            kept[(b, kh)] = g
+    picked = sorted(kept)
+    ref = oracle_decode_units(inp, w, picked, [kept[u] for u in picked], qref)
+    check_outputs(gpu, ref, w)
+
+
 PLANE_CASES = ["g4_k10", "g2_k10_short", "g4_k8_planes", "g1_k8_planes_short"]
 
 

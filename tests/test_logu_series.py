@@ -48,3 +48,4 @@ def test_dropping_the_sixth_term_would_break_the_bound(oracle_mod):
     short = math.log(L * (L - 1) / 2) + 2 * math.log(xb) + (L - 2) * math.log1p(-xb) + \
         math.log1p(a3 * r * (1 + a4 * r * (1 + a5 * r)))
     assert abs(short - exact) > 4e-7
+
