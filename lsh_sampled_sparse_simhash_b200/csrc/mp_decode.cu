@@ -55,17 +55,23 @@ __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__r
     const int l0 = blockIdx.x * TB;
     const size_t vec0 = (size_t)u0 * G;  // query vectors of a unit are consecutive: (b Hkv + kvh) G + g
 
-    grid_dependency_wait();
-    if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) {
-        status[0] = 0;  // the call's status word
-        status[1] = 0;  // the attention kernel's work counter
-    }
-
+    // q and W are never written by this library, and every kernel that reads
+    // the query codes of an earlier call has completed before this one starts
+    // (see grid_launch_dependents), so the codes are computed and written
+    // before the wait for the predecessor; only the status word waits.
+    auto finish = [&]() {
+        grid_dependency_wait();
+        if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) {
+            status[0] = 0;  // the call's status word
+            status[1] = 0;  // the attention kernel's work counter
+        }
+    };
     if (qcodes_in) {
         for (int i = tid; i < nu * G * TB; i += blockDim.x) {
             const int v = i / TB, l = l0 + i % TB;
             if (l < s.L) qcodes[(vec0 + v) * s.L + l] = qcodes_in[(vec0 + v) * s.L + l];
         }
+        finish();
         return;
     }
     // this lane's W quarter row first: its load overlaps the q staging below
@@ -123,6 +129,7 @@ __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__r
             qcodes[(vec0 + v) * s.L + l] = (uint16_t)code;
         }
     }
+    finish();
 }
 
 // Units per query-hash block: the most (up to kQhashVecs / G query vectors)
@@ -283,7 +290,10 @@ __device__ __forceinline__ uint32_t h2_at_least_2(uint32_t cnt)
 }
 
 constexpr int kByteWarps = 8;   // chunks (warps) per block
-constexpr int kByteRing = 12;   // tables in each warp's shared-memory ring (11 copies in flight)
+#ifndef MP_BYTE_RING
+#define MP_BYTE_RING 12
+#endif
+constexpr int kByteRing = MP_BYTE_RING;  // tables in each warp's shared-memory ring (one less in flight)
 
 // Each lane copies its own 16 code bytes of a table into its slot of the
 // warp's ring (cp.async, 16 bytes, bypassing L1) and reads back only that
@@ -1616,10 +1626,20 @@ __global__ void __launch_bounds__(32 * kMergeWarps) merge_kernel(Shape s, const 
     const int b = bh / s.Hq, h = bh % s.Hq, kvh = h / G, g = h % G;
     const int unit = b * s.Hkv + kvh;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    grid_dependency_wait();
+    // the lengths come from work before this kernel's predecessor, and so do
+    // the per-chunk counts when a separate scan kernel wrote them (has_d; the
+    // fused kernel, the predecessor otherwise, writes them itself): those
+    // reads go before the wait
     int N = seq_lens[b];
     N = N < 0 ? 0 : (N > max_len ? max_len : N);
     const int nch = (N + chunk_tokens - 1) / chunk_tokens;
+    int ns = 0;
+    auto count_sampled = [&]() {
+        for (int j = tid; j < nch; j += blockDim.x) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
+    };
+    if (has_d) count_sampled();
+    grid_dependency_wait();
+    if (!has_d) count_sampled();
     const int nsp = ((nch + span - 1) / span) * subs;  // live chunk splits
     const int dsp = ngroups * subs;                     // the exact-set split (if has_d)
     const size_t base = (size_t)bh * (dsp + 1);
@@ -1628,9 +1648,6 @@ __global__ void __launch_bounds__(32 * kMergeWarps) merge_kernel(Shape s, const 
     // stay inside the partial arrays), only the fold does
     auto live = [&](int j) { return j < nsp || (has_d && j == dsp); };
 
-    // n_sampled: the chunks' per-head counts
-    int ns = 0;
-    for (int j = tid; j < nch; j += blockDim.x) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
     // each warp folds splits warp, warp + 4, ... with a running maximum; the
     // loads of kMergeBatch splits go out together before any of them is used
     float m = -INFINITY, Ls = 0.f;
@@ -1741,20 +1758,24 @@ struct SplitPlan {
     int nchunk, span, subs, ngroups, nsplit;
 };
 
+#ifndef MP_ATT_TARGET_BLOCKS
+#define MP_ATT_TARGET_BLOCKS 2400
+#endif
 static SplitPlan split_plan(const Shape &s, int max_len)
 {
+    constexpr int kTarget = MP_ATT_TARGET_BLOCKS;
     SplitPlan p;
     const int C = chunk_tokens(s);
     p.nchunk = (max_len + C - 1) / C;
     const int blocks = p.nchunk * s.B * s.Hkv;
-    if (blocks >= 1200) {
-        p.span = std::min(kMaxSpan, blocks / 1200);
+    if (blocks >= kTarget) {
+        p.span = std::min(kMaxSpan, blocks / kTarget);
         p.subs = 1;
     } else {
-        // few chunks: split each chunk's list so that about 1200 blocks run,
+        // few chunks: split each chunk's list so that about kTarget blocks run,
         // but give every block at least ~1024 tokens' worth of candidates
         p.span = 1;
-        const int by_count = blocks > 0 ? (1200 + blocks - 1) / blocks : 1;
+        const int by_count = blocks > 0 ? (kTarget + blocks - 1) / blocks : 1;
         p.subs = std::max(1, std::min({8, by_count, C / 1024}));
     }
     p.ngroups = (p.nchunk + p.span - 1) / p.span;

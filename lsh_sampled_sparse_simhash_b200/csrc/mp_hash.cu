@@ -42,11 +42,12 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
     uint16_t *wsm = reinterpret_cast<uint16_t *>(sm_raw);
     float *xs = reinterpret_cast<float *>(sm_raw + (size_t)T * s.K * kHeadDim * 2);
     uint8_t *bits = reinterpret_cast<uint8_t *>(xs + s.Hkv * (kHeadDim + 4));
-    grid_dependency_wait();
-    // the block's W rows into shared memory first: they do not wait for the position
+    // the block's W rows into shared memory first: no kernel writes W, so the
+    // copies go out before the wait for the predecessor
     for (int i = tid; i < ncol * (kHeadDim / 8); i += blockDim.x)
         cp_async_16(wsm + (size_t)i * 8, W + (size_t)c_begin * kHeadDim + (size_t)i * 8, 16);
     cp_async_commit();
+    grid_dependency_wait();
     const int pos = seq_lens[b];
     asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");  // (release) this block has read pos
     const bool ok = pos >= 0 && pos < s.Ncap;
