@@ -68,6 +68,10 @@ def parse(argv=None):
                    help="key-code layout (default: the workload's, i.e. bytes for K=8, planes for K=10)")
     p.add_argument("--no-graph", action="store_true",
                    help="launch every timed step eagerly instead of replaying a captured CUDA graph")
+    p.add_argument("--k-format", default="bf16", choices=["bf16", "int8"],
+                   help="K rows gathered by the attention: the bf16 cache, or its int8 copy (per-row "
+                        "power-of-two scale; opt-in reduced precision, written by mp_quantize_keys and "
+                        "mp_append_token_q8)")
     p.add_argument("--decode-path", default="auto", choices=["auto", "split", "fused", "tc"],
                    help="decode kernels: auto, split (scan then attention), fused (one kernel; bit planes) or tc "
                         "(scan then the tcgen05 attention kernel)")
@@ -113,15 +117,22 @@ def step_tokens(lens_after):
     return int(np.sum(lens_after))
 
 
-def decode_bytes(w, lens_after, union_rows):
+def row_bytes(w, k_format="bf16"):
+    """Bytes of one gathered (token, kv head) row: k + v in bf16 (512 at
+    d = 128), or the int8 k, its 16-byte {scale, norm} record and the bf16 v
+    (400)."""
+    return (w.head_dim + 16 if k_format == "int8" else 2 * w.head_dim) + 2 * w.head_dim
+
+
+def decode_bytes(w, lens_after, union_rows, k_format="bf16"):
     """Algorithmic HBM bytes of one decode over post-append lengths: the key
     codes of every (token, kv head) (L*K/8 bytes each), the unique sampled
-    K/V rows and the exact-set rows (512 bytes per row: k + v, bf16)."""
+    K/V rows and the exact-set rows (row_bytes each)."""
     LK = w.n_tables * w.k_bits
     code_bytes = int(np.sum(lens_after)) * w.n_kv_heads * LK // 8
     d_rows = sum(min(w.sink, int(n)) + int(n) - max(min(w.sink, int(n)), int(n) - w.window)
                  for n in lens_after) * w.n_kv_heads
-    return code_bytes + (union_rows + d_rows) * 2 * w.head_dim * 2, code_bytes, d_rows
+    return code_bytes + (union_rows + d_rows) * row_bytes(w, k_format), code_bytes, d_rows
 
 
 def step_description(w):
@@ -189,7 +200,7 @@ class ClockSampler:
 # --------------------------------------------------------- our arm ----
 
 class Bench:
-    def __init__(self, w, device, path="auto"):
+    def __init__(self, w, device, path="auto", k_format="bf16"):
         import torch
         import lsh_sampled_sparse_simhash_b200 as mp
         from workloads import make_inputs
@@ -229,22 +240,39 @@ class Bench:
                      "tc": mp.MP_PATH_TC}[path]
         self.graph_error = None
         self.with_hash = hash_in_step(w)
+        self.q8 = k_format == "int8"
+        if self.q8:
+            self.k8 = torch.empty((B, w.n_kv_heads, w.capacity, d), dtype=torch.int8, device=device)
+            self.kmeta = torch.empty((B, w.n_kv_heads, w.capacity, 4), dtype=torch.float32, device=device)
         fused = self.path == mp.MP_PATH_FUSED
-        # append 1, decode: qhash + (scan, attention | fused) + merge; hash 1 if in the step
-        self.launches_per_step = 1 + (3 if fused else 4) + (1 if self.with_hash else 0)
+        # append 1, decode: qhash + (scan, attention | fused) + merge; hash 1
+        # (and with int8 keys the quantisation, 1) if in the step
+        self.launches_per_step = 1 + (3 if fused else 4) + ((2 if self.q8 else 1) if self.with_hash else 0)
         # prefill: the codes of the cached keys (the step's append adds the new token's)
         self.hash()
         torch.cuda.synchronize()
 
     def hash(self):
         self.mp.hash_keys(self.shape, self.K, self.W, self.prefill, self.codes, seq_lens=self.lens0)
+        if self.q8:
+            self.mp.quantize_keys(self.shape, self.K, self.k8, self.kmeta, n_tokens=self.prefill,
+                                  seq_lens=self.lens0)
 
     def append(self):
-        self.mp.append_token(self.shape, self.k_new, self.v_new, self.W, self.K, self.V, self.codes, self.lens)
+        if self.q8:
+            self.mp.append_token_q8(self.shape, self.k_new, self.v_new, self.W, self.K, self.V, self.codes,
+                                    self.lens, self.k8, self.kmeta)
+        else:
+            self.mp.append_token(self.shape, self.k_new, self.v_new, self.W, self.K, self.V, self.codes, self.lens)
 
-    def decode(self):
-        self.mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
-                              self.out, self.lse, self.ns, self.ws, path=self.path)
+    def decode(self, member_out=None):
+        if self.q8:
+            self.mp.decode_attend_q8(self.shape, self.q, self.W, self.codes, self.k8, self.kmeta, self.V,
+                                     self.lens, self.max_len, self.out, self.lse, self.ns, self.ws,
+                                     member_out=member_out, path=self.path)
+        else:
+            self.mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
+                                  self.out, self.lse, self.ns, self.ws, member_out=member_out, path=self.path)
 
     def calls(self):
         """The library calls of one step (the lengths are reset before it)."""
@@ -263,8 +291,7 @@ class Bench:
         w = self.w
         self.step()
         mem = torch.zeros((w.batch, w.n_q_heads, w.capacity), dtype=torch.uint8, device=self.q.device)
-        self.mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
-                              self.out, self.lse, self.ns, self.ws, member_out=mem, path=self.path)
+        self.decode(member_out=mem)
         torch.cuda.synchronize()
         m = mem.view(w.batch, w.n_kv_heads, w.group, w.capacity).amax(dim=2)
         u = int(m.sum().item())
@@ -655,7 +682,7 @@ def main():
     import __graft_entry__
     __graft_entry__.build()
     w = workload_for_rank(args.workload, rank, args.code_layout)
-    bench = Bench(w, device, args.decode_path)
+    bench = Bench(w, device, args.decode_path, args.k_format)
     union, mean_ns = bench.union_rows()
 
     def barrier():
@@ -697,7 +724,7 @@ def main():
         peaks = load_peaks()
         layout = config_of(w)["code_layout"]
         lens_after = bench.inp["seq_lens"] + 1
-        dec_bytes, code_bytes, d_rows = decode_bytes(w, lens_after, union)
+        dec_bytes, code_bytes, d_rows = decode_bytes(w, lens_after, union, args.k_format)
         LK = w.n_tables * w.k_bits
         hash_rows = int(bench.inp["seq_lens"].sum()) * w.n_kv_heads
         hash_flops = 2.0 * hash_rows * w.head_dim * LK
@@ -716,7 +743,7 @@ def main():
         dec_roof = dict(kernel="mp_decode_attend (qhash + scan + attend + merge)", bound="hbm",
                         achieved=dec_bytes / (decode_ms / 1e3) / 1e9, peak=peaks["hbm"], unit="GB/s",
                         algorithmic=dec_bytes, units=dec_units,
-                        traffic=traffic_record("decode", w.name, layout))
+                        traffic=traffic_record("decode" if args.k_format == "bf16" else "decode_q8", w.name, layout))
         dec_roof["frac"] = dec_roof["achieved"] / dec_roof["peak"]
         dec_roof["frac_of_nominal_8tbs"] = dec_roof["achieved"] / 8000.0  # nominal HBM3e figure, for context
         ms_step = total_ms / args.steps
@@ -733,13 +760,16 @@ def main():
                                    "merge), timed over the timed region")
         roofline["peak_source"] = peaks["source"] + " HBM copy"
         roofline["algorithmic_bytes"] = dec_bytes
-        roofline["bytes"] = dict(codes=code_bytes, union_rows=union, exact_rows=d_rows, row_bytes=2 * w.head_dim * 2)
+        roofline["bytes"] = dict(codes=code_bytes, union_rows=union, exact_rows=d_rows,
+                                 row_bytes=row_bytes(w, args.k_format))
         roofline["frac_of_nominal_8tbs"] = roofline["achieved"] / 8000.0
         line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True,
-                    scaling="weak", vs_baseline=None, dtype="bf16-in/fp32-acc", data="synthetic",
+                    scaling="weak", vs_baseline=None,
+                    dtype="bf16-in/fp32-acc" if args.k_format == "bf16" else
+                    "bf16 q/v + int8 k (per-row power-of-two scale)/fp32-acc", data="synthetic",
                     config=config_of(w),
-                    launch=dict(decode_path=args.decode_path,
+                    launch=dict(decode_path=args.decode_path, k_format=args.k_format,
                                 mode="cuda-graph replay per step" if graph is not None else
                                 "eager launches" + (f" ({bench.graph_error})" if bench.graph_error else "")),
                     roofline=roofline,

@@ -10,16 +10,19 @@ from ._binding import (  # noqa: F401
     MagicPIGError,
     Shape,
     append_token,
+    append_token_q8,
     codes_bytes,
     codes_shape,
     decode_attend,
     decode_attend_noalloc,
+    decode_attend_q8,
     decode_workspace_bytes,
     hash_keys,
     hash_keys_range,
     hash_queries,
     library,
     library_path,
+    quantize_keys,
     read_status,
     status_string,
     MP_OK,
@@ -40,8 +43,8 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "MagicPIGError", "Shape", "append_token", "codes_bytes", "codes_shape", "decode_attend",
-    "decode_attend_noalloc",
+    "MagicPIGError", "Shape", "append_token", "append_token_q8", "codes_bytes", "codes_shape", "decode_attend",
+    "decode_attend_noalloc", "decode_attend_q8", "quantize_keys",
     "decode_workspace_bytes", "hash_keys", "hash_keys_range", "hash_queries", "library", "library_path", "read_status",
     "status_string",
 ]

@@ -25,6 +25,7 @@
 
 #include "mp_common.cuh"
 #include "mp_kernels.cuh"
+#include "mp_kquant.cuh"
 #include "mp_logu.cuh"
 
 namespace mp {
@@ -725,6 +726,12 @@ constexpr int kAttStages = 2;               // cp.async ring depth (3 blocks fit
 constexpr int kRowBytes = kHeadDim * 2;     // 256
 constexpr int kRowStride = kRowBytes + 16;  // padded: conflict-free ldmatrix / 8-byte reads
 constexpr int kStageBytes = kAttRows * kRowStride * 2;  // K rows then V rows
+// int8 keys (mp_decode_attend_q8): 128-byte rows, padded to 144 (conflict-free ldmatrix)
+constexpr int kRowStrideQ8 = kHeadDim + 16;
+template <bool Q8>
+constexpr int att_k_stride() { return Q8 ? kRowStrideQ8 : kRowStride; }
+template <bool Q8>
+constexpr int att_stage_bytes() { return kAttRows * (att_k_stride<Q8>() + kRowStride); }
 
 struct AttendArgs {
     Shape s;
@@ -743,6 +750,8 @@ struct AttendArgs {
     float *pm, *pl, *pacc;  // [B*Hq][ngroups*subs+1], [..][..][128]
     LogU lu;
     float scale;  // 1/sqrt(d)
+    const int8_t *k8;      // int8 keys [B][Hkv][Ncap][128] (attend_kernel<G, true>), else null
+    const float *kmeta;    // their per-row records {scale, squared norm, 0, 0} [B][Hkv][Ncap][4]
 };
 
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
@@ -758,6 +767,43 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
 {
     uint32_t r;
     asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(r) : "r"(x));
+    return r;
+}
+
+__device__ __forceinline__ void ldmatrix_x2(uint32_t &r0, uint32_t &r1, const void *smem_row)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(smem_u32(smem_row)));
+}
+
+// D(16x8, fp32) += A(16x16, f16, row) * B(16x8, f16, col)
+__device__ __forceinline__ void mma_f16_16816(float &d0, float &d1, float &d2, float &d3, uint32_t a0, uint32_t a1,
+                                              uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four int8 values (bytes of r) -> two f16x2, exactly: byte b becomes the half
+// 0x6400 | (b ^ 0x80), i.e. 1024 + b + 128, and 1152 is subtracted.
+__device__ __forceinline__ void s8x4_to_f16x2(uint32_t r, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t x = r ^ 0x80808080u;
+    asm("prmt.b32 %0, %1, %2, 0x4140;" : "=r"(lo) : "r"(x), "r"(0x64646464u));  // bytes 0, 1
+    asm("prmt.b32 %0, %1, %2, 0x4342;" : "=r"(hi) : "r"(x), "r"(0x64646464u));  // bytes 2, 3
+    asm("add.rn.f16x2 %0, %0, %1;" : "+r"(lo) : "r"(0xE480E480u));                // - 1152
+    asm("add.rn.f16x2 %0, %0, %1;" : "+r"(hi) : "r"(0xE480E480u));
+}
+
+// {lo, hi} -> f16x2 (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
 
@@ -803,16 +849,25 @@ struct AttnWarp {
 
 // Loads the Q^T fragments of the G heads starting at query vector vec0 and
 // clears the state (the 1/|q| values come later, from attn_qinv's shared array).
-template <int G>
+// With int8 keys (Q8) the fragments are f16 and follow the keys' dimension
+// order inside each 16-dim step (see attn_tile): slots 2t, 2t + 1, 2t + 8,
+// 2t + 9 of step ks hold dims 16 ks + 4t .. 16 ks + 4t + 3.
+template <int G, bool Q8 = false>
 __device__ __forceinline__ void attn_begin(AttnWarp<G> &w, const uint16_t *q, size_t vec0, int lane)
 {
     const int gq = lane >> 2, tq = lane & 3;
 #pragma unroll
     for (int ks = 0; ks < 8; ks++) {
         if (gq < G) {
-            const uint32_t *qp = reinterpret_cast<const uint32_t *>(q + (vec0 + gq) * kHeadDim);
-            w.qb[ks][0] = qp[(ks * 16 + 2 * tq) >> 1];
-            w.qb[ks][1] = qp[(ks * 16 + 2 * tq + 8) >> 1];
+            if constexpr (Q8) {
+                const uint16_t *qp = q + (vec0 + gq) * kHeadDim + ks * 16 + 4 * tq;
+                w.qb[ks][0] = pack_f16x2(bf16_to_f32(qp[0]), bf16_to_f32(qp[1]));
+                w.qb[ks][1] = pack_f16x2(bf16_to_f32(qp[2]), bf16_to_f32(qp[3]));
+            } else {
+                const uint32_t *qp = reinterpret_cast<const uint32_t *>(q + (vec0 + gq) * kHeadDim);
+                w.qb[ks][0] = qp[(ks * 16 + 2 * tq) >> 1];
+                w.qb[ks][1] = qp[(ks * 16 + 2 * tq + 8) >> 1];
+            }
         } else {
             w.qb[ks][0] = w.qb[ks][1] = 0u;
         }
@@ -850,10 +905,18 @@ __device__ __forceinline__ void attn_set_qinv(AttnWarp<G> &w, const float *qinv,
 // One 64-row tile for this warp: its 16 K rows at ks_ and V rows at vs_
 // (kRowStride apart, the tile's rows 16 warp ..), meta[64] = the rows' head
 // masks (| 0x100 for the exact set); ucos / uval are this warp's [16 G] scratch.
-template <int G>
+//
+// With int8 keys (Q8): K rows are 128 bytes (kRowStrideQ8 apart) and kq
+// holds the 16 rows' {scale, squared norm} records.  One ldmatrix.x2 per
+// 16-dim step gives lane (g, t) the bytes of dims 4t .. 4t + 3 of rows g and
+// g + 8; widened exactly to f16 they fill fragment slots 2t, 2t + 1, 2t + 8,
+// 2t + 9, a fixed permutation of the step's dims that the query fragments
+// follow too (attn_begin), so the dot products are unchanged.  Scores are
+// scaled by the row's scale; |k|^2 is the stored norm (no Gram products).
+template <int G, bool Q8 = false>
 __device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, const uint8_t *vs_,
                                           const uint32_t *meta, int warp, int lane, float scale, const LogU &lu,
-                                          float *ucos, float *uval)
+                                          float *ucos, float *uval, const float4 *kq = nullptr)
 {
     const float scale2 = scale * kLog2e;  // scores in log2 units
     const int gq = lane >> 2, tq = lane & 3;
@@ -864,23 +927,42 @@ __device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, co
     float c[4] = {0.f, 0.f, 0.f, 0.f};
     float na, nb;
     {
-        float g0[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStride + (lane >> 4) * 16;
+        if constexpr (Q8) {
+            const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStrideQ8;
 #pragma unroll
-        for (int kst = 0; kst < 8; kst++) {
-            uint32_t a0, a1, a2, a3;
-            ldmatrix_x4(a0, a1, a2, a3, arow + kst * 32);
-            mma_bf16_16816(c[0], c[1], c[2], c[3], a0, a1, a2, a3, w.qb[kst][0], w.qb[kst][1]);
-            mma_bf16_16816(g0[0], g0[1], g0[2], g0[3], a0, a1, a2, a3, a0, a2);  // columns: rows 0-7
-            mma_bf16_16816(g1[0], g1[1], g1[2], g1[3], a0, a1, a2, a3, a1, a3);  // columns: rows 8-15
+            for (int kst = 0; kst < 8; kst++) {
+                uint32_t r0, r1, a0, a1, a2, a3;
+                ldmatrix_x2(r0, r1, arow + kst * 16);
+                s8x4_to_f16x2(r0, a0, a2);
+                s8x4_to_f16x2(r1, a1, a3);
+                mma_f16_16816(c[0], c[1], c[2], c[3], a0, a1, a2, a3, w.qb[kst][0], w.qb[kst][1]);
+            }
+            const float4 m0 = kq[warp * 16 + gq], m1 = kq[warp * 16 + gq + 8];
+            c[0] *= m0.x;
+            c[1] *= m0.x;
+            c[2] *= m1.x;
+            c[3] *= m1.x;
+            na = m0.y;
+            nb = m1.y;
+        } else {
+            float g0[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStride + (lane >> 4) * 16;
+#pragma unroll
+            for (int kst = 0; kst < 8; kst++) {
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4(a0, a1, a2, a3, arow + kst * 32);
+                mma_bf16_16816(c[0], c[1], c[2], c[3], a0, a1, a2, a3, w.qb[kst][0], w.qb[kst][1]);
+                mma_bf16_16816(g0[0], g0[1], g0[2], g0[3], a0, a1, a2, a3, a0, a2);  // columns: rows 0-7
+                mma_bf16_16816(g1[0], g1[1], g1[2], g1[3], a0, a1, a2, a3, a1, a3);  // columns: rows 8-15
+            }
+            // |k_r|^2 = Gram[r][r]: row gq sits in lane 4 gq + gq/2 (g0, element gq & 1),
+            // row gq + 8 in the same lane (g1, element 2 + (gq & 1)).
+            const int src = 4 * gq + (gq >> 1);
+            const float d0 = (gq & 1) ? g0[1] : g0[0];
+            const float d1 = (gq & 1) ? g1[3] : g1[2];
+            na = __shfl_sync(0xffffffffu, d0, src);
+            nb = __shfl_sync(0xffffffffu, d1, src);
         }
-        // |k_r|^2 = Gram[r][r]: row gq sits in lane 4 gq + gq/2 (g0, element gq & 1),
-        // row gq + 8 in the same lane (g1, element 2 + (gq & 1)).
-        const int src = 4 * gq + (gq >> 1);
-        const float d0 = (gq & 1) ? g0[1] : g0[0];
-        const float d1 = (gq & 1) ? g1[3] : g1[2];
-        na = __shfl_sync(0xffffffffu, d0, src);
-        nb = __shfl_sync(0xffffffffu, d1, src);
     }
 
     // ---- log-weights: s (exact) or s - log u (sampled), -inf if absent ----
@@ -1030,13 +1112,15 @@ __device__ __forceinline__ void attn_store_partial(AttnWarp<G> &w, float *red, i
     }
 }
 
-template <int G>
+template <int G, bool Q8>
 __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     constexpr int kWarpRows = kAttRows / 4;                   // rows of a tile per warp
-    constexpr int kWarpStage = kWarpRows * kRowStride * 2;    // one warp's K rows then V rows
+    constexpr int KS = att_k_stride<Q8>();                    // K row stride in shared memory
+    constexpr int kWarpStage = kWarpRows * (KS + kRowStride); // one warp's K rows then V rows
     __shared__ uint32_t meta[4][kAttStages][kWarpRows];       // per warp: headmask | exact << 8
+    __shared__ float4 kq[Q8 ? 4 : 1][Q8 ? kAttStages : 1][kWarpRows];  // int8 keys: {scale, |k|^2} per row
     __shared__ float ucos[4][16 * G];                // per warp: cos of pairs needing log u
     __shared__ float uval[4][16 * G];                // per warp: their log u
     __shared__ float qinv[G];
@@ -1110,10 +1194,12 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
 
     const size_t vec0 = (size_t)b * s.Hq + (size_t)kvh * G;
     AttnWarp<G> w;
-    attn_begin<G>(w, a.q, vec0, lane);
+    attn_begin<G, Q8>(w, a.q, vec0, lane);
     attn_qinv<G>(a.q, vec0, warp, lane, qinv);
 
-    const uint16_t *kbase = a.kc + (size_t)unit * s.Ncap * kHeadDim;
+    const uint16_t *kbase = Q8 ? nullptr : a.kc + (size_t)unit * s.Ncap * kHeadDim;
+    const int8_t *k8base = Q8 ? a.k8 + (size_t)unit * s.Ncap * kHeadDim : nullptr;
+    const float *kmbase = Q8 ? a.kmeta + (size_t)unit * s.Ncap * kQ8MetaFloats : nullptr;
     const uint16_t *vbase = a.vc + (size_t)unit * s.Ncap * kHeadDim;
     const int ntiles = (nrows + kAttRows - 1) / kAttRows;
 
@@ -1138,7 +1224,7 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
 
     auto issue = [&](int tile, int stage) {
         uint8_t *ks_ = wring + stage * kWarpStage;
-        uint8_t *vs_ = ks_ + kWarpRows * kRowStride;
+        uint8_t *vs_ = ks_ + kWarpRows * KS;
         const int col = lane & 15;
 #pragma unroll
         for (int i = 0; i < kWarpRows / 2; i++) {
@@ -1147,7 +1233,16 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
             const bool ok = ent != 0xFFFFFFFFu;
             const int tok = ok ? (int)(ent & 0xFFFFFFu) : 0;
             const size_t off = (size_t)tok * kHeadDim + col * 8;
-            cp_async_16(ks_ + r * kRowStride + col * 16, kbase + off, ok ? 16 : 0);
+            if constexpr (Q8) {  // 8 pieces of the int8 row, then its 16-byte record
+                if (col < 9) {
+                    void *dst = col < 8 ? (void *)(ks_ + r * KS + col * 16) : (void *)&kq[warp][stage][r];
+                    const void *src = col < 8 ? (const void *)(k8base + (size_t)tok * kHeadDim + col * 16)
+                                              : (const void *)(kmbase + (size_t)tok * kQ8MetaFloats);
+                    cp_async_16(dst, src, ok ? 16 : 0);
+                }
+            } else {
+                cp_async_16(ks_ + r * KS + col * 16, kbase + off, ok ? 16 : 0);
+            }
             cp_async_16(vs_ + r * kRowStride + col * 16, vbase + off, ok ? 16 : 0);
             if (col == 0) meta[warp][stage][r] = ok ? (dsplit ? dmeta : (ent >> 24)) : 0u;
         }
@@ -1177,8 +1272,8 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
         const int stage = tile % kAttStages;
         const uint8_t *ks_ = wring + stage * kWarpStage;
         // the warp's own 16 rows, addressed as warp 0 of a tile
-        attn_tile<G>(w, ks_, ks_ + kWarpRows * kRowStride, meta[warp][stage], 0, lane, a.scale, a.lu, ucos[warp],
-                     uval[warp]);
+        attn_tile<G, Q8>(w, ks_, ks_ + kWarpRows * KS, meta[warp][stage], 0, lane, a.scale, a.lu, ucos[warp],
+                         uval[warp], kq[Q8 ? warp : 0][Q8 ? stage : 0]);
         if (fetcher) ents[warp][tile & 1][lane] = pend;  // slot of tile + 2, read after the next __syncwarp
         __syncwarp();  // the stage may be refilled next iteration
     }
@@ -1904,7 +1999,8 @@ template <int G>
 static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint16_t *W, const void *codes,
                                    const uint16_t *kc, const uint16_t *vc, const int32_t *seq_lens,
                                    int max_len, float *out, float *lse, int32_t *n_sampled,
-                                   const Workspace &ws, const mp_decode_debug *dbg, cudaStream_t st)
+                                   const Workspace &ws, const mp_decode_debug *dbg, cudaStream_t st,
+                                   const int8_t *k8, const float *kmeta)
 {
     const int C = chunk_tokens(s);
     const SplitPlan sp = split_plan(s, max_len);
@@ -1987,11 +2083,18 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
 
     aa.lu = lu;
     aa.scale = scale;
-    if (!fused && path != MP_PATH_TC) {
-        const int sm = kAttStages * kStageBytes;
-        if ((e = ensure_smem(reinterpret_cast<const void *>(attend_kernel<G>), sm)) != cudaSuccess) return e;
+    aa.k8 = k8;
+    aa.kmeta = kmeta;
+    if (!fused && path != MP_PATH_TC && k8) {
+        const int sm = kAttStages * att_stage_bytes<true>();
+        if ((e = ensure_smem(reinterpret_cast<const void *>(attend_kernel<G, true>), sm)) != cudaSuccess) return e;
         dim3 grid(sp.nsplit, units);
-        if ((e = launch_pdl(attend_kernel<G>, grid, dim3(kAttThreads), sm, st, aa)) != cudaSuccess) return e;
+        if ((e = launch_pdl(attend_kernel<G, true>, grid, dim3(kAttThreads), sm, st, aa)) != cudaSuccess) return e;
+    } else if (!fused && path != MP_PATH_TC) {
+        const int sm = kAttStages * att_stage_bytes<false>();
+        if ((e = ensure_smem(reinterpret_cast<const void *>(attend_kernel<G, false>), sm)) != cudaSuccess) return e;
+        dim3 grid(sp.nsplit, units);
+        if ((e = launch_pdl(attend_kernel<G, false>, grid, dim3(kAttThreads), sm, st, aa)) != cudaSuccess) return e;
     } else if (!fused) {
         AttendTcArgs ta;
         ta.s = s;
@@ -2031,14 +2134,14 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
 cudaError_t launch_decode(const Shape &s, const uint16_t *q, const uint16_t *W, const void *codes,
                           const uint16_t *kc, const uint16_t *vc, const int32_t *seq_lens, int max_len,
                           float *out, float *lse, int32_t *n_sampled, void *workspace,
-                          const mp_decode_debug *dbg, cudaStream_t st)
+                          const mp_decode_debug *dbg, cudaStream_t st, const int8_t *k8, const float *kmeta)
 {
     const Workspace ws = workspace_layout(s, max_len, workspace);
     switch (s.G) {
-    case 1: return launch_decode_g<1>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st);
-    case 2: return launch_decode_g<2>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st);
-    case 4: return launch_decode_g<4>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st);
-    case 8: return launch_decode_g<8>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st);
+    case 1: return launch_decode_g<1>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8, kmeta);
+    case 2: return launch_decode_g<2>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8, kmeta);
+    case 4: return launch_decode_g<4>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8, kmeta);
+    case 8: return launch_decode_g<8>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8, kmeta);
     default: return cudaErrorInvalidValue;
     }
 }

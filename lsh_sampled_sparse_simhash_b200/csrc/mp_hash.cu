@@ -8,6 +8,7 @@
 //           code of token 32 w + t.
 #include "mp_common.cuh"
 #include "mp_kernels.cuh"
+#include "mp_kquant.cuh"
 
 namespace mp {
 
@@ -29,7 +30,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
                                                                 const uint16_t *__restrict__ v_new,
                                                                 const uint16_t *__restrict__ W, uint16_t *kc,
                                                                 uint16_t *vc, void *codes, int32_t *seq_lens,
-                                                                int32_t *status)
+                                                                int32_t *status, int8_t *k8, float *kmeta)
 {
     // shared: this block's W rows [T K][kHeadDim] bf16, the new keys
     // [Hkv][kHeadDim + 4] fp32 (element d at d + d / 32), the bits [Hkv][T K]
@@ -55,12 +56,19 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
         if (r == 0 && tid == 0) set_status(status, MP_ERR_CAPACITY);
     } else {
         const size_t unit0 = (size_t)b * s.Hkv;
-        if (r == 0) {  // the K and V rows, 16 bytes per thread
+        if (r == 0) {  // the K and V rows, 16 bytes per thread (no K row without a bf16 key cache)
             for (int i = tid; i < s.Hkv * 32; i += blockDim.x) {
                 const int h = i >> 5, isv = (i >> 4) & 1, e = i & 15;
+                if (!isv && !kc) continue;
                 const uint4 *src = reinterpret_cast<const uint4 *>((isv ? v_new : k_new) + (unit0 + h) * kHeadDim);
                 uint4 *dst = reinterpret_cast<uint4 *>((isv ? vc : kc) + ((unit0 + h) * s.Ncap + pos) * kHeadDim);
                 dst[e] = src[e];
+            }
+        } else if (r == 1 && k8) {  // the int8 copy of the new keys, a warp per kv head
+            for (int h = tid >> 5; h < s.Hkv; h += blockDim.x >> 5) {
+                const size_t row = (unit0 + h) * s.Ncap + pos;
+                quantize_key_row(k_new + (unit0 + h) * kHeadDim, k8 + row * kHeadDim, kmeta + row * kQ8MetaFloats,
+                                 tid & 31);
             }
         }
         for (int i = tid; i < s.Hkv * kHeadDim; i += blockDim.x) {
@@ -133,7 +141,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
 
 cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t *v_new, const uint16_t *W,
                           uint16_t *kc, uint16_t *vc, void *codes, int32_t *seq_lens, int32_t *status,
-                          cudaStream_t st)
+                          int8_t *k8, float *kmeta, cudaStream_t st)
 {
     const int T = (s.L + kAppendCluster - 1) / kAppendCluster;
     const size_t smem = (size_t)T * s.K * kHeadDim * 2 + (size_t)s.Hkv * (kHeadDim + 4) * sizeof(float) +
@@ -154,7 +162,7 @@ cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, append_kernel, s, k_new, v_new, W, kc, vc, codes, seq_lens, status);
+    return cudaLaunchKernelEx(&cfg, append_kernel, s, k_new, v_new, W, kc, vc, codes, seq_lens, status, k8, kmeta);
 }
 
 }  // namespace mp

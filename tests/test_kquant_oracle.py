@@ -1,0 +1,124 @@
+"""Pins for the int8 key format reference (oracle/kquant.py) and the accuracy
+contract of the int8 attention gather, all on the CPU.
+
+Q1  hand-worked rows: scale choice at the powers-of-two boundaries, round half
+    to even, the zero row, negative maxima
+Q2  on random rows: s is a power of two and the smallest with 127 s >= max|k|,
+    |q| <= 127, |k - s q| <= s / 2 (brute-force search of the scale exponent)
+Q3  s q is exactly a bf16 value, and quantising it again gives the same q, s;
+    the row record's squared norm is exactly |s q|^2
+Q4  the effect on the method's output: the fp64 oracle's decode on s q keys
+    stays within the int8 tolerance of its decode on the bf16 keys
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import kquant
+from workloads import WORKLOADS, bf16_bits_to_f32, f32_to_bf16_bits, make_inputs
+
+# per-head relative L2 of the int8-key decode against the bf16-key decode
+# (fp64 oracle on both); the GPU int8 path is held to this plus the bf16 path's
+# own tolerance against the oracle
+INT8_REL_L2_TOL = 2e-2
+
+
+def _bf(x):
+    return f32_to_bf16_bits(np.asarray(x, np.float32))
+
+
+def _row(vals, d=128):
+    r = np.zeros(d, np.float32)
+    r[:len(vals)] = vals
+    return _bf(r)
+
+
+@pytest.mark.parametrize("vals, s, q", [
+    ([127.0, -1.0, 0.5], 1.0, [127, -1, 0]),        # 0.5 ties to even 0
+    ([128.0, 3.0], 2.0, [64, 2]),                   # 127 * 1 < 128: one step up; 1.5 ties to even 2
+    ([-127.0, 2.5], 1.0, [-127, 2]),                # the maximum of |k| may be negative; 2.5 -> 2
+    ([63.5, 1.5], 0.5, [127, 3]),                   # 127 * 0.5 = 63.5 exactly fits
+    ([64.0, 0.75], 1.0, [64, 1]),                   # 127 * 0.5 < 64; 0.75 -> 1
+    ([0.0], 0.0, [0]),                              # zero row: s = 0, q = 0
+    ([1.0, -0.00390625], 2.0 ** -6, [64, 0]),       # -2^-8 / 2^-6 = -0.25 -> 0
+    ([3.5, 0.0546875], 2.0 ** -5, [112, 2]),        # 0.0546875 / 2^-5 = 1.75 -> 2
+])
+def test_hand_worked_rows(vals, s, q):
+    qq, ss = kquant.quantize_rows(_row(vals)[None])
+    assert ss[0] == s
+    assert list(qq[0, :len(q)]) == q
+    assert not qq[0, len(q):].any()
+
+
+def test_random_rows_bounds_and_smallest_scale():
+    rng = np.random.default_rng(3)
+    rows = rng.standard_normal((64, 128)) * np.exp(rng.uniform(-8, 8, (64, 1)))
+    kb = _bf(rows)
+    q, s = kquant.quantize_rows(kb)
+    k = bf16_bits_to_f32(kb).astype(np.float64)
+    for i in range(len(rows)):
+        amax = np.max(np.abs(k[i]))
+        # brute force: the smallest e in a wide range with 127 * 2^e >= amax
+        e = next(e for e in range(-140, 140) if 127.0 * 2.0 ** e >= amax)
+        assert s[i] == 2.0 ** e
+        assert np.all(np.abs(q[i].astype(np.int32)) <= 127)
+        assert np.all(np.abs(k[i] - s[i] * q[i]) <= s[i] / 2)
+        assert np.abs(q[i].astype(np.int32)).max() >= 64  # 63.5 s < amax, so some |q| rounds to >= 64
+
+
+def test_row_record_holds_scale_and_exact_squared_norm():
+    rng = np.random.default_rng(9)
+    kb = _bf(rng.standard_normal((16, 128)) * 3.0)
+    kb[3] = 0
+    q, s = kquant.quantize_rows(kb)
+    meta = kquant.row_meta(q, s)
+    assert meta.shape == (16, 4) and meta.dtype == np.float32
+    np.testing.assert_array_equal(meta[:, 0], s)
+    kt = bf16_bits_to_f32(kquant.dequantize_bits(q, s)).astype(np.float64)
+    np.testing.assert_array_equal(meta[:, 1].astype(np.float64), np.sum(kt * kt, axis=1))
+    assert meta[3, 1] == 0.0 and not meta[:, 2:].any()
+
+
+def test_dequantized_keys_are_bf16_and_a_fixed_point():
+    rng = np.random.default_rng(5)
+    kb = _bf(rng.standard_normal((32, 128)) * 2.0)
+    q, s = kquant.quantize_rows(kb)
+    kt = kquant.dequantize_bits(q, s)
+    np.testing.assert_array_equal(bf16_bits_to_f32(kt).astype(np.float64), q.astype(np.float64) * s[:, None])
+    q2, s2 = kquant.quantize_rows(kt)
+    np.testing.assert_array_equal(q2, q)
+    np.testing.assert_array_equal(s2, s)
+
+
+def test_int8_keys_change_the_oracle_decode_by_less_than_the_tolerance():
+    """The int8 gather's error budget, measured on the method itself: same
+    codes (hashed from the bf16 keys), keys replaced by s q."""
+    w = WORKLOADS["tiny"]
+    inp = make_inputs(w)
+    B, Hkv = w.batch, w.n_kv_heads
+    G = w.group
+    qcodes = oracle.simhash(inp["q"], inp["W"], w.k_bits, w.n_tables)
+    worst = 0.0
+    for b in range(B):
+        n = int(inp["seq_lens"][b])
+        if n == 0:
+            continue
+        for kh in range(Hkv):
+            Kb = inp["K"][b, kh, :n]
+            kc = oracle.simhash(Kb, inp["W"], w.k_bits, w.n_tables)
+            q8, s8 = kquant.quantize_rows(Kb)
+            Kt = kquant.dequantize_bits(q8, s8)
+            qs = inp["q"][b:b + 1, kh * G:(kh + 1) * G]
+            qc = qcodes[b:b + 1, kh * G:(kh + 1) * G]
+            args = dict(Kbits=w.k_bits, L=w.n_tables, sink=w.sink, window=w.window)
+            ref, _, _ = oracle.decode(qs, Kb[None, None], inp["V"][b:b + 1, kh:kh + 1, :n], kc[None, None], qc,
+                                      np.array([n], np.int32), **args)
+            alt, _, _ = oracle.decode(qs, Kt[None, None], inp["V"][b:b + 1, kh:kh + 1, :n], kc[None, None], qc,
+                                      np.array([n], np.int32), **args)
+            for g in range(G):
+                den = np.linalg.norm(ref[0, g])
+                e = np.linalg.norm(alt[0, g] - ref[0, g]) / (den if den > 0 else 1.0)
+                worst = max(worst, e)
+    assert 0.0 < worst <= INT8_REL_L2_TOL / 2, worst
