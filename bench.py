@@ -141,12 +141,20 @@ def step_description(w):
     return "append 1 token/sequence + LSH-sampled decode (key-hash build timed apart)"
 
 
+def code_layout_of(w):
+    """The key-code layout the library uses for this workload."""
+    if w.code_layout != "auto":
+        return w.code_layout
+    from lsh_sampled_sparse_simhash_b200 import auto_planes
+    return "planes" if auto_planes(w.batch, w.n_kv_heads, w.capacity, w.k_bits) else "bytes"
+
+
 def config_of(w):
     """The workload, identical on both arms (no launch or kernel-path keys)."""
     return dict(workload=w.name, batch=w.batch, q_heads=w.n_q_heads, kv_heads=w.n_kv_heads,
                 head_dim=w.head_dim, context=w.context, ragged_min=w.ragged_min or None, k_bits=w.k_bits,
                 n_tables=w.n_tables, sink=w.sink, window=w.window, planted_per_kv_head=w.n_planted,
-                code_layout=w.code_layout if w.code_layout != "auto" else ("bytes" if w.k_bits == 8 else "planes"),
+                code_layout=code_layout_of(w),
                 step=step_description(w),
                 l2="flushed between timed steps (256 MiB write)", parallelism="replicas (1 rank = 1 GPU)")
 

@@ -55,9 +55,16 @@ extern "C" {
 #define MP_ERR_TOO_LARGE (-7) /* beyond the fixed scratch of mp_decode_attend_noalloc */
 
 /* Key-code layouts (mp_shape.code_layout). */
-#define MP_CODES_AUTO 0   /* k_bits == 8: MP_CODES_BYTES; k_bits == 10: MP_CODES_PLANES */
+#define MP_CODES_AUTO 0   /* MP_CODES_PLANES, except MP_CODES_BYTES for k_bits == 8 when
+                             batch * n_kv_heads * capacity < MP_CODES_AUTO_PLANES_MIN */
 #define MP_CODES_BYTES 1  /* one byte per (table, token); k_bits == 8 only */
 #define MP_CODES_PLANES 2 /* bit planes of 32 tokens; any supported k_bits */
+/* Below this many (token, kv head) slots a K = 8 scan has too few 1024-token
+   chunks to fill the GPU with one warp each, and byte codes (512-token chunks)
+   scan faster: measured on one B200, 1 x 8 x 16.5k slots decode in 34 us with
+   bytes against 40 us with planes, 4 x 8 x 131k slots in 116 us with planes
+   against 118 us with bytes, 16 x 8 x 131k in 383 against 411 us. */
+#define MP_CODES_AUTO_PLANES_MIN (1 << 21)
 
 /*
  * Problem shape.  Supported: head_dim == 128; k_bits in {8, 10};

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     Shape,
     append_token,
     append_token_q8,
+    auto_planes,
     codes_bytes,
     codes_shape,
     decode_attend,
@@ -36,6 +37,7 @@ from ._binding import (  # noqa: F401
     MP_CODES_AUTO,
     MP_CODES_BYTES,
     MP_CODES_PLANES,
+    MP_CODES_AUTO_PLANES_MIN,
     MP_PATH_AUTO,
     MP_PATH_SPLIT,
     MP_PATH_FUSED,
@@ -43,7 +45,7 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "MagicPIGError", "Shape", "append_token", "append_token_q8", "codes_bytes", "codes_shape", "decode_attend",
+    "MagicPIGError", "Shape", "append_token", "append_token_q8", "auto_planes", "codes_bytes", "codes_shape", "decode_attend",
     "decode_attend_noalloc", "decode_attend_q8", "quantize_keys",
     "decode_workspace_bytes", "hash_keys", "hash_keys_range", "hash_queries", "library", "library_path", "read_status",
     "status_string",

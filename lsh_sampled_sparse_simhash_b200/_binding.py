@@ -43,6 +43,15 @@ class _CDebug(ctypes.Structure):
                 ("member_out", ctypes.c_void_p), ("path", ctypes.c_int32)]
 
 
+MP_CODES_AUTO_PLANES_MIN = 1 << 21  # include/magicpig.h
+
+
+def auto_planes(batch: int, n_kv_heads: int, capacity: int, k_bits: int) -> bool:
+    """MP_CODES_AUTO: bit planes, except byte codes for K = 8 problems with
+    fewer than MP_CODES_AUTO_PLANES_MIN (token, kv head) slots."""
+    return k_bits != 8 or batch * n_kv_heads * capacity >= MP_CODES_AUTO_PLANES_MIN
+
+
 @dataclasses.dataclass(frozen=True)
 class Shape:
     """Problem shape (see mp_shape in include/magicpig.h)."""
@@ -59,7 +68,10 @@ class Shape:
 
     @property
     def planes(self) -> bool:
-        return self.code_layout == MP_CODES_PLANES or (self.code_layout == MP_CODES_AUTO and self.k_bits != 8)
+        """Whether the key codes are bit planes (the library's rule for MP_CODES_AUTO)."""
+        if self.code_layout == MP_CODES_AUTO:
+            return auto_planes(self.batch, self.n_kv_heads, self.capacity, self.k_bits)
+        return self.code_layout == MP_CODES_PLANES
 
     def c(self) -> _CShape:
         return _CShape(*dataclasses.astuple(self))

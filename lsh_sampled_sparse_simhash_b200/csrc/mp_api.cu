@@ -23,8 +23,9 @@ int validate_shape(const mp_shape *in, Shape &s)
     s.L = in->n_tables;
     s.sink = in->sink;
     s.window = in->window;
-    if (in->code_layout == MP_CODES_AUTO)
-        s.planes = in->k_bits != 8;
+    if (in->code_layout == MP_CODES_AUTO)  // bit planes unless a K = 8 problem is small (see the header)
+        s.planes = in->k_bits != 8 ||
+                   (int64_t)in->batch * in->n_kv_heads * in->capacity >= MP_CODES_AUTO_PLANES_MIN;
     else if (in->code_layout == MP_CODES_BYTES)
         s.planes = 0;
     else if (in->code_layout == MP_CODES_PLANES)

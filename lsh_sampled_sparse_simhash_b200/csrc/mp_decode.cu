@@ -6,10 +6,11 @@
 //   scan    counts, per token and query head, the tables whose code equals the
 //           query's (bit-sliced counters saturating at 2), excludes the exact
 //           set D and compacts the sampled tokens (token id | head mask) in
-//           token order.  Byte codes: scan_k8_kernel, 16-byte streaming loads
-//           and a zero-byte test per 4 tokens.  Bit planes: scan_planes_kernel,
-//           persistent, 3-D TMA copies of 8 tables per stage into a ring,
-//           32 tokens per logic operation.
+//           token order.  Byte codes: scan_bytes_kernel, packed fp16
+//           compares of two tokens per instruction.  Bit planes:
+//           scan_planes_warp_kernel, 32 tokens per logic operation.  Both
+//           give each warp one chunk of one unit for all L tables, fed by
+//           the warp's own cp.async ring.
 //   attend  gathers the compacted K/V rows into a cp.async shared-memory
 //           ring, computes q.k for all query heads of the GQA group from one
 //           row load (bf16 mma.sync, fp32 accumulate), applies the -log u
@@ -417,20 +418,12 @@ __global__ void __launch_bounds__(32 * kByteWarps, G >= 8 ? 2 : MP_SCAN_BLOCKS_P
     compact_warp<G, 16, kChunkBytes>(s, unit, chunk, nchunk, t0, N, s.sink, min(N - s.window, N), hm, o, lane);
 }
 
-// ------------------------------------------------------ scan, bit planes ----
-// Bit-plane codes [unit][L][Ncap/32][K] (uint32).  Work item = one 1024-token
-// chunk of one (sequence, kv head) unit; a persistent block walks a
-// contiguous share of the live items.  Warp 8 is the producer: one 3-D TMA
-// copy (two for K = 10) brings a stage of 8 consecutive tables x the chunk's
-// 32 words x K planes into a ring of kScanStages(K) stages, tables past L
-// zero-filled.  Warps 0..7 consume: warp ts takes table 8 j + ts of stage j,
-// lane t the 32-token word t.  A token mismatches table l for head h iff some
-// plane differs from the query bit: mis = OR_b (plane_b ^ qmask_b), qmask_b =
-// 0 or ~0 from shared memory; two bit-sliced counters (seen >= 1, >= 2) per
-// head.  After an item's stages the consumers leave their counters in a
-// partial buffer (double-buffered by item parity) and go straight on; the
-// producer warp, once it has issued the next item's stages, folds the eight
-// splits and compacts the candidates, one item behind the consumers.
+// ---------------------------------------- bit planes: shared TMA pieces ----
+// Bit-plane codes [unit][L][Ncap/32][K] (uint32).  The fused scan + attend
+// kernel (fused_planes_kernel) brings them in by 3-D TMA copies: a stage is 8
+// consecutive tables x one 1024-token chunk's 32 words x K planes (two copies
+// for K = 10), tables past L zero-filled; a persistent block walks a
+// contiguous share of the live (sequence, kv head, chunk) items.
 constexpr int kScanConsumers = 8;  // consumer warps = table splits = tables per stage
 
 template <int KB>
@@ -484,238 +477,159 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, i
                  : "memory");
 }
 
-__device__ __forceinline__ void consumer_barrier() { asm volatile("bar.sync 1, %0;" ::"n"(kScanThreads) : "memory"); }
-__device__ __forceinline__ void bar_sync_all(int id) { asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kScanThreads + 32) : "memory"); }
-__device__ __forceinline__ void bar_arrive_all(int id) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kScanThreads + 32) : "memory"); }
+
+// ------------------------------------------------------ scan, bit planes ----
+// The bit-sliced test with the byte scan's structure: a warp owns one
+// 1024-token chunk of one unit for all L tables
+// (lane = one 32-token word), so no partial count ever crosses warps and no
+// block-wide barrier sits in the table loop.  A table's slab of the chunk
+// (32 words x K planes, 128 K contiguous bytes) goes through the warp's own
+// cp.async ring: the warp copies the slab in 16-byte pieces, lane i taking
+// pieces i, i + 32, .. (each copy instruction covers 512 contiguous bytes),
+// and a __syncwarp after the wait makes the other lanes' pieces visible.
+// Each 128-byte line of the slab stays one 128-byte line in shared memory (a
+// copy instruction whose pieces scatter across lines is served twice from L2).
+// K = 8: within line j the 16-byte pieces are XOR-swizzled by j & 1, so that
+// the two pieces of a word that a quarter warp reads (pieces 2t + i) fall in
+// distinct banks; K = 10: the slab is kept as is and lane t reads its 40 bytes
+// with five 8-byte loads (a half warp's 8-byte reads at stride 40 hit
+// distinct banks).
+// Per (table, head): mis = OR_b (plane_b ^ qmask_b), then s2 |= s1 & ~mis,
+// s1 |= ~mis; about K + 2 logic ops per 32 tokens.
+constexpr int kPlaneWarps = 8;
+#ifndef MP_PLANE_RING
+#define MP_PLANE_RING 8
+#endif
+constexpr int kPlaneRing = MP_PLANE_RING;  // tables in each warp's ring (one less in flight)
+
+template <int KB>
+__host__ __device__ constexpr int plane_slot_bytes() { return 32 * KB * 4; }
+
+// Shared-memory offset of 16-byte piece p of a K = 8 slab (line p >> 3,
+// position swizzled by the line's parity).
+__device__ __forceinline__ int plane_piece_k8(int p) { return ((p & ~7) | ((p ^ (p >> 3)) & 1) | (p & 6)) * 16; }
 
 template <int G, int KB>
-__global__ void __launch_bounds__(kScanThreads + 32) scan_planes_kernel(
-    const __grid_constant__ CUtensorMap tmap, Shape s, const uint16_t *__restrict__ qcodes,
+__global__ void __launch_bounds__(32 * kPlaneWarps) scan_planes_warp_kernel(
+    Shape s, const uint32_t *__restrict__ codes, const uint16_t *__restrict__ qcodes,
     const int32_t *__restrict__ seq_lens, int max_len, int nchunk, ScanOut o)
 {
-    using St = PlaneStage<KB>;
+    constexpr int D = kPlaneRing;
+    constexpr int SLOT = plane_slot_bytes<KB>();
+    constexpr int PIECES = SLOT / 16;  // 64 (K = 8) or 80 (K = 10)
     constexpr int QW = (KB + 3) & ~3;  // query masks per (table, head), padded to whole uint4s
-    constexpr int S = St::kStages, NC = kScanConsumers;
-    static_assert(NC * 32 == kScanThreads && 32 * 32 == kChunkPlanes, "8 consumer warps, a word per lane");
-    extern __shared__ __align__(1024) uint8_t dyn_raw[];
-    uint32_t *ring = reinterpret_cast<uint32_t *>(dyn_raw);  // [S][box][8 tables][kBoxWords]
-    uint32_t *qm = ring + S * St::kBytes / 4;                // [L][G][QW]
-    uint32_t *part = qm + s.L * G * QW;                      // [2 parities][G][2][kScanThreads]
-    __shared__ __align__(8) uint64_t full[S], empty[S];
-    __shared__ int range_sh[4];  // first item (b, kvh, chunk), item count
+    constexpr bool kPair = KB == 8;    // a word's planes are two 16-byte pieces
+    extern __shared__ __align__(16) uint32_t pw_smem[];  // ring [warps][D][SLOT], then qm [L][G][QW]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // The lengths and the codes come from work before the query hash: the
-    // work split and the producer's first code stages go ahead of grid_wait(),
-    // which the consumers pass before reading the query codes and the
-    // compactor before writing the candidate lists.
+    uint8_t *ring = reinterpret_cast<uint8_t *>(pw_smem) + warp * D * SLOT;
+    uint32_t *qm = pw_smem + kPlaneWarps * D * SLOT / 4;
+    const int unit = blockIdx.y, chunk = blockIdx.x * kPlaneWarps + warp;
+    const int b = unit / s.Hkv, kvh = unit % s.Hkv;
     grid_launch_dependents();
-
-    if (threadIdx.x == 0) {
-        // this block's contiguous share of the live items
-        long long total = 0;
-        for (int b = 0; b < s.B; b++) {
-            const int n = clamp_len(seq_lens, b, max_len, o.status, false);
-            total += (long long)s.Hkv * ((n + kChunkPlanes - 1) / kChunkPlanes);
+    // lengths and codes come from work before the query hash: read them first
+    const int N = clamp_len(seq_lens, b, max_len, o.status, false);
+    const bool reporter = blockIdx.x == 0 && kvh == 0 && threadIdx.x == 0;  // of a bad length of sequence b
+    if (blockIdx.x * kPlaneWarps * kChunkPlanes >= N) {  // the whole block is past the sequence
+        if (reporter) {
+            grid_wait();  // the status word is cleared by the query hash
+            clamp_len(seq_lens, b, max_len, o.status, true);
         }
-        long long x = total * blockIdx.x / gridDim.x;
-        const long long x1 = total * (blockIdx.x + 1) / gridDim.x;
-        range_sh[3] = (int)(x1 - x);
-        range_sh[0] = range_sh[1] = range_sh[2] = 0;
-        for (int b = 0; b < s.B && x1 > x; b++) {
-            const int n = min(max(seq_lens[b], 0), max_len);
-            const long long nch = (n + kChunkPlanes - 1) / kChunkPlanes, items = nch * s.Hkv;
-            if (x < items) {
-                range_sh[0] = b;
-                range_sh[1] = (int)(x / nch);
-                range_sh[2] = (int)(x % nch);
-                break;
+        return;
+    }
+    const int c0 = chunk * kChunkPlanes;
+    const bool live = c0 < N;  // warp-uniform
+    // words of this chunk that hold live tokens (the rest are zero-filled)
+    const int words = s.Ncap >> 5;
+    const int vw = live ? min(32, (N + 31) / 32 - chunk * 32) : 0;
+    const int vbytes = vw * KB * 4;
+    const uint8_t *src = reinterpret_cast<const uint8_t *>(codes) +
+                         (((size_t)unit * s.L * words + (size_t)chunk * 32) * KB) * 4;
+    const size_t tstride = (size_t)words * KB * 4;  // bytes between tables
+    auto copy_table = [&](int slot, const uint8_t *g) {
+        uint8_t *dst = ring + slot * SLOT;
+#pragma unroll
+        for (int i = 0; i < (PIECES + 31) / 32; i++) {
+            const int p = lane + 32 * i;  // piece = 16 bytes of the slab
+            if (p < PIECES) {
+                const int nb = min(max(vbytes - p * 16, 0), 16);  // zero-fill past the live words
+                cp_async_16(dst + (kPair ? plane_piece_k8(p) : p * 16), g + (nb ? p * 16 : 0), nb);
             }
-            x -= items;
         }
-        for (int i = 0; i < S; i++) {
-            mbar_init(smem_u32(&full[i]), 1);
-            mbar_init(smem_u32(&empty[i]), NC);
+    };
+    if (live) {
+        for (int l = 0; l < D - 1; l++) {
+            if (l < s.L) copy_table(l, src + l * tstride);
+            cp_async_commit();  // one group per table, empty past L, so the group count stays uniform
         }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    grid_wait();  // the query codes are the query hash's output
+    if (reporter) clamp_len(seq_lens, b, max_len, o.status, true);
+    for (int i = threadIdx.x; i < s.L * G; i += blockDim.x) {
+        const int l = i / G, g = i % G;
+        const unsigned code = qcodes[((size_t)b * s.Hq + kvh * G + g) * s.L + l];
+        uint4 *dst = reinterpret_cast<uint4 *>(qm + (size_t)i * QW);
+#pragma unroll
+        for (int q = 0; q < QW / 4; q++) {
+            uint32_t m[4];
+#pragma unroll
+            for (int x = 0; x < 4; x++) m[x] = 4 * q + x < KB ? 0u - ((code >> (4 * q + x)) & 1u) : 0u;
+            dst[q] = make_uint4(m[0], m[1], m[2], m[3]);
+        }
     }
     __syncthreads();
-    const int count = range_sh[3];
-    if (count <= 0) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) {
-            grid_wait();  // the status word is cleared by the query hash
-            for (int b = 0; b < s.B; b++) clamp_len(seq_lens, b, max_len, o.status, true);
-        }
-        return;
-    }
-    LiveCursor cur;
-    cur.b = range_sh[0];
-    cur.kvh = range_sh[1];
-    cur.chunk = range_sh[2];
-    cur.load_seq(seq_lens, max_len);
-    const int nst = (s.L + NC - 1) / NC;  // stages per item
+    if (!live) return;
 
-    if (warp == NC) {
-        // ------------------------------------------- producer + compactor ----
-        // Issue item it's stages, then fold and compact item it - 1 (whose
-        // stages were all issued earlier, so the consumers can finish it).
-        int e = 0;
-        bool ok = true;
-        LiveCursor pc = cur;
-        for (int it = 0; it <= count; it++) {
-            if (it < count) {
-                if (lane == 0 && ok) {
-                    const int x0 = pc.chunk * 32 * KB, z = pc.unit(s);
-                    for (int j = 0; j < nst; j++, e++) {
-                        const int st = e % S;
-                        if (e >= S && !mbar_wait_bounded(smem_u32(&empty[st]), (uint32_t)(e / S - 1) & 1u)) {
-                            set_status(o.status, MP_ERR_CUDA);
-                            ok = false;
-                            break;
-                        }
-                        mbar_expect_tx(smem_u32(&full[st]), St::kBytes);
+    uint32_t s1[G], s2[G];
 #pragma unroll
-                        for (int bx = 0; bx < St::kBoxes; bx++)
-                            tma_load_3d(smem_u32(ring) + (uint32_t)(st * St::kBytes + bx * NC * St::kBoxWords * 4),
-                                        &tmap, smem_u32(&full[st]), x0 + bx * St::kBoxWords, NC * j, z);
-                    }
-                }
-                __syncwarp();
-                pc.next(s, seq_lens, max_len);
+    for (int g = 0; g < G; g++) s1[g] = s2[g] = 0u;
+    int rs = 0;  // slot of table l
+    for (int l = 0; l < s.L; l++) {
+        cp_async_wait<D - 2>();  // table l has landed (groups 0 .. l complete)
+        __syncwarp();            // ... for every lane's pieces; and every lane is done with table l - 1
+        uint32_t pw[KB];
+        const uint8_t *rp = ring + rs * SLOT;
+        if constexpr (kPair) {
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(rp + plane_piece_k8(2 * lane + i));
+                pw[4 * i] = v.x;
+                pw[4 * i + 1] = v.y;
+                pw[4 * i + 2] = v.z;
+                pw[4 * i + 3] = v.w;
             }
-            if (it >= 1) {
-                const int ci = it - 1;
-                if (ci == 0) {
-                    grid_wait();
-                    if (blockIdx.x == 0 && lane == 0)
-                        for (int b = 0; b < s.B; b++) clamp_len(seq_lens, b, max_len, o.status, true);
-                }
-                bar_sync_all(2);  // the consumers' partials of item ci are in buffer ci & 1
-                const uint32_t *pp = part + (ci & 1) * (G * 2 * kScanThreads);
-                uint32_t s1[G], s2[G];
+        } else {
 #pragma unroll
-                for (int g = 0; g < G; g++) s1[g] = s2[g] = 0u;
-#pragma unroll 1
-                for (int t = 0; t < NC; t++) {
-#pragma unroll
-                    for (int g = 0; g < G; g++) {
-                        const uint32_t a1 = pp[(g * 2 + 0) * kScanThreads + t * 32 + lane];
-                        const uint32_t a2 = pp[(g * 2 + 1) * kScanThreads + t * 32 + lane];
-                        s2[g] |= a2 | (s1[g] & a1);
-                        s1[g] |= a1;
-                    }
-                }
-                if (ci + 1 < count) bar_arrive_all(3);  // item ci is read: the consumers may post item ci + 1
-                // tokens eligible for S: [sink, N - window) and below N
-                compact_warp<G, 32, kChunkPlanes>(s, cur.unit(s), cur.chunk, nchunk, cur.chunk * kChunkPlanes + lane * 32, cur.N,
-                                s.sink, min(cur.N - s.window, cur.N), s2, o, lane);
-                cur.next(s, seq_lens, max_len);
+            for (int i = 0; i < KB / 2; i++) {
+                const uint2 v = *reinterpret_cast<const uint2 *>(rp + lane * KB * 4 + i * 8);
+                pw[2 * i] = v.x;
+                pw[2 * i + 1] = v.y;
             }
         }
-        // every copy issued lands before the block exits (the last use of each stage)
-        if (lane == 0)
-            for (int st = 0; st < S && st < e; st++) {
-                const int last = st + ((e - 1 - st) / S) * S;
-                mbar_wait_bounded(smem_u32(&full[st]), (uint32_t)(last / S) & 1u);
-            }
-        return;
-    }
-
-    // ------------------------------------------------------- consumers ----
-    const int ts = warp;
-    const int box = (lane * KB) / St::kBoxWords, in_box = lane * KB - box * St::kBoxWords;
-    const int lane_off = box * NC * St::kBoxWords + ts * St::kBoxWords + in_box;  // words into a stage
-    int e = 0, qm_unit = -1;
-    bool dead = false;  // a copy never landed: stop waiting, keep the barriers in step
-    grid_wait();        // the query codes are the query hash's output
-    for (int it = 0; it < count; it++, cur.next(s, seq_lens, max_len)) {
-        const int unit = cur.unit(s);
-        if (unit != qm_unit) {  // uniform over the consumers
-            if (qm_unit >= 0) consumer_barrier();  // every consumer is done with the old masks
-            for (int i = threadIdx.x; i < s.L * G; i += kScanThreads) {
-                const int l = i / G, g = i % G;
-                const unsigned code = qcodes[((size_t)cur.b * s.Hq + cur.kvh * G + g) * s.L + l];
-                uint4 *dst = reinterpret_cast<uint4 *>(qm + (size_t)i * QW);
-#pragma unroll
-                for (int q = 0; q < QW / 4; q++) {
-                    uint32_t m[4];
-#pragma unroll
-                    for (int x = 0; x < 4; x++) m[x] = 4 * q + x < KB ? 0u - ((code >> (4 * q + x)) & 1u) : 0u;
-                    dst[q] = make_uint4(m[0], m[1], m[2], m[3]);
-                }
-            }
-            consumer_barrier();
-            qm_unit = unit;
-        }
-        uint32_t s1[G], s2[G];
-#pragma unroll
-        for (int g = 0; g < G; g++) s1[g] = s2[g] = 0u;
-        for (int j = 0; j < nst; j++, e++) {
-            const int st = e % S;
-            if (!dead) {
-                // every lane waits (bounded); the warp goes on only if all saw the stage land
-                const bool landed = mbar_wait_bounded(smem_u32(&full[st]), (uint32_t)(e / S) & 1u);
-                if (!__all_sync(0xffffffffu, landed)) {
-                    if (lane == 0) set_status(o.status, MP_ERR_CUDA);
-                    dead = true;
-                }
-            }
-            const int l = ts + NC * j;
-            const bool live = !dead && l < s.L;
-            uint32_t pw[KB];
-            if (live) {
-                const uint32_t *src = ring + st * (St::kBytes / 4) + lane_off;
-                if constexpr (KB % 4 == 0) {
-#pragma unroll
-                    for (int q = 0; q < KB / 4; q++) {
-                        const uint4 v = reinterpret_cast<const uint4 *>(src)[q];
-                        pw[4 * q] = v.x;
-                        pw[4 * q + 1] = v.y;
-                        pw[4 * q + 2] = v.z;
-                        pw[4 * q + 3] = v.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < KB / 2; q++) {
-                        const uint2 v = reinterpret_cast<const uint2 *>(src)[q];
-                        pw[2 * q] = v.x;
-                        pw[2 * q + 1] = v.y;
-                    }
-                }
-#pragma unroll
-                for (int g = 0; g < G; g++) {
-                    const uint4 *m4 = reinterpret_cast<const uint4 *>(qm + (l * G + g) * QW);
-                    uint32_t mis = 0u;
-#pragma unroll
-                    for (int q = 0; q < QW / 4; q++) {
-                        const uint4 mq = m4[q];
-                        const uint32_t mm[4] = {mq.x, mq.y, mq.z, mq.w};
-#pragma unroll
-                        for (int x = 0; x < 4; x++)
-                            if (4 * q + x < KB) mis |= pw[4 * q + x] ^ mm[x];
-                    }
-                    s2[g] |= s1[g] & ~mis;
-                    s1[g] |= ~mis;
-                }
-            }
-            // Release the stage only once every lane has used (so received) its
-            // words; the proxy fence orders those reads before the TMA refill.
-            __syncwarp();
-            if (lane == 0 && !dead) {
-                fence_proxy_async_smem();
-                mbar_arrive(smem_u32(&empty[st]));
-            }
-        }
-        // this item's split partials -> buffer it & 1, once the producer has read
-        // item it - 1 (so each barrier generation sees exactly one item)
-        if (it >= 1) bar_sync_all(3);
-        uint32_t *pp = part + (it & 1) * (G * 2 * kScanThreads);
+        // refill the slot of table l - 1 (every lane has used it) with table l + D - 1
+        const int ws_ = rs == 0 ? D - 1 : rs - 1;
+        if (l + D - 1 < s.L) copy_table(ws_, src + (size_t)(l + D - 1) * tstride);
+        cp_async_commit();
+        rs = rs + 1 == D ? 0 : rs + 1;
 #pragma unroll
         for (int g = 0; g < G; g++) {
-            pp[(g * 2 + 0) * kScanThreads + threadIdx.x] = s1[g];
-            pp[(g * 2 + 1) * kScanThreads + threadIdx.x] = s2[g];
+            const uint4 *m4 = reinterpret_cast<const uint4 *>(qm + (l * G + g) * QW);
+            uint32_t mis = 0u;
+#pragma unroll
+            for (int q = 0; q < QW / 4; q++) {
+                const uint4 mq = m4[q];
+                const uint32_t mm[4] = {mq.x, mq.y, mq.z, mq.w};
+#pragma unroll
+                for (int x = 0; x < 4; x++)
+                    if (4 * q + x < KB) mis |= pw[4 * q + x] ^ mm[x];
+            }
+            s2[g] |= s1[g] & ~mis;
+            s1[g] |= ~mis;
         }
-        bar_arrive_all(2);
     }
+    cp_async_wait<0>();
+    // Tokens eligible for S: [sink, N - window) and below N.
+    compact_warp<G, 32, kChunkPlanes>(s, unit, chunk, nchunk, c0 + lane * 32, N, s.sink, min(N - s.window, N), s2, o,
+                                      lane);
 }
 
 // ---------------------------------------------------------------- attend ----
@@ -724,14 +638,21 @@ constexpr int kMaxSpan = 64;                // scan chunks per attention block, 
 constexpr int kAttRows = 64;                // rows per tile (4 warps x 16)
 constexpr int kAttStages = 2;               // cp.async ring depth (3 blocks fit per SM)
 constexpr int kRowBytes = kHeadDim * 2;     // 256
-constexpr int kRowStride = kRowBytes + 16;  // padded: conflict-free ldmatrix / 8-byte reads
+// K / V rows in shared memory are unpadded; within each 128-byte line the
+// 16-byte pieces are XOR-swizzled by row & 7 (att_piece), so that a global
+// line lands in one shared line (a copy whose pieces straddle shared lines is
+// fetched from L2 twice) and the 8 rows an ldmatrix reads hit distinct banks.
+constexpr int kRowStride = kRowBytes;
 constexpr int kStageBytes = kAttRows * kRowStride * 2;  // K rows then V rows
-// int8 keys (mp_decode_attend_q8): 128-byte rows, padded to 144 (conflict-free ldmatrix)
-constexpr int kRowStrideQ8 = kHeadDim + 16;
+// int8 keys (mp_decode_attend_q8): 128-byte rows
+constexpr int kRowStrideQ8 = kHeadDim;
 template <bool Q8>
 constexpr int att_k_stride() { return Q8 ? kRowStrideQ8 : kRowStride; }
 template <bool Q8>
 constexpr int att_stage_bytes() { return kAttRows * (att_k_stride<Q8>() + kRowStride); }
+
+// Byte offset of 16-byte piece c of row `row` within the row.
+__device__ __forceinline__ int att_piece(int row, int c) { return (c ^ (row & 7)) << 4; }
 
 struct AttendArgs {
     Shape s;
@@ -929,10 +850,11 @@ __device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, co
     {
         if constexpr (Q8) {
             const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStrideQ8;
+            const int r7 = lane & 7;  // the row's swizzle
 #pragma unroll
             for (int kst = 0; kst < 8; kst++) {
                 uint32_t r0, r1, a0, a1, a2, a3;
-                ldmatrix_x2(r0, r1, arow + kst * 16);
+                ldmatrix_x2(r0, r1, arow + ((kst ^ r7) << 4));
                 s8x4_to_f16x2(r0, a0, a2);
                 s8x4_to_f16x2(r1, a1, a3);
                 mma_f16_16816(c[0], c[1], c[2], c[3], a0, a1, a2, a3, w.qb[kst][0], w.qb[kst][1]);
@@ -946,11 +868,13 @@ __device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, co
             nb = m1.y;
         } else {
             float g0[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f};
-            const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStride + (lane >> 4) * 16;
+            // piece 2 kst + (lane >> 4) of row lane & 15, swizzled by lane & 7
+            const uint8_t *arow = ks_ + (warp * 16 + (lane & 15)) * kRowStride;
+            const int sw = (lane >> 4) ^ (lane & 7);
 #pragma unroll
             for (int kst = 0; kst < 8; kst++) {
                 uint32_t a0, a1, a2, a3;
-                ldmatrix_x4(a0, a1, a2, a3, arow + kst * 32);
+                ldmatrix_x4(a0, a1, a2, a3, arow + (((2 * kst) ^ sw) << 4));
                 mma_bf16_16816(c[0], c[1], c[2], c[3], a0, a1, a2, a3, w.qb[kst][0], w.qb[kst][1]);
                 mma_bf16_16816(g0[0], g0[1], g0[2], g0[3], a0, a1, a2, a3, a0, a2);  // columns: rows 0-7
                 mma_bf16_16816(g1[0], g1[1], g1[2], g1[3], a0, a1, a2, a3, a1, a3);  // columns: rows 8-15
@@ -1035,13 +959,14 @@ __device__ __forceinline__ void attn_tile(AttnWarp<G> &w, const uint8_t *ks_, co
     const uint32_t bh0 = movmatrix_trans(hi_g), bh1 = movmatrix_trans(hi_g8);
     const uint32_t bl0 = movmatrix_trans(lo_g), bl1 = movmatrix_trans(lo_g8);
     {
+        // piece 2 mt + (mrow & 1) of row 8 (mrow >> 1) + (lane & 7), swizzled by lane & 7
         const int mrow = lane >> 3;
-        const uint8_t *vrow =
-            vs_ + (warp * 16 + (mrow >> 1) * 8 + (lane & 7)) * kRowStride + (mrow & 1) * 16;
+        const uint8_t *vrow = vs_ + (warp * 16 + (mrow >> 1) * 8 + (lane & 7)) * kRowStride;
+        const int sw = (mrow & 1) ^ (lane & 7);
 #pragma unroll
         for (int mt = 0; mt < 8; mt++) {
             uint32_t a0, a1, a2, a3;
-            ldmatrix_x4_trans(a0, a1, a2, a3, vrow + mt * 32);
+            ldmatrix_x4_trans(a0, a1, a2, a3, vrow + (((2 * mt) ^ sw) << 4));
             mma_bf16_16816(w.acc[mt][0], w.acc[mt][1], w.acc[mt][2], w.acc[mt][3], a0, a1, a2, a3, bh0, bh1);
             mma_bf16_16816(w.acc[mt][0], w.acc[mt][1], w.acc[mt][2], w.acc[mt][3], a0, a1, a2, a3, bl0, bl1);
         }
@@ -1235,15 +1160,15 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
             const size_t off = (size_t)tok * kHeadDim + col * 8;
             if constexpr (Q8) {  // 8 pieces of the int8 row, then its 16-byte record
                 if (col < 9) {
-                    void *dst = col < 8 ? (void *)(ks_ + r * KS + col * 16) : (void *)&kq[warp][stage][r];
+                    void *dst = col < 8 ? (void *)(ks_ + r * KS + att_piece(r, col)) : (void *)&kq[warp][stage][r];
                     const void *src = col < 8 ? (const void *)(k8base + (size_t)tok * kHeadDim + col * 16)
                                               : (const void *)(kmbase + (size_t)tok * kQ8MetaFloats);
                     cp_async_16(dst, src, ok ? 16 : 0);
                 }
             } else {
-                cp_async_16(ks_ + r * KS + col * 16, kbase + off, ok ? 16 : 0);
+                cp_async_16(ks_ + r * KS + att_piece(r, col), kbase + off, ok ? 16 : 0);
             }
-            cp_async_16(vs_ + r * kRowStride + col * 16, vbase + off, ok ? 16 : 0);
+            cp_async_16(vs_ + r * kRowStride + att_piece(r, col), vbase + off, ok ? 16 : 0);
             if (col == 0) meta[warp][stage][r] = ok ? (dsplit ? dmeta : (ent >> 24)) : 0u;
         }
     };
@@ -1288,7 +1213,7 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
 // ------------------------------------------------ fused scan + attend ----
 // Bit-plane codes only.  One persistent block of 14 warps per SM walks a
 // contiguous share of the live (sequence, kv head, 1024-token chunk) items,
-// like scan_planes_kernel, and attends each item's candidates itself, so the
+// like the bit-plane scan, and attends each item's candidates itself, so the
 // candidate lists never leave shared memory and the code stream and the K/V
 // row gathers of different items overlap on the same SM:
 //   warp 0      TMA producer of the code stages (8 tables per 3-D copy);
@@ -1363,7 +1288,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_planes_kernel(const __
     grid_dependency_wait();
 
     if (threadIdx.x == 0) {
-        // this block's contiguous share of the live items (as scan_planes_kernel)
+        // this block's contiguous share of the live items
         long long total = 0;
         for (int b = 0; b < s.B; b++) {
             const int n = clamp_len(a.seq_lens, b, a.max_len, a.status, blockIdx.x == 0);
@@ -1667,8 +1592,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_planes_kernel(const __
                 const bool ok = ent != 0xFFFFFFFFu;
                 const int tok = ok ? (int)(ent & 0xFFFFFFu) : 0;
                 const size_t off = (size_t)tok * kHeadDim + col * 8;
-                cp_async_16(ks_ + r * kRowStride + col * 16, kbase + off, ok ? 16 : 0);
-                cp_async_16(vs_ + r * kRowStride + col * 16, vbase + off, ok ? 16 : 0);
+                cp_async_16(ks_ + r * kRowStride + att_piece(r, col), kbase + off, ok ? 16 : 0);
+                cp_async_16(vs_ + r * kRowStride + att_piece(r, col), vbase + off, ok ? 16 : 0);
                 if (col == 0) meta[grp][stage][r] = ok ? ((ent >> 24) ? (ent >> 24) : dmeta) : 0u;
             }
         };
@@ -1928,37 +1853,17 @@ static LogU make_logu(const Shape &s)
 // Persistent plane scan: as many blocks as fit on the device at once (at
 // most one per possible item); each walks its share of the live items.
 template <int G, int KB>
-static cudaError_t launch_scan_planes(const Shape &s, const uint32_t *codes, const Workspace &ws,
-                                      const int32_t *seq_lens, int max_len, int nchunk, const ScanOut &so,
-                                      cudaStream_t st)
+static cudaError_t launch_scan_planes_warp(const Shape &s, const uint32_t *codes, const Workspace &ws,
+                                           const int32_t *seq_lens, int max_len, int nchunk, const ScanOut &so,
+                                           cudaStream_t st)
 {
-    using Stg = PlaneStage<KB>;
-    const size_t sm = (size_t)Stg::kStages * Stg::kBytes + (size_t)s.L * G * ((KB + 3) & ~3) * sizeof(uint32_t) +
-                      (size_t)2 * G * 2 * kScanThreads * sizeof(uint32_t);
-    const void *fn = reinterpret_cast<const void *>(scan_planes_kernel<G, KB>);
+    const size_t sm = (size_t)kPlaneWarps * kPlaneRing * plane_slot_bytes<KB>() +
+                      (size_t)s.L * G * ((KB + 3) & ~3) * sizeof(uint32_t);
+    const void *fn = reinterpret_cast<const void *>(scan_planes_warp_kernel<G, KB>);
     cudaError_t e = ensure_smem(fn, (int)sm);
     if (e != cudaSuccess) return e;
-    // codes as a 3-D uint32 tensor: (word x plane) within a table, table, unit
-    const int words = s.Ncap >> 5;
-    const uint64_t dims[3] = {(uint64_t)words * KB, (uint64_t)s.L, (uint64_t)s.B * s.Hkv};
-    const uint64_t strides[2] = {(uint64_t)words * KB * 4, (uint64_t)s.L * words * KB * 4};
-    const uint32_t box[3] = {(uint32_t)Stg::kBoxWords, (uint32_t)kScanConsumers, 1};
-    CUtensorMap tmap;
-    if (!encode_tensor_map(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, codes, dims, strides, box,
-                           CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    }
-    int per_sm = 1;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kScanThreads + 32, sm)) != cudaSuccess)
-        return e;
-    const long long items = (long long)nchunk * s.B * s.Hkv;
-    const int grid = (int)std::max(1LL, std::min(items, (long long)std::max(per_sm, 1) * sms));
-    return launch_pdl(scan_planes_kernel<G, KB>, dim3(grid), dim3(kScanThreads + 32), sm, st, tmap, s,
+    dim3 grid((nchunk + kPlaneWarps - 1) / kPlaneWarps, s.B * s.Hkv);
+    return launch_pdl(scan_planes_warp_kernel<G, KB>, grid, dim3(32 * kPlaneWarps), sm, st, s, codes,
                       (const uint16_t *)ws.qcodes, seq_lens, max_len, nchunk, so);
 }
 
@@ -2055,11 +1960,11 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
                            static_cast<const uint8_t *>(codes), (const uint16_t *)ws.qcodes, seq_lens, max_len,
                            nchunk, so);
         } else if (s.K == 8) {
-            e = launch_scan_planes<G, 8>(s, static_cast<const uint32_t *>(codes), ws, seq_lens, max_len, nchunk,
-                                         so, st);
+            e = launch_scan_planes_warp<G, 8>(s, static_cast<const uint32_t *>(codes), ws, seq_lens, max_len,
+                                              nchunk, so, st);
         } else {
-            e = launch_scan_planes<G, 10>(s, static_cast<const uint32_t *>(codes), ws, seq_lens, max_len, nchunk,
-                                          so, st);
+            e = launch_scan_planes_warp<G, 10>(s, static_cast<const uint32_t *>(codes), ws, seq_lens, max_len,
+                                               nchunk, so, st);
         }
         if (e != cudaSuccess) return e;
     }

@@ -176,3 +176,12 @@ def test_int8_key_entry_points_checked(lib):
         dbg = B._CDebug(None, None, None, path)
         assert d(ctypes.byref(s), A, A, A, A, A, A, A, 1024, A, A, A, A, need.value, ctypes.byref(dbg),
                  None) == want, path
+
+
+def test_auto_layout_threshold_matches_header():
+    """The binding's copy of the MP_CODES_AUTO rule uses the header's threshold."""
+    m = re.search(r"#define MP_CODES_AUTO_PLANES_MIN \(1 << (\d+)\)", open(HEADER).read())
+    assert m and mp.MP_CODES_AUTO_PLANES_MIN == 1 << int(m.group(1))
+    assert not mp.auto_planes(1, 8, 16512, 8)        # a 16k-token layer: byte codes
+    assert mp.auto_planes(4, 8, 131200, 8)           # four 128k-token sequences: bit planes
+    assert mp.auto_planes(1, 1, 128, 10)             # K = 10: always bit planes

@@ -65,7 +65,7 @@ def test_both_arms_report_the_same_config():
     import workloads
     w = workloads.get(bench.DEFAULT_WORKLOAD)
     cfg = bench.config_of(w)
-    assert cfg["workload"] == "ragged16" and cfg["code_layout"] == "bytes"
+    assert cfg["workload"] == "ragged16" and cfg["code_layout"] == "planes"
     assert not {"launch", "decode_path", "mode"} & set(cfg)
     assert cfg == bench.config_of(workloads.get("ragged16"))
 

@@ -390,7 +390,7 @@ def test_overlong_length_is_clamped_and_reported():
 
 # ------------------------------------------------ full-size configurations ----
 
-FULL = ["llama8b_16k", "batch8_64k", "batch4_128k", "ragged16", "ragged16_planes"]
+FULL = ["llama8b_16k", "batch8_64k", "batch4_128k", "ragged16", "ragged16_bytes"]
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -428,7 +428,11 @@ def _full_size(name, path):
         query codes), bit-exact;
       - out / lse of 8 units spread over the length range (shortest and
         longest included) against the fp64 estimator on the same codes."""
-    w = WORKLOADS[name] if name in WORKLOADS else WORKLOADS[name.rsplit("_", 1)[0]].with_(code_layout="planes")
+    if name in WORKLOADS:
+        w = WORKLOADS[name]
+    else:  # <workload>_<layout>
+        base, layout = name.rsplit("_", 1)
+        w = WORKLOADS[base].with_(code_layout=layout)
     inp = make_inputs(w)
     run = Run(w, inp)
     run.alloc_decode(run.max_len + 1)
