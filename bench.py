@@ -257,14 +257,23 @@ class Bench:
         # (and with int8 keys the quantisation, 1) if in the step
         self.launches_per_step = 1 + (3 if fused else 4) + ((2 if self.q8 else 1) if self.with_hash else 0)
         # prefill: the codes of the cached keys (the step's append adds the new token's)
-        self.hash()
+        self.build()
         torch.cuda.synchronize()
 
     def hash(self):
+        """The key-hash build of the cached keys."""
         self.mp.hash_keys(self.shape, self.K, self.W, self.prefill, self.codes, seq_lens=self.lens0)
+
+    def quantize(self):
+        """The int8 copy of the cached keys (with --k-format int8)."""
         if self.q8:
             self.mp.quantize_keys(self.shape, self.K, self.k8, self.kmeta, n_tokens=self.prefill,
                                   seq_lens=self.lens0)
+
+    def build(self):
+        """Everything a prefill leaves in the cache: codes (and the int8 copy)."""
+        self.hash()
+        self.quantize()
 
     def append(self):
         if self.q8:
@@ -285,7 +294,7 @@ class Bench:
     def calls(self):
         """The library calls of one step (the lengths are reset before it)."""
         if self.with_hash:
-            self.hash()
+            self.build()
         self.append()
         self.decode()
 
@@ -442,7 +451,7 @@ class Bench:
                 side.wait_stream(main)
                 with torch.cuda.stream(side):
                     self.in_dev.copy_(hin, non_blocking=True)
-                self.hash()
+                self.build()
                 main.wait_stream(side)
             else:
                 self.in_dev.copy_(hin, non_blocking=True)
