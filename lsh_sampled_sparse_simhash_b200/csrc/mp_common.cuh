@@ -141,6 +141,34 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t a, uint32_t parity)
     return mbar_try_wait(a, parity) || mbar_wait_bounded_slow(a, parity);
 }
 
+// Per-chunk ready flags between the collision scan and the attention (see
+// attend_kernel): a release store after the chunk's list is written, an
+// acquire load before it is read.
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(int32_t *p, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Bounded wait for a nonzero flag: false once kWaitLimitNs has passed.
+static __device__ __noinline__ bool flag_wait_bounded_slow(const int32_t *p)
+{
+    const uint64_t t0 = globaltimer();
+    while (ld_acquire_gpu(p) == 0) {
+        if (globaltimer() - t0 > kWaitLimitNs) return false;
+        __nanosleep(128);
+    }
+    return true;
+}
+__device__ __forceinline__ bool flag_wait_bounded(const int32_t *p)
+{
+    return ld_acquire_gpu(p) != 0 || flag_wait_bounded_slow(p);
+}
+
 // Orders this thread's earlier generic-proxy shared-memory accesses before its
 // later async-proxy ones (a buffer that was read is about to be refilled).
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }

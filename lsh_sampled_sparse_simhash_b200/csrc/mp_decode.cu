@@ -46,7 +46,8 @@ template <int G>
 __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__restrict__ q,
                                                     const uint16_t *__restrict__ W,
                                                     const uint16_t *__restrict__ qcodes_in,
-                                                    uint16_t *__restrict__ qcodes, int32_t *status, int ug)
+                                                    uint16_t *__restrict__ qcodes, int32_t *status, int ug,
+                                                    int32_t *ready, int nready)
 {
     __shared__ float qs[kQhashVecs][kHeadDim + 4];  // element d at d + d / 32: the 4 quarters hit distinct banks
     __shared__ uint8_t bits[kQhashVecs][kQhashCols];
@@ -61,12 +62,21 @@ __global__ void __launch_bounds__(256) qhash_kernel(Shape s, const uint16_t *__r
     // the query codes of an earlier call has completed before this one starts
     // (see grid_launch_dependents), so the codes are computed and written
     // before the wait for the predecessor; only the status word waits.
+    // After the wait: clear the call's status word, the tcgen05 attention's
+    // work counter and the scan's per-chunk ready flags (word 15 of each
+    // chunk's count record, i < nready), and make the clears visible before
+    // the scan may launch: the attention, which starts once every scan block
+    // has started, reads the flags without waiting for the scan to finish.
     auto finish = [&]() {
-        grid_dependency_wait();
+        grid_wait();
         if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) {
             status[0] = 0;  // the call's status word
             status[1] = 0;  // the attention kernel's work counter
         }
+        const int nb = gridDim.x * gridDim.y, bid = blockIdx.y * gridDim.x + blockIdx.x;
+        for (int i = bid * blockDim.x + tid; i < nready; i += nb * blockDim.x) ready[(size_t)i * 16 + 15] = 0;
+        __threadfence();
+        grid_launch_dependents();
     };
     if (qcodes_in) {
         for (int i = tid; i < nu * G * TB; i += blockDim.x) {
@@ -251,6 +261,16 @@ __device__ __forceinline__ void compact_warp(const Shape &s, int unit, int chunk
     }
 }
 
+// After a warp has written its chunk's candidate list and counts: every
+// lane's writes are made visible, then the chunk's ready flag (word 15 of its
+// count record, cleared by the query hash) is released to the attention.
+__device__ __forceinline__ void mark_chunk_ready(const ScanOut &o, int unit, int chunk, int nchunk, int lane)
+{
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) st_release_gpu(o.cnt + ((size_t)unit * nchunk + chunk) * 16 + 15, 1);
+}
+
 // -------------------------------------------------- scan, byte codes (K = 8) ----
 // Byte codes [unit][L][Ncap].  A warp owns a 512-token chunk of one unit for
 // all L tables (lane = 16 consecutive tokens, one 16-byte streaming load per
@@ -416,6 +436,7 @@ __global__ void __launch_bounds__(32 * kByteWarps, G >= 8 ? 2 : MP_SCAN_BLOCKS_P
     }
     // Tokens eligible for S: [sink, N - window) and below N.
     compact_warp<G, 16, kChunkBytes>(s, unit, chunk, nchunk, t0, N, s.sink, min(N - s.window, N), hm, o, lane);
+    mark_chunk_ready(o, unit, chunk, nchunk, lane);
 }
 
 // ---------------------------------------- bit planes: shared TMA pieces ----
@@ -630,6 +651,7 @@ __global__ void __launch_bounds__(32 * kPlaneWarps) scan_planes_warp_kernel(
     // Tokens eligible for S: [sink, N - window) and below N.
     compact_warp<G, 32, kChunkPlanes>(s, unit, chunk, nchunk, c0 + lane * 32, N, s.sink, min(N - s.window, N), s2, o,
                                       lane);
+    mark_chunk_ready(o, unit, chunk, nchunk, lane);
 }
 
 // ---------------------------------------------------------------- attend ----
@@ -673,6 +695,7 @@ struct AttendArgs {
     float scale;  // 1/sqrt(d)
     const int8_t *k8;      // int8 keys [B][Hkv][Ncap][128] (attend_kernel<G, true>), else null
     const float *kmeta;    // their per-row records {scale, squared norm, 0, 0} [B][Hkv][Ncap][4]
+    int32_t *status;       // the call's status word (a ready flag that never came: MP_ERR_CUDA)
 };
 
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
@@ -1054,15 +1077,35 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int unit = blockIdx.y, split = blockIdx.x;
     const int b = unit / s.Hkv, kvh = unit % s.Hkv;
-    grid_dependency_wait();
     const bool dsplit = split == a.ngroups * a.subs;
     const int grp = split / a.subs, sub = split % a.subs;
     const int c_begin = grp * a.span;
     const uint32_t *lists = a.cand + ((size_t)unit * a.nchunk + c_begin) * a.chunk_tokens;
+    // This kernel starts once every block of the scan has started, so all
+    // work before the scan (the append's rows and lengths) is complete and
+    // visible; the scan's own output is not waited for as a whole: a block
+    // waits only for the ready flags of the chunks it reads (the exact-set
+    // block reads none), and then lets the merge launch.  Blocks of early
+    // units thus run beside the scan's last blocks.
+    int N = a.seq_lens[b];
+    N = N < 0 ? 0 : (N > a.max_len ? a.max_len : N);
+    const int nch = (N + a.chunk_tokens - 1) / a.chunk_tokens;
+    if (!dsplit && c_begin >= nch) return;
+    if (!dsplit) {
+        if (tid == 0) {
+            const int c_end = min(c_begin + a.span, nch);
+            bool ok = true;
+            for (int c = c_begin; c < c_end && ok; c++)
+                ok = flag_wait_bounded(a.cnt + ((size_t)unit * a.nchunk + c) * 16 + 15);
+            if (!ok) set_status(a.status, MP_ERR_CUDA);
+        }
+        __syncthreads();
+    }
+    grid_launch_dependents();
     // A block that takes one chunk's whole list (span = subs = 1) reads the
-    // list's count and the first two tiles' entries together with the length:
-    // none of these loads waits for another (entries past the count are
-    // dropped below; they stay inside the chunk's list).
+    // list's count and the first two tiles' entries together: none of these
+    // loads waits for another (entries past the count are dropped below; they
+    // stay inside the chunk's list).
     const bool direct = !dsplit && a.span == 1 && a.subs == 1;
     int dcount = 0;
     uint32_t pre0 = 0xFFFFFFFFu, pre1 = 0xFFFFFFFFu;
@@ -1073,10 +1116,6 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
             pre1 = lists[kAttRows + warp * kWarpRows + lane];
         }
     }
-    int N = a.seq_lens[b];
-    N = N < 0 ? 0 : (N > a.max_len ? a.max_len : N);
-    const int nch = (N + a.chunk_tokens - 1) / a.chunk_tokens;
-    if (!dsplit && c_begin >= nch) return;
 
     // Rows of this block: its share of the concatenated candidate lists of
     // chunks [c_begin, c_end), or the exact set D.
@@ -1646,20 +1685,15 @@ __global__ void __launch_bounds__(32 * kMergeWarps) merge_kernel(Shape s, const 
     const int b = bh / s.Hq, h = bh % s.Hq, kvh = h / G, g = h % G;
     const int unit = b * s.Hkv + kvh;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // the lengths come from work before this kernel's predecessor, and so do
-    // the per-chunk counts when a separate scan kernel wrote them (has_d; the
-    // fused kernel, the predecessor otherwise, writes them itself): those
-    // reads go before the wait
+    // the lengths come from work before this kernel's predecessor: that read
+    // goes before the wait; the per-chunk counts (the scan's, made visible to
+    // the attention by the ready flags, or the fused kernel's) after it
     int N = seq_lens[b];
     N = N < 0 ? 0 : (N > max_len ? max_len : N);
     const int nch = (N + chunk_tokens - 1) / chunk_tokens;
-    int ns = 0;
-    auto count_sampled = [&]() {
-        for (int j = tid; j < nch; j += blockDim.x) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
-    };
-    if (has_d) count_sampled();
     grid_dependency_wait();
-    if (!has_d) count_sampled();
+    int ns = 0;
+    for (int j = tid; j < nch; j += blockDim.x) ns += cnt[((size_t)unit * nchunk + j) * 16 + 1 + g];
     const int nsp = ((nch + span - 1) / span) * subs;  // live chunk splits
     const int dsp = ngroups * subs;                     // the exact-set split (if has_d)
     const size_t base = (size_t)bh * (dsp + 1);
@@ -1916,7 +1950,8 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
         const int TB = qhash_tables_per_block(s.K), ug = qhash_units_per_block(s, G);
         dim3 grid((s.L + TB - 1) / TB, (units + ug - 1) / ug);
         e = launch_pdl(qhash_kernel<G>, grid, dim3(256), 0, st, s, q, W,
-                       (const uint16_t *)(dbg ? dbg->qcodes_in : nullptr), ws.qcodes, ws.status, ug);
+                       (const uint16_t *)(dbg ? dbg->qcodes_in : nullptr), ws.qcodes, ws.status, ug, ws.cnt,
+                       units * nchunk);
         if (e != cudaSuccess) return e;
     }
     ScanOut so{ws.cand, ws.cnt, dbg ? dbg->member_out : nullptr, ws.status};
@@ -1990,6 +2025,7 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     aa.scale = scale;
     aa.k8 = k8;
     aa.kmeta = kmeta;
+    aa.status = ws.status;
     if (!fused && path != MP_PATH_TC && k8) {
         const int sm = kAttStages * att_stage_bytes<true>();
         if ((e = ensure_smem(reinterpret_cast<const void *>(attend_kernel<G, true>), sm)) != cudaSuccess) return e;
@@ -2056,15 +2092,15 @@ cudaError_t launch_hash_queries(const Shape &s, const uint16_t *q, const uint16_
 {
     const int TB = qhash_tables_per_block(s.K), units = s.B * s.Hkv;
     const uint16_t *none = nullptr;
-    int32_t *no_status = nullptr;
+    int32_t *no_status = nullptr, *no_flags = nullptr;
     if (s.G != 1 && s.G != 2 && s.G != 4 && s.G != 8) return cudaErrorInvalidValue;
     const int ug = qhash_units_per_block(s, s.G);
     dim3 grid((s.L + TB - 1) / TB, (units + ug - 1) / ug);
     switch (s.G) {
-    case 1: return launch_pdl(qhash_kernel<1>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug);
-    case 2: return launch_pdl(qhash_kernel<2>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug);
-    case 4: return launch_pdl(qhash_kernel<4>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug);
-    default: return launch_pdl(qhash_kernel<8>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug);
+    case 1: return launch_pdl(qhash_kernel<1>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug, no_flags, 0);
+    case 2: return launch_pdl(qhash_kernel<2>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug, no_flags, 0);
+    case 4: return launch_pdl(qhash_kernel<4>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug, no_flags, 0);
+    default: return launch_pdl(qhash_kernel<8>, grid, dim3(256), 0, st, s, q, W, none, qcodes, no_status, ug, no_flags, 0);
     }
 }
 
