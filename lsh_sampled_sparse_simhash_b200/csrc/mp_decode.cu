@@ -1816,16 +1816,22 @@ struct SplitPlan {
 #ifndef MP_ATT_TARGET_BLOCKS
 #define MP_ATT_TARGET_BLOCKS 2400
 #endif
+#ifndef MP_ATT_TARGET_DIV
+#define MP_ATT_TARGET_DIV 6
+#endif
 static SplitPlan split_plan(const Shape &s, int max_len)
 {
     SplitPlan p;
     const int C = chunk_tokens(s);
     p.nchunk = (max_len + C - 1) / C;
     const int blocks = p.nchunk * s.B * s.Hkv;
-    // more, shorter splits pay off on large problems (ragged16: 2400 blocks
-    // 421.5 us per step against 443.4 at 1200), fewer on small ones (ragged4:
-    // 124 us at 1200 against 130 at 2400)
-    const int kTarget = std::min(MP_ATT_TARGET_BLOCKS, std::max(1200, blocks / 12));
+    // More, shorter splits pay off on large problems, fewer on small ones.
+    // Measured per step (bit-plane codes, attention started by the scan's
+    // ready flags): ragged16 (16512 chunk-blocks) 342 us at 2400 blocks (6
+    // chunks a block) against 350 at 4128, 358 at 5504, 367 at 8256 and 355
+    // at 1376; ragged4 and batch8_64k (4128 and 4160) the same within 1% from
+    // 1200 to 2064 blocks.
+    const int kTarget = std::min(MP_ATT_TARGET_BLOCKS, std::max(1200, blocks / MP_ATT_TARGET_DIV));
     if (blocks >= kTarget) {
         p.span = std::min(kMaxSpan, blocks / kTarget);
         p.subs = 1;
