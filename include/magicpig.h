@@ -170,6 +170,12 @@ typedef struct mp_decode_debug {
     uint16_t *qcodes_out;      /* [B][Hq][L]: copy of the query codes used */
     uint8_t *member_out;       /* [B][Hq][Ncap]: 1 iff token i is in S_h (i < N_b) */
     int32_t path;              /* MP_PATH_*: which kernel path to take */
+    int32_t skip_scan;         /* nonzero: launch no collision scan (MP_PATH_AUTO / MP_PATH_SPLIT
+                                  only, else MP_ERR_ARG), so that the attention's bounded waits for
+                                  the scan's per-chunk ready flags run out: each waiting block gives
+                                  up after 1 s, records MP_ERR_CUDA in the status word and returns
+                                  without reading a candidate list; out / lse / n_sampled are then
+                                  undefined.  Tests the failure path without a GPU fault. */
 } mp_decode_debug;
 
 /* Workspace bytes that mp_decode_attend needs for sequences up to max_len. */

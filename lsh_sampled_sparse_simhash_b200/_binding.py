@@ -40,7 +40,7 @@ class _CShape(ctypes.Structure):
 
 class _CDebug(ctypes.Structure):
     _fields_ = [("qcodes_in", ctypes.c_void_p), ("qcodes_out", ctypes.c_void_p),
-                ("member_out", ctypes.c_void_p), ("path", ctypes.c_int32)]
+                ("member_out", ctypes.c_void_p), ("path", ctypes.c_int32), ("skip_scan", ctypes.c_int32)]
 
 
 MP_CODES_AUTO_PLANES_MIN = 1 << 21  # include/magicpig.h
@@ -189,10 +189,12 @@ def append_token(shape: Shape, k_new, v_new, W, k_cache, v_cache, codes, seq_len
 
 
 def decode_attend(shape: Shape, q, W, codes, k_cache, v_cache, seq_lens, max_len: int, out, lse, n_sampled,
-                  workspace, qcodes_in=None, qcodes_out=None, member_out=None, path: int = 0, stream=None):
+                  workspace, qcodes_in=None, qcodes_out=None, member_out=None, path: int = 0, skip_scan: bool = False,
+                  stream=None):
     dbg = None
-    if qcodes_in is not None or qcodes_out is not None or member_out is not None or path:
-        dbg = ctypes.byref(_CDebug(_ptr(qcodes_in), _ptr(qcodes_out), _ptr(member_out), int(path)))
+    if qcodes_in is not None or qcodes_out is not None or member_out is not None or path or skip_scan:
+        dbg = ctypes.byref(_CDebug(_ptr(qcodes_in), _ptr(qcodes_out), _ptr(member_out), int(path),
+                                   int(bool(skip_scan))))
     nbytes = workspace.numel() * workspace.element_size()
     _check(library().mp_decode_attend(ctypes.byref(shape.c()), _ptr(q), _ptr(W), _ptr(codes), _ptr(k_cache),
                                       _ptr(v_cache), _ptr(seq_lens), int(max_len), _ptr(out), _ptr(lse),

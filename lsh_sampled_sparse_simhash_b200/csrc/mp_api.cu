@@ -207,6 +207,7 @@ int mp_decode_attend(const mp_shape *shape, const void *q, const void *W, const 
             return MP_ERR_ALIGN;
         if (debug->path < MP_PATH_AUTO || debug->path > MP_PATH_TC) return MP_ERR_ARG;
         if (debug->path == MP_PATH_FUSED && (!s.planes || s.G > 4)) return MP_ERR_SHAPE;
+        if (debug->skip_scan && debug->path != MP_PATH_AUTO && debug->path != MP_PATH_SPLIT) return MP_ERR_ARG;
     }
     return cuda_status(launch_decode(s, static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(W), codes,
                                      static_cast<const uint16_t *>(k_cache), static_cast<const uint16_t *>(v_cache),

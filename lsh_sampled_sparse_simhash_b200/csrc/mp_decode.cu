@@ -1092,14 +1092,17 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     const int nch = (N + a.chunk_tokens - 1) / a.chunk_tokens;
     if (!dsplit && c_begin >= nch) return;
     if (!dsplit) {
+        __shared__ int flags_ok;
         if (tid == 0) {
             const int c_end = min(c_begin + a.span, nch);
             bool ok = true;
             for (int c = c_begin; c < c_end && ok; c++)
                 ok = flag_wait_bounded(a.cnt + ((size_t)unit * a.nchunk + c) * 16 + 15);
             if (!ok) set_status(a.status, MP_ERR_CUDA);
+            flags_ok = ok;
         }
         __syncthreads();
+        if (!flags_ok) return;  // a list that never became ready is not read
     }
     grid_launch_dependents();
     // A block that takes one chunk's whole list (span = subs = 1) reads the
@@ -1991,7 +1994,7 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
         if (e != cudaSuccess) return e;
         if (!fused && path == MP_PATH_FUSED) return cudaErrorNotSupported;
     }
-    if (nchunk > 0 && !fused) {
+    if (nchunk > 0 && !fused && !(dbg && dbg->skip_scan)) {
         if (!s.planes) {
             const size_t sm = (size_t)kByteWarps * kByteRing * kChunkBytes + (size_t)s.L * std::max(G, 4) * sizeof(uint32_t);
             if ((e = ensure_smem(reinterpret_cast<const void *>(scan_bytes_kernel<G>), (int)sm)) != cudaSuccess)

@@ -111,7 +111,8 @@ class Run:
                              device="cuda")
         self.kmeta = torch.full((w.batch, w.n_kv_heads, w.capacity, 4), -1.0, dtype=torch.float32, device="cuda")
 
-    def decode(self, qcodes_in: Optional[np.ndarray] = None, member: bool = True, path: int = 0, q8: bool = False):
+    def decode(self, qcodes_in: Optional[np.ndarray] = None, member: bool = True, path: int = 0, q8: bool = False,
+               skip_scan: bool = False):
         """One decode step; with q8 the K rows come from the int8 copy."""
         w = self.w
         mem = torch.zeros((w.batch, w.n_q_heads, w.capacity), dtype=torch.uint8, device="cuda") if member else None
@@ -124,7 +125,7 @@ class Run:
         else:
             mp.decode_attend(self.shape, self.q, self.W, self.codes, self.K, self.V, self.lens, self.max_len,
                              self.out, self.lse, self.ns, self.ws, qcodes_in=qci, qcodes_out=qco, member_out=mem,
-                             path=path)
+                             path=path, skip_scan=skip_scan)
         torch.cuda.synchronize()
         res = dict(out=host(self.out), lse=host(self.lse), ns=host(self.ns), qcodes=host(qco, np.uint16))
         if member:

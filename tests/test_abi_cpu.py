@@ -185,3 +185,18 @@ def test_auto_layout_threshold_matches_header():
     assert not mp.auto_planes(1, 8, 16512, 8)        # a 16k-token layer: byte codes
     assert mp.auto_planes(4, 8, 131200, 8)           # four 128k-token sequences: bit planes
     assert mp.auto_planes(1, 1, 128, 10)             # K = 10: always bit planes
+
+
+def test_skip_scan_hook_only_on_the_split_path(lib):
+    """mp_decode_debug.skip_scan (the failure-path test hook) is refused with
+    the fused and tcgen05 paths, whose kernels would not wait for the scan's
+    flags; rejected on the host, so nothing launches."""
+    A = 1 << 12
+    s = good_shape(code_layout=2, n_q_heads=8)
+    need = ctypes.c_size_t()
+    assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 1024, ctypes.byref(need)) == 0
+    for path in (mp.MP_PATH_FUSED, mp.MP_PATH_TC):
+        dbg = B._CDebug(None, None, None, path, 1)
+        rc = lib.mp_decode_attend(ctypes.byref(s), A, A, A, A, A, A, 1024, A, A, A, A, need.value, ctypes.byref(dbg),
+                                  None)
+        assert rc == mp.MP_ERR_ARG, (path, rc)

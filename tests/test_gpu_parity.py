@@ -479,3 +479,27 @@ def _full_size(name, path):
     worst = check_outputs(gpu, ref, w)
     print(f"{name} (path {path}): {len(units)} units' candidate sets exact; worst rel-L2 {worst:.2e} over "
           f"{len(picked)} units; mean |S_h| {gpu['ns'].mean():.0f}; {exempt} near-zero code bits exempt")
+
+
+@pytest.mark.parametrize("case", ["tiny_g1_k8", "g4_k8_planes"])
+def test_attention_wait_for_a_missing_scan_runs_out(case):
+    """Failure path without a GPU fault: with the scan left out (test hook),
+    no chunk's ready flag is ever set, so every attention block that reads a
+    candidate list gives up after its bounded wait, records MP_ERR_CUDA and
+    returns without reading one.  The context stays usable: the next call on
+    the same buffers is clean and matches the oracle."""
+    import time
+    w = SMALL_CASES[case]
+    inp = make_inputs(w)
+    run = Run(w, inp)
+    units, codes, _ = oracle_codes_all(run)
+    run.set_codes(codes, units)
+    qref, _ = oracle_query_codes(inp, w)
+    t0 = time.time()
+    bad = run.decode(qcodes_in=qref, skip_scan=True)
+    assert bad["status"] == mp.MP_ERR_CUDA
+    assert time.time() - t0 < 30
+    good = run.decode(qcodes_in=qref)
+    assert good["status"] == 0
+    ref = oracle_decode_units(inp, w, units, codes, qref)
+    check_outputs(good, ref, w)
