@@ -10,7 +10,6 @@ namespace mp {
 
 constexpr int kHeadDim = 128;
 constexpr int kMaxGroup = 8;
-constexpr int kScanThreads = 256;  // scan block: token groups x table splits
 constexpr int kSplitsK8 = 8;       // byte codes: tables l = ts, ts + 8, ... per split
 constexpr int kSplitsPlanes = 8;   // bit planes: tables l = ts, ts + 8, ... per split (a warp each)
 constexpr int kChunkBytes = 512;   // scan chunk (tokens) for byte codes: 32 groups x 16 tokens
@@ -43,11 +42,16 @@ __device__ __forceinline__ void grid_dependency_wait()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 // The two halves, for a kernel with work that does not depend on its
-// immediate predecessor.  Every kernel of this library lets its successor
-// launch only after its own wait has returned, so when a kernel starts, all
-// stream work before its predecessor is complete and visible: code before
-// grid_wait() may read that (cached codes, lengths), but nothing its
-// predecessor writes, and it writes no global memory.
+// immediate predecessor.  The kernels of this library let their successor
+// launch only after their own wait has returned (the query hash only at its
+// very end, after clearing the status words and ready flags), so when a
+// kernel starts, all stream work before its predecessor is complete and
+// visible: code before grid_wait() may read that (cached codes, lengths), but
+// nothing its predecessor writes.  Two exceptions, each with its own
+// ordering: the collision scan lets the attention launch as soon as it starts
+// (the attention then waits per chunk on the scan's ready flags, not on the
+// scan grid), and the attention lets the merge launch once its own flags are
+// in (the merge waits for the whole attention grid before reading).
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void grid_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
