@@ -37,6 +37,9 @@ SMALL_CASES = {
     "g4_k8_planes": TINY.with_(name="k8p", batch=2, n_q_heads=8, n_kv_heads=2, context=9100, n_planted=16,
                                seed=2006, code_layout="planes"),
     "g1_k8_planes_short": TINY.with_(name="k8p1", context=1000, n_planted=8, seed=2007, code_layout="planes"),
+    # capacity 1536: the last 1024-token chunk of every unit is half past the capacity
+    "g4_k8_planes_part_chunk": TINY.with_(name="k8pc", batch=3, n_q_heads=8, n_kv_heads=2, context=1500,
+                                         ragged_min=600, n_planted=8, seed=2008, code_layout="planes"),
 }
 
 
@@ -165,7 +168,7 @@ def test_ragged_batch_of_many_units():
     check_outputs(gpu, ref, w)
 
 
-PLANE_CASES = ["g4_k10", "g2_k10_short", "g4_k8_planes", "g1_k8_planes_short"]
+PLANE_CASES = ["g4_k10", "g2_k10_short", "g4_k8_planes", "g1_k8_planes_short", "g4_k8_planes_part_chunk"]
 
 
 @pytest.mark.parametrize("path", [mp.MP_PATH_SPLIT, mp.MP_PATH_FUSED])
