@@ -89,6 +89,22 @@ def test_decode_bytes_hand_count():
     assert codes == 103 * 2 * 75
     assert d_rows == (68 + 3) * 2
     assert total == codes + (10 + d_rows) * 512
+    # int8 keys: 128 B of K, its 16-byte record and 256 B of V per row
+    total8, codes8, d_rows8 = bench.decode_bytes(w, np.array([100, 3]), 10, "int8")
+    assert (codes8, d_rows8) == (codes, d_rows)
+    assert total8 == codes + (10 + d_rows) * (128 + 16 + 256)
+
+
+def test_code_layout_of_follows_the_library_rule():
+    """The bench reports the layout the library picks for MP_CODES_AUTO:
+    bit planes for the large K = 8 workloads and K = 10, byte codes for the
+    16k-token layer."""
+    import workloads
+    assert bench.code_layout_of(workloads.get("ragged16")) == "planes"
+    assert bench.code_layout_of(workloads.get("ragged4")) == "planes"
+    assert bench.code_layout_of(workloads.get("batch8_64k")) == "planes"
+    assert bench.code_layout_of(workloads.get("llama8b_16k")) == "bytes"
+    assert bench.code_layout_of(workloads.get("ragged16").with_(code_layout="bytes")) == "bytes"
 
 
 def test_oracle_sample_units_spread_over_the_batch():
