@@ -93,9 +93,10 @@ typedef struct mp_shape {
  *                   (l, w, b) = bit b of the table-l code of token 32*w + t
  *                   (the K planes of each 32-token group are adjacent).
  * Both use exactly L*K/8 bytes per token; mp_codes_bytes gives the size.  The
- * byte layout is the default for k_bits == 8; the plane layout lets the
- * collision scan compare 32 tokens per logical operation (about 4x fewer
- * integer operations than byte compares for K = 8).
+ * plane layout lets the collision scan test 32 tokens per logical operation
+ * (K + 2 operations per 32 tokens and query head, against one packed compare
+ * per token and head for bytes), which MP_CODES_AUTO uses except on small
+ * K = 8 problems.
  */
 int mp_codes_bytes(const mp_shape *shape, size_t *bytes);
 
@@ -106,8 +107,8 @@ int mp_codes_bytes(const mp_shape *shape, size_t *bytes);
  *   W      bf16 [L*K][d]            hyperplanes, row c = l*K + b
  *   seq_lens  int32 [B] device, nullable: if given, unit (b, .) hashes only
  *          tokens [0, min(seq_lens[b], n_tokens)) (ragged batches)
- *   codes  out, layout above; only the hashed tokens are written (for
- *          k_bits == 10 the last partial 32-token word is rewritten whole).
+ *   codes  out, layout above; only the hashed tokens are written (with bit
+ *          planes the last partial 32-token word is rewritten whole).
  *   status int32 device word (nullable): MP_ERR_CUDA if the kernel's internal
  *          pipeline stalled (a bounded wait expired; the codes are then
  *          incomplete).  Never written on success.
