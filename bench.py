@@ -119,8 +119,8 @@ def step_tokens(lens_after):
 
 def row_bytes(w, k_format="bf16"):
     """Bytes of one gathered (token, kv head) row: k + v in bf16 (512 at
-    d = 128), or the int8 k, its 16-byte {scale, norm} record and the bf16 v
-    (400)."""
+    d = 128), or the 144-byte int8 row (values and {scale, norm} record) and
+    the bf16 v (400)."""
     return (w.head_dim + 16 if k_format == "int8" else 2 * w.head_dim) + 2 * w.head_dim
 
 
@@ -250,8 +250,7 @@ class Bench:
         self.with_hash = hash_in_step(w)
         self.q8 = k_format == "int8"
         if self.q8:
-            self.k8 = torch.empty((B, w.n_kv_heads, w.capacity, d), dtype=torch.int8, device=device)
-            self.kmeta = torch.empty((B, w.n_kv_heads, w.capacity, 4), dtype=torch.float32, device=device)
+            self.k8 = torch.empty((B, w.n_kv_heads, w.capacity, mp.Q8_ROW_BYTES), dtype=torch.int8, device=device)
         fused = self.path == mp.MP_PATH_FUSED
         # append 1, decode: qhash + (scan, attention | fused) + merge; hash 1
         # (and with int8 keys the quantisation, 1) if in the step
@@ -267,7 +266,7 @@ class Bench:
     def quantize(self):
         """The int8 copy of the cached keys (with --k-format int8)."""
         if self.q8:
-            self.mp.quantize_keys(self.shape, self.K, self.k8, self.kmeta, n_tokens=self.prefill,
+            self.mp.quantize_keys(self.shape, self.K, self.k8, n_tokens=self.prefill,
                                   seq_lens=self.lens0)
 
     def build(self):
@@ -278,13 +277,13 @@ class Bench:
     def append(self):
         if self.q8:
             self.mp.append_token_q8(self.shape, self.k_new, self.v_new, self.W, self.K, self.V, self.codes,
-                                    self.lens, self.k8, self.kmeta)
+                                    self.lens, self.k8)
         else:
             self.mp.append_token(self.shape, self.k_new, self.v_new, self.W, self.K, self.V, self.codes, self.lens)
 
     def decode(self, member_out=None):
         if self.q8:
-            self.mp.decode_attend_q8(self.shape, self.q, self.W, self.codes, self.k8, self.kmeta, self.V,
+            self.mp.decode_attend_q8(self.shape, self.q, self.W, self.codes, self.k8, self.V,
                                      self.lens, self.max_len, self.out, self.lse, self.ns, self.ws,
                                      member_out=member_out, path=self.path)
         else:

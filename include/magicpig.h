@@ -238,13 +238,15 @@ int mp_decode_attend_noalloc(const mp_shape *shape, const void *q, const void *W
  * int8 keys for the attention gather (opt-in; the method itself reads the
  * cached keys in their own precision, so this is a reduced-precision variant
  * of the step, not part of the method's description).  The bf16 key cache
- * stays authoritative: the hash codes are always computed from it, and the
- * int8 copy only replaces the K rows that the sampled attention gathers
- * (144 bytes per row instead of 256; the V rows and codes are unchanged).
+ * stays authoritative for hashing: the codes are always computed from bf16
+ * keys, and the int8 copy only replaces the K rows that the sampled attention
+ * gathers (144 bytes per row instead of 256; the V rows and codes are
+ * unchanged).
  *
- * Format: row (b, h, i) of the bf16 keys k (d = 128 values) is stored as
- *   k8[b][h][i][j] = rint(k_j / s)   (round half to even; int8 in [-127, 127])
- *   kmeta[b][h][i] = {s, |s q|^2, 0, 0}   (fp32 x 4, 16 bytes)
+ * Format: row (b, h, i) of the bf16 keys k (d = 128 values) is stored as 144
+ * contiguous bytes, k8[b][h][i][0 .. 143]:
+ *   bytes 0 .. 127    q_j = rint(k_j / s)   (round half to even; int8 in [-127, 127])
+ *   bytes 128 .. 143  the record {s, |s q|^2, 0, 0}   (fp32 x 4)
  * where s = 2^e is the smallest power of two with 127 s >= max_j |k_j| (s = 0
  * and q = 0 for a zero row).  s is a power of two, so s * q is exactly a bf16
  * value and the stored squared norm is exact: the attention runs on the keys
@@ -253,42 +255,42 @@ int mp_decode_attend_noalloc(const mp_shape *shape, const void *q, const void *W
  * score products as f16 (exact for bf16 values of magnitude 2^-17 .. 65504).
  * Expected cost, measured on the fp64 estimator: about 1e-2 relative L2 on
  * the output of a head.
- *   k8      int8 [B][Hkv][Ncap][d], 16-byte aligned, caller-owned
- *   kmeta   fp32 [B][Hkv][Ncap][4], 16-byte aligned, caller-owned
+ *   k8  int8 [B][Hkv][Ncap][MP_Q8_ROW_BYTES], 16-byte aligned, caller-owned
  */
+#define MP_Q8_ROW_BYTES 144
 
 /*
- * Writes the int8 copy (k8, kmeta) of key rows [first_token, first_token +
+ * Writes the int8 rows (k8) of key rows [first_token, first_token +
  * n_tokens) of every (b, kv head), stopping at seq_lens[b] when seq_lens
  * (int32 [B], device, nullable) is given.  Errors: MP_ERR_ARG (null pointer),
  * MP_ERR_ALIGN, MP_ERR_CAPACITY (range outside [0, Ncap]); nothing launched.
  */
 int mp_quantize_keys(const mp_shape *shape, const void *k_cache, const int32_t *seq_lens, int32_t first_token,
-                     int32_t n_tokens, int8_t *k8, float *kmeta, void *stream);
+                     int32_t n_tokens, int8_t *k8, void *stream);
 
 /*
- * mp_append_token that also writes the int8 copy of each appended key row
- * into k8 / kmeta at the same position (one launch).  Same arguments and
- * status behaviour as mp_append_token otherwise, except that k_cache may be
- * NULL: then no bf16 key row is written, and a caller that decodes only
- * through mp_decode_attend_q8 keeps 400 instead of 512 bytes of key-value
- * cache per (token, kv head) (the bf16 keys are needed again only to rebuild
- * the codes, e.g. for a new W).
+ * mp_append_token that also writes the int8 row of each appended key into
+ * k8 at the same position (one launch).  Same arguments and status behaviour
+ * as mp_append_token otherwise, except that k_cache may be NULL: then no bf16
+ * key row is written, and a caller that decodes only through
+ * mp_decode_attend_q8 keeps 400 instead of 512 bytes of key-value cache per
+ * (token, kv head) (the bf16 keys are needed again only to rebuild the codes,
+ * e.g. for a new W).
  */
 int mp_append_token_q8(const mp_shape *shape, const void *k_new, const void *v_new, const void *W,
-                       void *k_cache, void *v_cache, void *codes, int32_t *seq_lens, int8_t *k8, float *kmeta,
-                       int32_t *status, void *stream);
+                       void *k_cache, void *v_cache, void *codes, int32_t *seq_lens, int8_t *k8, int32_t *status,
+                       void *stream);
 
 /*
- * mp_decode_attend with the K rows gathered from the int8 copy (k8, kmeta)
- * instead of a bf16 cache; every other argument and result as there.
+ * mp_decode_attend with the K rows gathered from the int8 rows (k8) instead
+ * of a bf16 cache; every other argument and result as there.
  * debug->path may be MP_PATH_AUTO or MP_PATH_SPLIT; MP_PATH_FUSED and
  * MP_PATH_TC return MP_ERR_SHAPE (those kernels read bf16 keys only).
  */
 int mp_decode_attend_q8(const mp_shape *shape, const void *q, const void *W, const void *codes,
-                        const int8_t *k8, const float *kmeta, const void *v_cache, const int32_t *seq_lens,
-                        int32_t max_len, float *out, float *lse, int32_t *n_sampled, void *workspace,
-                        size_t workspace_bytes, const mp_decode_debug *debug, void *stream);
+                        const int8_t *k8, const void *v_cache, const int32_t *seq_lens, int32_t max_len,
+                        float *out, float *lse, int32_t *n_sampled, void *workspace, size_t workspace_bytes,
+                        const mp_decode_debug *debug, void *stream);
 
 /* Synchronises `stream` and reads the status word of a decode workspace. */
 int mp_read_status(const void *workspace, int32_t *status, void *stream);

@@ -38,6 +38,7 @@ from ._binding import (  # noqa: F401
     MP_CODES_BYTES,
     MP_CODES_PLANES,
     MP_CODES_AUTO_PLANES_MIN,
+    Q8_ROW_BYTES,
     MP_PATH_AUTO,
     MP_PATH_SPLIT,
     MP_PATH_FUSED,

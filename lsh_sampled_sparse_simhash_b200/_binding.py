@@ -98,9 +98,9 @@ def library() -> ctypes.CDLL:
         lib.mp_decode_attend.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P, SZ,
                                          ctypes.POINTER(_CDebug), P]
         lib.mp_decode_attend_noalloc.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P, P]
-        lib.mp_quantize_keys.argtypes = [SP, P, P, I32, I32, P, P, P]
-        lib.mp_append_token_q8.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P]
-        lib.mp_decode_attend_q8.argtypes = [SP, P, P, P, P, P, P, P, I32, P, P, P, P, SZ,
+        lib.mp_quantize_keys.argtypes = [SP, P, P, I32, I32, P, P]
+        lib.mp_append_token_q8.argtypes = [SP, P, P, P, P, P, P, P, P, P, P]
+        lib.mp_decode_attend_q8.argtypes = [SP, P, P, P, P, P, P, I32, P, P, P, P, SZ,
                                             ctypes.POINTER(_CDebug), P]
         lib.mp_read_status.argtypes = [P, ctypes.POINTER(I32), P]
         lib.mp_status_string.argtypes = [ctypes.c_int]
@@ -212,25 +212,28 @@ def decode_attend_noalloc(shape: Shape, q, W, codes, k_cache, v_cache, seq_lens,
                                               _stream(stream)), "mp_decode_attend_noalloc")
 
 
-def quantize_keys(shape: Shape, k_cache, k8, kmeta, first_token: int = 0, n_tokens: Optional[int] = None,
+Q8_ROW_BYTES = 144  # MP_Q8_ROW_BYTES
+
+
+def quantize_keys(shape: Shape, k_cache, k8, first_token: int = 0, n_tokens: Optional[int] = None,
                   seq_lens=None, stream=None):
-    """Writes the int8 copy of key rows [first_token, first_token + n_tokens)
-    (default: the whole capacity): k8 int8 [B,Hkv,Ncap,d] and kmeta fp32
-    [B,Hkv,Ncap,4] = {power-of-two scale, squared norm of the int8 row times
-    the scale, 0, 0} per row."""
+    """Writes the int8 rows of key rows [first_token, first_token + n_tokens)
+    (default: the whole capacity) into k8, int8 [B,Hkv,Ncap,144]: 128 int8
+    values, then the fp32 record {power-of-two scale, squared norm of the
+    int8 row times the scale, 0, 0}."""
     n = shape.capacity - int(first_token) if n_tokens is None else int(n_tokens)
     _check(library().mp_quantize_keys(ctypes.byref(shape.c()), _ptr(k_cache), _ptr(seq_lens), int(first_token), n,
-                                      _ptr(k8), _ptr(kmeta), _stream(stream)), "mp_quantize_keys")
+                                      _ptr(k8), _stream(stream)), "mp_quantize_keys")
 
 
-def append_token_q8(shape: Shape, k_new, v_new, W, k_cache, v_cache, codes, seq_lens, k8, kmeta, status=None,
+def append_token_q8(shape: Shape, k_new, v_new, W, k_cache, v_cache, codes, seq_lens, k8, status=None,
                     stream=None):
     _check(library().mp_append_token_q8(ctypes.byref(shape.c()), _ptr(k_new), _ptr(v_new), _ptr(W),
                                         _ptr(k_cache), _ptr(v_cache), _ptr(codes), _ptr(seq_lens), _ptr(k8),
-                                        _ptr(kmeta), _ptr(status), _stream(stream)), "mp_append_token_q8")
+                                        _ptr(status), _stream(stream)), "mp_append_token_q8")
 
 
-def decode_attend_q8(shape: Shape, q, W, codes, k8, kmeta, v_cache, seq_lens, max_len: int, out, lse, n_sampled,
+def decode_attend_q8(shape: Shape, q, W, codes, k8, v_cache, seq_lens, max_len: int, out, lse, n_sampled,
                      workspace, qcodes_in=None, qcodes_out=None, member_out=None, path: int = 0, stream=None):
     """decode_attend with the K rows gathered from the int8 copy."""
     dbg = None
@@ -238,7 +241,7 @@ def decode_attend_q8(shape: Shape, q, W, codes, k8, kmeta, v_cache, seq_lens, ma
         dbg = ctypes.byref(_CDebug(_ptr(qcodes_in), _ptr(qcodes_out), _ptr(member_out), int(path)))
     nbytes = workspace.numel() * workspace.element_size()
     _check(library().mp_decode_attend_q8(ctypes.byref(shape.c()), _ptr(q), _ptr(W), _ptr(codes), _ptr(k8),
-                                         _ptr(kmeta), _ptr(v_cache), _ptr(seq_lens), int(max_len), _ptr(out),
+                                         _ptr(v_cache), _ptr(seq_lens), int(max_len), _ptr(out),
                                          _ptr(lse), _ptr(n_sampled), _ptr(workspace), nbytes, dbg,
                                          _stream(stream)), "mp_decode_attend_q8")
 

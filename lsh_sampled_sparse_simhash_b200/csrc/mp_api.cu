@@ -147,36 +147,36 @@ int mp_append_token(const mp_shape *shape, const void *k_new, const void *v_new,
     if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return MP_ERR_ALIGN;
     return cuda_status(launch_append(s, static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new),
                                      static_cast<const uint16_t *>(W), static_cast<uint16_t *>(k_cache),
-                                     static_cast<uint16_t *>(v_cache), codes, seq_lens, status, nullptr, nullptr,
+                                     static_cast<uint16_t *>(v_cache), codes, seq_lens, status, nullptr,
                                      static_cast<cudaStream_t>(stream)));
 }
 
 int mp_quantize_keys(const mp_shape *shape, const void *k_cache, const int32_t *seq_lens, int32_t first_token,
-                     int32_t n_tokens, int8_t *k8, float *kmeta, void *stream)
+                     int32_t n_tokens, int8_t *k8, void *stream)
 {
     Shape s;
     int r = validate_shape(shape, s);
     if (r) return r;
-    if ((r = check_ptrs({k_cache, k8, kmeta}))) return r;
+    if ((r = check_ptrs({k_cache, k8}))) return r;
     if (seq_lens && (reinterpret_cast<uintptr_t>(seq_lens) & 3u)) return MP_ERR_ALIGN;
     if (first_token < 0 || n_tokens < 0 || (int64_t)first_token + n_tokens > s.Ncap) return MP_ERR_CAPACITY;
     return cuda_status(launch_quantize_keys(s, static_cast<const uint16_t *>(k_cache), seq_lens, first_token,
-                                            n_tokens, k8, kmeta, static_cast<cudaStream_t>(stream)));
+                                            n_tokens, k8, static_cast<cudaStream_t>(stream)));
 }
 
 int mp_append_token_q8(const mp_shape *shape, const void *k_new, const void *v_new, const void *W, void *k_cache,
-                       void *v_cache, void *codes, int32_t *seq_lens, int8_t *k8, float *kmeta, int32_t *status,
+                       void *v_cache, void *codes, int32_t *seq_lens, int8_t *k8, int32_t *status,
                        void *stream)
 {
     Shape s;
     int r = validate_shape(shape, s);
     if (r) return r;
-    if ((r = check_ptrs({k_new, v_new, W, v_cache, codes, seq_lens, k8, kmeta}))) return r;
+    if ((r = check_ptrs({k_new, v_new, W, v_cache, codes, seq_lens, k8}))) return r;
     if (k_cache && !aligned16(k_cache)) return MP_ERR_ALIGN;  // null: the int8 copy is the only key cache
     if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return MP_ERR_ALIGN;
     return cuda_status(launch_append(s, static_cast<const uint16_t *>(k_new), static_cast<const uint16_t *>(v_new),
                                      static_cast<const uint16_t *>(W), static_cast<uint16_t *>(k_cache),
-                                     static_cast<uint16_t *>(v_cache), codes, seq_lens, status, k8, kmeta,
+                                     static_cast<uint16_t *>(v_cache), codes, seq_lens, status, k8,
                                      static_cast<cudaStream_t>(stream)));
 }
 
@@ -216,14 +216,14 @@ int mp_decode_attend(const mp_shape *shape, const void *q, const void *W, const 
 }
 
 int mp_decode_attend_q8(const mp_shape *shape, const void *q, const void *W, const void *codes, const int8_t *k8,
-                        const float *kmeta, const void *v_cache, const int32_t *seq_lens, int32_t max_len,
+                        const void *v_cache, const int32_t *seq_lens, int32_t max_len,
                         float *out, float *lse, int32_t *n_sampled, void *workspace, size_t workspace_bytes,
                         const mp_decode_debug *debug, void *stream)
 {
     Shape s;
     int r = validate_shape(shape, s);
     if (r) return r;
-    if ((r = check_ptrs({q, W, codes, k8, kmeta, v_cache, seq_lens, out, lse, n_sampled, workspace}))) return r;
+    if ((r = check_ptrs({q, W, codes, k8, v_cache, seq_lens, out, lse, n_sampled, workspace}))) return r;
     if (max_len < 0 || max_len > s.Ncap) return MP_ERR_CAPACITY;
     if (workspace_bytes < decode_workspace_bytes(s, max_len)) return MP_ERR_WORKSPACE;
     if (debug) {
@@ -234,7 +234,7 @@ int mp_decode_attend_q8(const mp_shape *shape, const void *q, const void *W, con
     }
     return cuda_status(launch_decode(s, static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(W), codes,
                                      nullptr, static_cast<const uint16_t *>(v_cache), seq_lens, max_len, out, lse,
-                                     n_sampled, workspace, debug, static_cast<cudaStream_t>(stream), k8, kmeta));
+                                     n_sampled, workspace, debug, static_cast<cudaStream_t>(stream), k8));
 }
 
 int mp_read_status(const void *workspace, int32_t *status, void *stream)

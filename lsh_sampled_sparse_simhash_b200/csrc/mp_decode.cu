@@ -693,8 +693,7 @@ struct AttendArgs {
     float *pm, *pl, *pacc;  // [B*Hq][ngroups*subs+1], [..][..][128]
     LogU lu;
     float scale;  // 1/sqrt(d)
-    const int8_t *k8;      // int8 keys [B][Hkv][Ncap][128] (attend_kernel<G, true>), else null
-    const float *kmeta;    // their per-row records {scale, squared norm, 0, 0} [B][Hkv][Ncap][4]
+    const int8_t *k8;      // int8 key rows [B][Hkv][Ncap][kQ8RowBytes] (attend_kernel<G, true>), else null
     int32_t *status;       // the call's status word (a ready flag that never came: MP_ERR_CUDA)
 };
 
@@ -1165,8 +1164,7 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
     attn_qinv<G>(a.q, vec0, warp, lane, qinv);
 
     const uint16_t *kbase = Q8 ? nullptr : a.kc + (size_t)unit * s.Ncap * kHeadDim;
-    const int8_t *k8base = Q8 ? a.k8 + (size_t)unit * s.Ncap * kHeadDim : nullptr;
-    const float *kmbase = Q8 ? a.kmeta + (size_t)unit * s.Ncap * kQ8MetaFloats : nullptr;
+    const int8_t *k8base = Q8 ? a.k8 + (size_t)unit * s.Ncap * kQ8RowBytes : nullptr;
     const uint16_t *vbase = a.vc + (size_t)unit * s.Ncap * kHeadDim;
     const int ntiles = (nrows + kAttRows - 1) / kAttRows;
 
@@ -1200,12 +1198,10 @@ __global__ void __launch_bounds__(kAttThreads, 3) attend_kernel(AttendArgs a)
             const bool ok = ent != 0xFFFFFFFFu;
             const int tok = ok ? (int)(ent & 0xFFFFFFu) : 0;
             const size_t off = (size_t)tok * kHeadDim + col * 8;
-            if constexpr (Q8) {  // 8 pieces of the int8 row, then its 16-byte record
+            if constexpr (Q8) {  // the 9 pieces of the 144-byte row: 8 of values, then the record
                 if (col < 9) {
                     void *dst = col < 8 ? (void *)(ks_ + r * KS + att_piece(r, col)) : (void *)&kq[warp][stage][r];
-                    const void *src = col < 8 ? (const void *)(k8base + (size_t)tok * kHeadDim + col * 16)
-                                              : (const void *)(kmbase + (size_t)tok * kQ8MetaFloats);
-                    cp_async_16(dst, src, ok ? 16 : 0);
+                    cp_async_16(dst, k8base + (size_t)tok * kQ8RowBytes + col * 16, ok ? 16 : 0);
                 }
             } else {
                 cp_async_16(ks_ + r * KS + att_piece(r, col), kbase + off, ok ? 16 : 0);
@@ -1948,7 +1944,7 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
                                    const uint16_t *kc, const uint16_t *vc, const int32_t *seq_lens,
                                    int max_len, float *out, float *lse, int32_t *n_sampled,
                                    const Workspace &ws, const mp_decode_debug *dbg, cudaStream_t st,
-                                   const int8_t *k8, const float *kmeta)
+                                   const int8_t *k8)
 {
     const int C = chunk_tokens(s);
     const SplitPlan sp = split_plan(s, max_len);
@@ -2033,7 +2029,6 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
     aa.lu = lu;
     aa.scale = scale;
     aa.k8 = k8;
-    aa.kmeta = kmeta;
     aa.status = ws.status;
     if (!fused && path != MP_PATH_TC && k8) {
         const int sm = kAttStages * att_stage_bytes<true>();
@@ -2084,14 +2079,14 @@ static cudaError_t launch_decode_g(const Shape &s, const uint16_t *q, const uint
 cudaError_t launch_decode(const Shape &s, const uint16_t *q, const uint16_t *W, const void *codes,
                           const uint16_t *kc, const uint16_t *vc, const int32_t *seq_lens, int max_len,
                           float *out, float *lse, int32_t *n_sampled, void *workspace,
-                          const mp_decode_debug *dbg, cudaStream_t st, const int8_t *k8, const float *kmeta)
+                          const mp_decode_debug *dbg, cudaStream_t st, const int8_t *k8)
 {
     const Workspace ws = workspace_layout(s, max_len, workspace);
     switch (s.G) {
-    case 1: return launch_decode_g<1>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8, kmeta);
-    case 2: return launch_decode_g<2>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8, kmeta);
-    case 4: return launch_decode_g<4>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8, kmeta);
-    case 8: return launch_decode_g<8>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8, kmeta);
+    case 1: return launch_decode_g<1>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8);
+    case 2: return launch_decode_g<2>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8);
+    case 4: return launch_decode_g<4>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8);
+    case 8: return launch_decode_g<8>(s, q, W, codes, kc, vc, seq_lens, max_len, out, lse, n_sampled, ws, dbg, st, k8);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
                                                                 const uint16_t *__restrict__ v_new,
                                                                 const uint16_t *__restrict__ W, uint16_t *kc,
                                                                 uint16_t *vc, void *codes, int32_t *seq_lens,
-                                                                int32_t *status, int8_t *k8, float *kmeta)
+                                                                int32_t *status, int8_t *k8)
 {
     // shared: this block's W rows [T K][kHeadDim] bf16, the new keys
     // [Hkv][kHeadDim + 4] fp32 (element d at d + d / 32), the bits [Hkv][T K]
@@ -67,8 +67,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
         } else if (r == 1 && k8) {  // the int8 copy of the new keys, a warp per kv head
             for (int h = tid >> 5; h < s.Hkv; h += blockDim.x >> 5) {
                 const size_t row = (unit0 + h) * s.Ncap + pos;
-                quantize_key_row(k_new + (unit0 + h) * kHeadDim, k8 + row * kHeadDim, kmeta + row * kQ8MetaFloats,
-                                 tid & 31);
+                quantize_key_row(k_new + (unit0 + h) * kHeadDim, k8 + row * kQ8RowBytes, tid & 31);
             }
         }
         for (int i = tid; i < s.Hkv * kHeadDim; i += blockDim.x) {
@@ -141,7 +140,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape s, const u
 
 cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t *v_new, const uint16_t *W,
                           uint16_t *kc, uint16_t *vc, void *codes, int32_t *seq_lens, int32_t *status,
-                          int8_t *k8, float *kmeta, cudaStream_t st)
+                          int8_t *k8, cudaStream_t st)
 {
     const int T = (s.L + kAppendCluster - 1) / kAppendCluster;
     const size_t smem = (size_t)T * s.K * kHeadDim * 2 + (size_t)s.Hkv * (kHeadDim + 4) * sizeof(float) +
@@ -162,7 +161,7 @@ cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, append_kernel, s, k_new, v_new, W, kc, vc, codes, seq_lens, status, k8, kmeta);
+    return cudaLaunchKernelEx(&cfg, append_kernel, s, k_new, v_new, W, kc, vc, codes, seq_lens, status, k8);
 }
 
 }  // namespace mp

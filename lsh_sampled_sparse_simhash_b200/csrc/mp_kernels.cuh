@@ -23,21 +23,20 @@ cudaError_t launch_hash_keys_tc(const Shape &s, const uint16_t *keys, const uint
                                 int tok0, int n_tokens, void *codes, int32_t *status, cudaStream_t st);
 cudaError_t launch_hash_queries(const Shape &s, const uint16_t *q, const uint16_t *W, uint16_t *qcodes,
                                 cudaStream_t st);
-// k8 / kmeta (nullable): also write the int8 copy of the new keys (mp_kquant.cuh).
+// k8 (nullable): also write the int8 rows of the new keys (mp_kquant.cuh).
 cudaError_t launch_append(const Shape &s, const uint16_t *k_new, const uint16_t *v_new, const uint16_t *W,
                           uint16_t *kc, uint16_t *vc, void *codes, int32_t *seq_lens, int32_t *status,
-                          int8_t *k8, float *kmeta, cudaStream_t st);
-// With k8 / kmeta (non-null) the attention gathers the int8 keys and their
-// {scale, squared norm} records instead of kc (the two-kernel path only).
+                          int8_t *k8, cudaStream_t st);
+// With k8 (non-null) the attention gathers the int8 key rows (values and
+// {scale, squared norm} record) instead of kc (the two-kernel path only).
 cudaError_t launch_decode(const Shape &s, const uint16_t *q, const uint16_t *W, const void *codes,
                           const uint16_t *kc, const uint16_t *vc, const int32_t *seq_lens, int max_len,
                           float *out, float *lse, int32_t *n_sampled, void *workspace,
-                          const mp_decode_debug *dbg, cudaStream_t st, const int8_t *k8 = nullptr,
-                          const float *kmeta = nullptr);
+                          const mp_decode_debug *dbg, cudaStream_t st, const int8_t *k8 = nullptr);
 // int8 copy of the keys of tokens [tok0, tok0 + n_tokens) of every unit (with
 // seq_lens, unit (b, .) stops at seq_lens[b]).
 cudaError_t launch_quantize_keys(const Shape &s, const uint16_t *kc, const int32_t *seq_lens, int tok0, int n_tokens,
-                                 int8_t *k8, float *kmeta, cudaStream_t st);
+                                 int8_t *k8, cudaStream_t st);
 size_t decode_workspace_bytes(const Shape &s, int max_len);
 
 // Sampled attention on the tensor cores (mp_attend_tc.cu): every work item of

@@ -16,7 +16,7 @@ constexpr int kQuantRowsPerBlock = 8 * kQuantRowsPerWarp;
 // unit (b, .) stops at seq_lens[b].
 __global__ void __launch_bounds__(256) quantize_keys_kernel(Shape s, const uint16_t *__restrict__ kc,
                                                             const int32_t *__restrict__ seq_lens, int tok0,
-                                                            int n_tokens, int8_t *k8, float *kmeta)
+                                                            int n_tokens, int8_t *k8)
 {
     grid_dependency_wait();
     const int unit = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -41,19 +41,19 @@ __global__ void __launch_bounds__(256) quantize_keys_kernel(Shape s, const uint1
         float sc, n2;
         quantize_values<8, 16>(x, packed, sc, n2);  // every lane takes part (the shuffles span the warp)
         if (t < end) {
-            reinterpret_cast<uint2 *>(k8 + (row0 + t) * kHeadDim)[hl] = make_uint2(packed[0], packed[1]);
-            if (hl == 0)
-                *reinterpret_cast<float4 *>(kmeta + (row0 + t) * kQ8MetaFloats) = make_float4(sc, n2, 0.f, 0.f);
+            int8_t *rowp = k8 + (row0 + t) * kQ8RowBytes;
+            reinterpret_cast<uint2 *>(rowp)[hl] = make_uint2(packed[0], packed[1]);
+            if (hl == 0) *reinterpret_cast<float4 *>(rowp + kHeadDim) = make_float4(sc, n2, 0.f, 0.f);
         }
     }
 }
 
 cudaError_t launch_quantize_keys(const Shape &s, const uint16_t *kc, const int32_t *seq_lens, int tok0, int n_tokens,
-                                 int8_t *k8, float *kmeta, cudaStream_t st)
+                                 int8_t *k8, cudaStream_t st)
 {
     if (n_tokens == 0) return cudaSuccess;
     dim3 grid((n_tokens + kQuantRowsPerBlock - 1) / kQuantRowsPerBlock, s.B * s.Hkv);
-    return launch_pdl(quantize_keys_kernel, grid, dim3(256), 0, st, s, kc, seq_lens, tok0, n_tokens, k8, kmeta);
+    return launch_pdl(quantize_keys_kernel, grid, dim3(256), 0, st, s, kc, seq_lens, tok0, n_tokens, k8);
 }
 
 }  // namespace mp

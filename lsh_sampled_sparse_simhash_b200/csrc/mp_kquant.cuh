@@ -8,11 +8,12 @@
 // (at most 8 significant bits), so the keys the attention kernel effectively
 // uses can be written back as bf16 and checked against the fp64 oracle.
 //
-// Beside the int8 row goes a 16-byte record {s, |s q|^2, 0, 0} (fp32): the
-// gather fetches it with one 16-byte copy, and the stored squared norm saves
-// the attention kernel the K K^T products it would otherwise need for the
-// collision probability.  sum_j q_j^2 <= 128 * 127^2 < 2^24 is an exact fp32
-// integer and s^2 a power of two, so the stored norm is exact.
+// The int8 values are followed, in the same 144-byte row, by a 16-byte
+// record {s, |s q|^2, 0, 0} (fp32): the gather fetches row and record as one
+// contiguous piece, and the stored squared norm saves the attention kernel
+// the K K^T products it would otherwise need for the collision probability.
+// sum_j q_j^2 <= 128 * 127^2 < 2^24 is an exact fp32 integer and s^2 a power
+// of two, so the stored norm is exact.
 #pragma once
 
 #include <math.h>
@@ -21,7 +22,7 @@
 
 namespace mp {
 
-constexpr int kQ8MetaFloats = 4;  // {scale, squared norm, 0, 0} per key row
+constexpr int kQ8RowBytes = kHeadDim + 16;  // 128 int8 values, then the record
 
 // Quantises one row spread over W lanes (aligned groups of W lanes of the
 // warp; every lane of the warp calls this), each holding E consecutive values
@@ -59,16 +60,17 @@ __device__ __forceinline__ void quantize_values(const float (&x)[E], uint32_t (&
     norm2 = (float)sq * s * s;
 }
 
-// One warp quantises one row: lane l takes dims 4 l .. 4 l + 3.
-__device__ __forceinline__ void quantize_key_row(const uint16_t *k, int8_t *q8, float *meta, int lane)
+// One warp quantises one row into q8row (kQ8RowBytes): lane l takes dims
+// 4 l .. 4 l + 3.
+__device__ __forceinline__ void quantize_key_row(const uint16_t *k, int8_t *q8row, int lane)
 {
     const uint2 v = reinterpret_cast<const uint2 *>(k)[lane];
     const float x[4] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y)};
     uint32_t packed[1];
     float s, n2;
     quantize_values<4, 32>(x, packed, s, n2);
-    reinterpret_cast<uint32_t *>(q8)[lane] = packed[0];
-    if (lane == 0) *reinterpret_cast<float4 *>(meta) = make_float4(s, n2, 0.f, 0.f);
+    reinterpret_cast<uint32_t *>(q8row)[lane] = packed[0];
+    if (lane == 0) *reinterpret_cast<float4 *>(q8row + kHeadDim) = make_float4(s, n2, 0.f, 0.f);
 }
 
 }  // namespace mp

@@ -11,6 +11,8 @@ bf16 values becomes
     q_j = round-half-to-even(k_j / s)                             (int8, |q_j| <= 127)
     meta = {s, |s q|^2, 0, 0}                                     (fp32 x 4 per row)
 
+stored as one 144-byte row: the 128 int8 values, then the record.
+
 and the attention then runs on k~ = s q.  This module writes that definition
 out in fp64 numpy, one row at a time, so that a reader can check it by eye.
 """
@@ -61,6 +63,15 @@ def row_meta(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     meta[..., 1] = n2
     assert np.array_equal(meta[..., 1].astype(np.float64), n2), "squared norm not exact in fp32"
     return meta
+
+
+def pack_rows(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """The stored rows, int8 [..., 144]: q, then the record's 16 bytes."""
+    meta = row_meta(q, s)
+    out = np.zeros(np.shape(q)[:-1] + (144,), np.int8)
+    out[..., :128] = q
+    out[..., 128:] = meta.view(np.int8).reshape(np.shape(q)[:-1] + (16,))
+    return out
 
 
 def dequantize_bits(q: np.ndarray, s: np.ndarray) -> np.ndarray:

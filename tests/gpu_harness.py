@@ -103,13 +103,12 @@ class Run:
         return unpack_codes(a, self.w.k_bits, self.w.n_tables, n, self.shape.planes)
 
     def alloc_q8(self):
-        """int8 key copy and its row records, filled with a sentinel (0x55
-        bytes, records of -1) so that rows the library does not write stay
+        """int8 key rows (128 values + the 16-byte record), filled with a
+        sentinel (0x55 bytes) so that rows the library does not write stay
         recognisable."""
         w = self.w
-        self.k8 = torch.full((w.batch, w.n_kv_heads, w.capacity, w.head_dim), 0x55, dtype=torch.int8,
+        self.k8 = torch.full((w.batch, w.n_kv_heads, w.capacity, mp.Q8_ROW_BYTES), 0x55, dtype=torch.int8,
                              device="cuda")
-        self.kmeta = torch.full((w.batch, w.n_kv_heads, w.capacity, 4), -1.0, dtype=torch.float32, device="cuda")
 
     def decode(self, qcodes_in: Optional[np.ndarray] = None, member: bool = True, path: int = 0, q8: bool = False,
                skip_scan: bool = False):
@@ -119,7 +118,7 @@ class Run:
         qco = torch.zeros((w.batch, w.n_q_heads, w.n_tables), dtype=torch.int16, device="cuda")
         qci = dev(qcodes_in) if qcodes_in is not None else None
         if q8:
-            mp.decode_attend_q8(self.shape, self.q, self.W, self.codes, self.k8, self.kmeta, self.V, self.lens,
+            mp.decode_attend_q8(self.shape, self.q, self.W, self.codes, self.k8, self.V, self.lens,
                                 self.max_len, self.out, self.lse, self.ns, self.ws, qcodes_in=qci, qcodes_out=qco,
                                 member_out=mem, path=path)
         else:

@@ -151,31 +151,32 @@ def test_int8_key_entry_points_checked(lib):
     s = good_shape()
     A = 1 << 12
     q = lib.mp_quantize_keys
-    assert q(ctypes.byref(s), None, None, 0, 10, A, A, None) == mp.MP_ERR_ARG
-    assert q(ctypes.byref(s), A, None, 0, 10, A, None, None) == mp.MP_ERR_ARG
-    assert q(ctypes.byref(s), A, None, 0, 10, A + 8, A, None) == mp.MP_ERR_ALIGN
-    assert q(ctypes.byref(s), A, A + 2, 0, 10, A, A, None) == mp.MP_ERR_ALIGN
-    assert q(ctypes.byref(s), A, None, 1000, 25, A, A, None) == mp.MP_ERR_CAPACITY
-    assert q(ctypes.byref(s), A, None, -1, 10, A, A, None) == mp.MP_ERR_CAPACITY
-    assert q(ctypes.byref(s), A, None, 0, -1, A, A, None) == mp.MP_ERR_CAPACITY
+    assert q(ctypes.byref(s), None, None, 0, 10, A, None) == mp.MP_ERR_ARG
+    assert q(ctypes.byref(s), A, None, 0, 10, None, None) == mp.MP_ERR_ARG
+    assert q(ctypes.byref(s), A, None, 0, 10, A + 8, None) == mp.MP_ERR_ALIGN
+    assert q(ctypes.byref(s), A, A + 2, 0, 10, A, None) == mp.MP_ERR_ALIGN
+    assert q(ctypes.byref(s), A, None, 1000, 25, A, None) == mp.MP_ERR_CAPACITY
+    assert q(ctypes.byref(s), A, None, -1, 10, A, None) == mp.MP_ERR_CAPACITY
+    assert q(ctypes.byref(s), A, None, 0, -1, A, None) == mp.MP_ERR_CAPACITY
     ap = lib.mp_append_token_q8
-    assert ap(ctypes.byref(s), A, A, A, A, A, A, A, None, A, None, None) == mp.MP_ERR_ARG
-    assert ap(ctypes.byref(s), A, A, A, A + 2, A, A, A, A, A, None, None) == mp.MP_ERR_ALIGN  # k_cache may be NULL
-    assert ap(ctypes.byref(s), A, A, A, A, None, A, A, A, A, None, None) == mp.MP_ERR_ARG     # v_cache may not
-    assert ap(ctypes.byref(s), A, A, A, A, A, A, A, A, A + 4, None, None) == mp.MP_ERR_ALIGN
-    assert ap(ctypes.byref(s), A, A, A, A, A, A, A, A, A, A + 2, None) == mp.MP_ERR_ALIGN
+    assert ap(ctypes.byref(s), A, A, A, A, A, A, A, None, None, None) == mp.MP_ERR_ARG
+    assert ap(ctypes.byref(s), A, A, A, A, A, A, A, A + 4, None, None) == mp.MP_ERR_ALIGN
+    assert ap(ctypes.byref(s), A, A, A, A, A, A, A, A, A + 2, None) == mp.MP_ERR_ALIGN
+    assert ap(ctypes.byref(s), A, A, A, A + 2, A, A, A, A, None, None) == mp.MP_ERR_ALIGN  # k_cache may be NULL
+    assert ap(ctypes.byref(s), A, A, A, A, None, A, A, A, None, None) == mp.MP_ERR_ARG     # v_cache may not
     need = ctypes.c_size_t()
     assert lib.mp_decode_workspace_bytes(ctypes.byref(s), 1024, ctypes.byref(need)) == 0
     d = lib.mp_decode_attend_q8
-    assert d(ctypes.byref(s), A, A, A, None, A, A, A, 1024, A, A, A, A, need.value, None, None) == mp.MP_ERR_ARG
-    assert d(ctypes.byref(s), A, A, A, A, A + 4, A, A, 1024, A, A, A, A, need.value, None, None) == mp.MP_ERR_ALIGN
-    assert d(ctypes.byref(s), A, A, A, A, A, A, A, 1024, A, A, A, A, need.value - 1, None, None) \
-        == mp.MP_ERR_WORKSPACE
-    assert d(ctypes.byref(s), A, A, A, A, A, A, A, 1025, A, A, A, A, need.value, None, None) == mp.MP_ERR_CAPACITY
+    assert d(ctypes.byref(s), A, A, A, None, A, A, 1024, A, A, A, A, need.value, None, None) == mp.MP_ERR_ARG
+    assert d(ctypes.byref(s), A, A, A, A + 4, A, A, 1024, A, A, A, A, need.value, None, None) == mp.MP_ERR_ALIGN
+    assert d(ctypes.byref(s), A, A, A, A, A, A, 1024, A, A, A, A, need.value - 1, None, None) == mp.MP_ERR_WORKSPACE
+    assert d(ctypes.byref(s), A, A, A, A, A, A, 1025, A, A, A, A, need.value, None, None) == mp.MP_ERR_CAPACITY
     for path, want in [(mp.MP_PATH_FUSED, mp.MP_ERR_SHAPE), (mp.MP_PATH_TC, mp.MP_ERR_SHAPE), (4, mp.MP_ERR_ARG)]:
         dbg = B._CDebug(None, None, None, path)
-        assert d(ctypes.byref(s), A, A, A, A, A, A, A, 1024, A, A, A, A, need.value, ctypes.byref(dbg),
+        assert d(ctypes.byref(s), A, A, A, A, A, A, 1024, A, A, A, A, need.value, ctypes.byref(dbg),
                  None) == want, path
+    m = re.search(r"#define MP_Q8_ROW_BYTES (\d+)", open(HEADER).read())
+    assert m and int(m.group(1)) == B.Q8_ROW_BYTES == 144
 
 
 def test_auto_layout_threshold_matches_header():

@@ -68,13 +68,16 @@ def _units(w):
 
 
 def _check_q8_rows(run, inp, units_rows):
-    """Bit-exact int8 rows and row records for {(b, kh): row indices}."""
+    """Bit-exact 144-byte int8 rows (values and record) for {(b, kh): row indices}."""
     k8 = host(run.k8)
-    km = host(run.kmeta)
     for (b, kh), rows in units_rows.items():
         q, s = kquant.quantize_rows(inp["K"][b, kh, rows])
-        np.testing.assert_array_equal(k8[b, kh, rows], q, err_msg=f"int8 rows b={b} kh={kh}")
-        np.testing.assert_array_equal(km[b, kh, rows], kquant.row_meta(q, s), err_msg=f"records b={b} kh={kh}")
+        np.testing.assert_array_equal(k8[b, kh, rows], kquant.pack_rows(q, s), err_msg=f"int8 rows b={b} kh={kh}")
+
+
+def _meta(k8_rows):
+    """The fp32 records of stored rows [..., 144]."""
+    return np.ascontiguousarray(k8_rows[..., 128:]).view(np.float32)
 
 
 @pytest.mark.parametrize("case", ["tiny_g1_k8", "g4_k8_ragged_tail", "g8_k8_mu_offset"])
@@ -84,15 +87,15 @@ def test_quantize_keys_bit_exact_and_bounded_by_lengths(case):
     _plant_edge_rows(inp)
     run = Run(w, inp)
     run.alloc_q8()
-    mp.quantize_keys(run.shape, run.K, run.k8, run.kmeta, seq_lens=run.lens)
+    mp.quantize_keys(run.shape, run.K, run.k8, seq_lens=run.lens)
     torch.cuda.synchronize()
     lens = inp["seq_lens"]
     _check_q8_rows(run, inp, {(b, kh): np.arange(int(lens[b])) for b, kh in _units(w)})
     k8 = host(run.k8)
-    km = host(run.kmeta)
+    km = _meta(k8)
     for b, kh in _units(w):
         n = int(lens[b])
-        assert (k8[b, kh, n:] == 0x55).all() and (km[b, kh, n:] == -1.0).all(), "rows past the length written"
+        assert (k8[b, kh, n:] == 0x55).all(), "rows past the length written"
     assert list(km[0, 0, 5]) == [0.0, 0.0, 0.0, 0.0] and not k8[0, 0, 5].any()
     assert list(km[0, 0, 6]) == [1.0, 127.0 ** 2 + 1.0, 0.0, 0.0] and list(k8[0, 0, 6, :3]) == [127, -1, 0]
     assert list(km[0, 0, 7]) == [2.0, 4.0 * (64 ** 2 + 2 ** 2 + 2 ** 2), 0.0, 0.0]
@@ -107,7 +110,7 @@ def test_quantize_keys_token_range():
     run = Run(w, inp)
     run.alloc_q8()
     t0, n = 1000, 777
-    mp.quantize_keys(run.shape, run.K, run.k8, run.kmeta, first_token=t0, n_tokens=n)
+    mp.quantize_keys(run.shape, run.K, run.k8, first_token=t0, n_tokens=n)
     torch.cuda.synchronize()
     _check_q8_rows(run, inp, {u: np.arange(t0, t0 + n) for u in _units(w)})
     k8 = host(run.k8)
@@ -117,7 +120,7 @@ def test_quantize_keys_token_range():
 def _q8_run(w, inp):
     run = Run(w, inp)
     run.alloc_q8()
-    mp.quantize_keys(run.shape, run.K, run.k8, run.kmeta, seq_lens=run.lens)
+    mp.quantize_keys(run.shape, run.K, run.k8, seq_lens=run.lens)
     return run
 
 
@@ -184,7 +187,7 @@ def test_append_q8_writes_the_int8_row():
         plain.hash_keys(w.context)
         status = torch.zeros(2, dtype=torch.int32, device="cuda")
         mp.append_token_q8(run.shape, run.k_new, run.v_new, run.W, run.K, run.V, run.codes, run.lens, run.k8,
-                           run.kmeta, status[:1])
+                           status[:1])
         mp.append_token(plain.shape, plain.k_new, plain.v_new, plain.W, plain.K, plain.V, plain.codes, plain.lens,
                         status[1:])
         torch.cuda.synchronize()
@@ -193,10 +196,8 @@ def test_append_q8_writes_the_int8_row():
             assert torch.equal(a, c)
         pos = w.context
         k8 = host(run.k8)
-        km = host(run.kmeta)
         q, s = kquant.quantize_rows(inp["k_new"])
-        np.testing.assert_array_equal(k8[:, :, pos], q)
-        np.testing.assert_array_equal(km[:, :, pos], kquant.row_meta(q, s))
+        np.testing.assert_array_equal(k8[:, :, pos], kquant.pack_rows(q, s))
         assert (k8[:, :, pos + 1:] == 0x55).all()
 
 
@@ -212,12 +213,10 @@ def test_append_q8_without_a_bf16_key_cache():
     run.alloc_decode(w.context + 1)
     alt.alloc_decode(w.context + 1)
     K_before = alt.K.clone()
-    mp.append_token_q8(run.shape, run.k_new, run.v_new, run.W, run.K, run.V, run.codes, run.lens, run.k8,
-                       run.kmeta)
-    mp.append_token_q8(alt.shape, alt.k_new, alt.v_new, alt.W, None, alt.V, alt.codes, alt.lens, alt.k8, alt.kmeta)
+    mp.append_token_q8(run.shape, run.k_new, run.v_new, run.W, run.K, run.V, run.codes, run.lens, run.k8)
+    mp.append_token_q8(alt.shape, alt.k_new, alt.v_new, alt.W, None, alt.V, alt.codes, alt.lens, alt.k8)
     torch.cuda.synchronize()
-    for a, c in ((run.V, alt.V), (run.codes, alt.codes), (run.lens, alt.lens), (run.k8, alt.k8),
-                 (run.kmeta, alt.kmeta)):
+    for a, c in ((run.V, alt.V), (run.codes, alt.codes), (run.lens, alt.lens), (run.k8, alt.k8)):
         assert torch.equal(a, c)
     assert torch.equal(alt.K, K_before)
     g1 = run.decode(q8=True)
@@ -239,9 +238,8 @@ def test_full_size_q8_ragged16():
     run.alloc_q8()
     run.alloc_decode(run.max_len + 1)
     run.hash_keys(run.max_len)
-    mp.quantize_keys(run.shape, run.K, run.k8, run.kmeta, seq_lens=run.lens)
-    mp.append_token_q8(run.shape, run.k_new, run.v_new, run.W, run.K, run.V, run.codes, run.lens, run.k8,
-                       run.kmeta)
+    mp.quantize_keys(run.shape, run.K, run.k8, seq_lens=run.lens)
+    mp.append_token_q8(run.shape, run.k_new, run.v_new, run.W, run.K, run.V, run.codes, run.lens, run.k8)
     torch.cuda.synchronize()
     new_lens = host(run.lens)
     assert (new_lens == inp["seq_lens"] + 1).all()

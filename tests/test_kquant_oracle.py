@@ -79,6 +79,10 @@ def test_row_record_holds_scale_and_exact_squared_norm():
     kt = bf16_bits_to_f32(kquant.dequantize_bits(q, s)).astype(np.float64)
     np.testing.assert_array_equal(meta[:, 1].astype(np.float64), np.sum(kt * kt, axis=1))
     assert meta[3, 1] == 0.0 and not meta[:, 2:].any()
+    rows = kquant.pack_rows(q, s)
+    assert rows.shape == (16, 144) and rows.dtype == np.int8
+    np.testing.assert_array_equal(rows[:, :128], q)
+    np.testing.assert_array_equal(rows[:, 128:].copy().view(np.float32), meta)
 
 
 def test_dequantized_keys_are_bf16_and_a_fixed_point():
