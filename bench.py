@@ -75,7 +75,10 @@ def parse(argv=None):
     p.add_argument("--decode-path", default="auto", choices=["auto", "split", "fused", "tc"],
                    help="decode kernels: auto, split (scan then attention), fused (one kernel; bit planes) or tc "
                         "(scan then the tcgen05 attention kernel)")
-    return p.parse_args(argv)
+    args = p.parse_args(argv)
+    if args.k_format == "int8" and args.decode_path in ("fused", "tc"):
+        p.error("--k-format int8 runs on the split path only (--decode-path auto or split)")
+    return args
 
 
 def load_peaks():

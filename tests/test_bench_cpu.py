@@ -6,6 +6,7 @@ import json
 import os
 
 import numpy as np
+import pytest
 
 import bench
 
@@ -113,3 +114,11 @@ def test_oracle_sample_units_spread_over_the_batch():
     smp = bench.OracleSample(w)
     assert smp.units == [(0, 0), (4, 1), (8, 2), (12, 3)]
     assert "(N_b + 1) / 8" in smp.describe()
+
+
+def test_int8_keys_only_on_the_split_path():
+    assert bench.parse(["--k-format", "int8"]).k_format == "int8"
+    assert bench.parse(["--k-format", "int8", "--decode-path", "split"]).decode_path == "split"
+    for path in ("fused", "tc"):
+        with pytest.raises(SystemExit):
+            bench.parse(["--k-format", "int8", "--decode-path", path])
