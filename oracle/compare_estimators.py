@@ -8,6 +8,8 @@ tokens |S_h| that MagicPIG's LSH test selects for that head:
 
   magicpig        fp64 oracle of the method (SimHash codes, >= 2-of-L
                   collisions, weights exp(s - log u), exact set D)
+  magicpig_int8   the same on the int8 keys s q of the library's opt-in
+                  reduced-precision gather (oracle/kquant.py; same codes)
   topk            D plus the |S_h| highest-scored tokens, renormalised
   oracle_sampling D plus |S_h| i.i.d. draws from the exact softmax
 
@@ -24,7 +26,7 @@ import json
 
 import numpy as np
 
-from oracle import attend, build, collide, simhash
+from oracle import attend, build, collide, kquant, simhash
 from oracle.estimators import exact_attention, oracle_sampling, rel_l2, scores, topk_attention, exact_set
 
 
@@ -43,6 +45,8 @@ def compare_unit(w, q_bits, W_bits, b: int, kvh: int, n: int, rng: np.random.Gen
     qcodes = simhash(qh, W_bits, w.k_bits, w.n_tables)
     member, nsamp = collide(kcodes, qcodes, w.sink, w.window)
     K, V = _f64(Kb), _f64(Vb)
+    q8, s8 = kquant.quantize_rows(Kb)
+    Kt = kquant.dequantize_bits(q8, s8)
     needles = planted_positions(w, b, kvh, n)
     d = exact_set(n, w.sink, w.window)
     rows = []
@@ -50,6 +54,7 @@ def compare_unit(w, q_bits, W_bits, b: int, kvh: int, n: int, rng: np.random.Gen
         q = _f64(qh[g])
         ref = exact_attention(q, K, V)
         mp_out, _ = attend(qh[g], Kb, Vb, member[g], w.sink, w.window, w.k_bits, w.n_tables)
+        mp8_out, _ = attend(qh[g], Kt, Vb, member[g], w.sink, w.window, w.k_bits, w.n_tables)
         k = int(nsamp[g])
         tk = topk_attention(q, K, V, k, w.sink, w.window)
         osamp = [rel_l2(oracle_sampling(q, K, V, k, w.sink, w.window, rng), ref) for _ in range(draws)]
@@ -59,7 +64,8 @@ def compare_unit(w, q_bits, W_bits, b: int, kvh: int, n: int, rng: np.random.Gen
         nd = needles[~d[needles]] if len(needles) else needles
         rows.append(dict(
             budget=k, n=n,
-            magicpig=rel_l2(mp_out, ref), topk=rel_l2(tk, ref), oracle_sampling=float(np.mean(osamp)),
+            magicpig=rel_l2(mp_out, ref), magicpig_int8=rel_l2(mp8_out, ref), topk=rel_l2(tk, ref),
+            oracle_sampling=float(np.mean(osamp)),
             recall_magicpig=float(member[g][nd].mean()) if len(nd) else float("nan"),
             recall_topk=float(np.mean([t in top for t in nd])) if len(nd) else float("nan")))
     return rows
@@ -87,7 +93,7 @@ def compare(name: str, units: int, seed: int = 0, **overrides):
 
 def summary(rows):
     out = {}
-    for m in ("magicpig", "topk", "oracle_sampling"):
+    for m in ("magicpig", "magicpig_int8", "topk", "oracle_sampling"):
         v = np.array([r[m] for r in rows])
         out[m] = dict(mean_rel_l2=float(v.mean()), max_rel_l2=float(v.max()))
     out["budget_fraction"] = float(np.mean([r["budget"] / r["n"] for r in rows]))
