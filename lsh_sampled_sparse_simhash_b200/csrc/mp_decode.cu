@@ -18,6 +18,9 @@
 //           extra split per (b, kv head) handles D exactly (weight exp(s)).
 //   merge   log-sum-exp merge of the per-split partials into out / lse, plus
 //           n_sampled.
+// The scan releases each chunk's candidate list with a ready flag, and the
+// attention, launched as soon as every scan block is running, starts on a
+// chunk once its flag is set instead of waiting for the whole scan.
 // With bit planes the scan and the attention can instead run as one kernel,
 // fused_planes_kernel (opt-in, MP_PATH_FUSED).
 #include <math.h>
